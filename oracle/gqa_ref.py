@@ -1,0 +1,229 @@
+"""Float64 CPU oracle for the fused-QKV projection and grouped-query attention.
+
+TEST INFRASTRUCTURE.  Only the test suite, the package's smoke check and the
+benchmark's CPU-baseline leg may import this module.  It shares no code with
+the CUDA library: it computes the plain definition of each step, in float64,
+with no tiling, no online softmax and no split of the key axis.
+
+Sources (page title, then section):
+
+* "Optimize LlamaAttention by fusing QKV projections" (huggingface/transformers
+  pull request #40092), the diff of ``LlamaAttention.forward``: one
+  ``qkv_proj`` linear layer replaces ``q_proj``/``k_proj``/``v_proj``; its
+  output is sliced into query ``[:nh*hd]``, key ``[nh*hd : nh*hd + nkv*hd]``
+  and value ``[nh*hd + nkv*hd :]`` features; the review thread notes that
+  ``repeat_kv`` later materialises the KV heads for every query head.
+* "MHA -> GQA: 提升 LLM 推理效率", section 3.2 (GQA Attention 计算): g query heads
+  share one KV head; MHA and MQA are the cases n_kv_heads = n_heads and 1.
+* "FlashAttention-3" (together.ai summary), section "FlashAttention方式のおさらい":
+  the tiled online-softmax algorithm is exact, so its result equals the plain
+  softmax(QK^T)V computed here.
+* custom-op overhead gist (``overhead.py``): ``forward(positions,
+  hidden_states)`` applies a position-dependent step to q and k only, after
+  the fused projection.
+
+Readings where the pages are silent (each restated in the design notes):
+
+* RoPE is the Llama "rotate_half" form: feature i pairs with i + hd/2,
+  inv_freq_i = theta^(-2i/hd), x'_i = x_i cos - x_{i+hd/2} sin,
+  x'_{i+hd/2} = x_{i+hd/2} cos + x_i sin, angle = position * inv_freq_i.
+* softmax scale is 1/sqrt(head_dim).
+* query head h reads KV head h // g (contiguous groups, ``repeat_kv``).
+* key t is visible to a query at position p iff t < kv_len and, when causal,
+  t <= p.  Default query positions are kv_len - S + s (bottom-right aligned).
+* a query with no visible key gets an all-zero output row.
+* the K/V cache slot of a token is its absolute position.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "fused_projection", "split_qkv", "rope_inv_freq", "apply_rope",
+    "qkv_rope_project", "kv_head_of", "softmax", "attend_row",
+    "prefill_attention", "decode_attention", "default_q_positions",
+]
+
+
+# --------------------------------------------------------------------------
+# a1: fused projection; a2 split (pull request #40092, LlamaAttention.forward)
+# --------------------------------------------------------------------------
+def fused_projection(x: np.ndarray, w_qkv: np.ndarray) -> np.ndarray:
+    """Y = X W^T for an ``nn.Linear`` weight stored ``[out_features, in_features]``
+    with no bias.  ``x`` is ``[..., hidden]``; returns ``[..., N_qkv]``."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_qkv, dtype=np.float64)
+    return x @ w.T
+
+
+def split_qkv(y: np.ndarray, n_heads: int, n_kv_heads: int, head_dim: int):
+    """Slice the fused output into per-head query/key/value features.
+
+    ``y`` is ``[B, S, N_qkv]``; returns q ``[B, S, nh, hd]``, k and v
+    ``[B, S, nkv, hd]``.  Within each block, head j owns features
+    ``j*hd .. (j+1)*hd - 1``."""
+    B, S, N = y.shape
+    qn, kn = n_heads * head_dim, n_kv_heads * head_dim
+    if N != qn + 2 * kn:
+        raise ValueError("fused width does not match (n_heads + 2 n_kv_heads) * head_dim")
+    q = y[..., :qn].reshape(B, S, n_heads, head_dim)
+    k = y[..., qn:qn + kn].reshape(B, S, n_kv_heads, head_dim)
+    v = y[..., qn + kn:].reshape(B, S, n_kv_heads, head_dim)
+    return q, k, v
+
+
+# --------------------------------------------------------------------------
+# a2: rotary position embedding (rotate_half pairing; theta from the workload)
+# --------------------------------------------------------------------------
+def rope_inv_freq(head_dim: int, theta: float) -> np.ndarray:
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    return np.power(np.float64(theta), -2.0 * i / head_dim)
+
+
+def apply_rope(t: np.ndarray, positions: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate ``t`` ``[B, S, H, hd]`` by the angle of each token's position
+    ``positions`` ``[B, S]``; pairs are (i, i + hd/2)."""
+    t = np.asarray(t, dtype=np.float64)
+    hd = t.shape[-1]
+    half = hd // 2
+    ang = np.asarray(positions, dtype=np.float64)[..., None] * rope_inv_freq(hd, theta)  # [B,S,half]
+    c = np.cos(ang)[:, :, None, :]
+    s = np.sin(ang)[:, :, None, :]
+    lo, hi = t[..., :half], t[..., half:]
+    return np.concatenate([lo * c - hi * s, hi * c + lo * s], axis=-1)
+
+
+def qkv_rope_project(x, w_qkv, positions, n_heads, n_kv_heads, head_dim, theta,
+                     k_cache, v_cache):
+    """Steps a1-a3: fused projection, RoPE on q and k, scatter.
+
+    Returns ``q`` head-major ``[B, nh, S, hd]`` and copies of the caches
+    ``[B, nkv, cap, hd]`` with token s of sequence b written at slot
+    ``positions[b, s]``; every other slot keeps its previous value.  Tokens
+    whose position lies outside ``[0, cap)`` are not written."""
+    y = fused_projection(x, w_qkv)
+    q, k, v = split_qkv(y, n_heads, n_kv_heads, head_dim)
+    q = apply_rope(q, positions, theta)
+    k = apply_rope(k, positions, theta)
+    kc = np.array(k_cache, dtype=np.float64, copy=True)
+    vc = np.array(v_cache, dtype=np.float64, copy=True)
+    B, S = positions.shape
+    cap = kc.shape[2]
+    for b in range(B):
+        for s in range(S):
+            p = int(positions[b, s])
+            if 0 <= p < cap:
+                kc[b, :, p, :] = k[b, s]
+                vc[b, :, p, :] = v[b, s]
+    return np.ascontiguousarray(q.transpose(0, 2, 1, 3)), kc, vc
+
+
+# --------------------------------------------------------------------------
+# a4-a6: attention (MHA -> GQA blog, section 3.2; FlashAttention recap)
+# --------------------------------------------------------------------------
+def kv_head_of(h: int, n_heads: int, n_kv_heads: int) -> int:
+    """KV head read by query head h: groups of g = nh/nkv consecutive heads."""
+    return h // (n_heads // n_kv_heads)
+
+
+def softmax(scores: np.ndarray) -> np.ndarray:
+    """Row softmax with max subtraction; a row of all -inf gives all zeros."""
+    s = np.asarray(scores, dtype=np.float64)
+    m = np.max(s, axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    e = np.exp(s - m)
+    z = np.sum(e, axis=-1, keepdims=True)
+    return np.divide(e, z, out=np.zeros_like(e), where=z > 0)
+
+
+def attend_row(q_vec, keys, values, n_visible=None):
+    """Plain attention of one query vector over ``keys``/``values`` ``[L, hd]``,
+    restricted to the first ``n_visible`` rows; returns (output, probs)."""
+    hd = keys.shape[-1]
+    L = keys.shape[0] if n_visible is None else int(n_visible)
+    if L <= 0:
+        return np.zeros(hd), np.zeros(0)
+    s = keys[:L] @ np.asarray(q_vec, dtype=np.float64) / np.sqrt(hd)
+    p = softmax(s[None, :])[0]
+    return p @ values[:L], p
+
+
+def default_q_positions(kv_lens: np.ndarray, S: int) -> np.ndarray:
+    """Bottom-right-aligned positions kv_len - S + s."""
+    return (np.asarray(kv_lens, dtype=np.int64)[:, None] - S + np.arange(S)[None, :])
+
+
+def prefill_attention(q, k_cache, v_cache, kv_lens, causal, q_positions=None,
+                      rows=None, chunk=1024):
+    """Exact attention for every query row (or the ``rows`` subset).
+
+    q ``[B, nh, S, hd]``; caches ``[B, nkv, cap, hd]``; kv_lens ``[B]``.
+    Returns O ``[B, S, nh, hd]`` (when ``rows`` is a list of (b, h, s) triples,
+    an array ``[len(rows), hd]`` instead)."""
+    q = np.asarray(q, dtype=np.float64)
+    kc = np.asarray(k_cache, dtype=np.float64)
+    vc = np.asarray(v_cache, dtype=np.float64)
+    B, nh, S, hd = q.shape
+    nkv = kc.shape[1]
+    kv_lens = np.asarray(kv_lens, dtype=np.int64)
+    pos = default_q_positions(kv_lens, S) if q_positions is None else np.asarray(q_positions, dtype=np.int64)
+    scale = 1.0 / np.sqrt(hd)
+
+    def visible_mask(b, s_idx):
+        L = int(kv_lens[b])
+        t = np.arange(L)[None, :]
+        vis = np.ones((len(s_idx), L), dtype=bool)
+        if causal:
+            vis &= t <= pos[b, s_idx][:, None]
+        return vis, L
+
+    if rows is not None:
+        out = np.zeros((len(rows), hd))
+        for i, (b, h, s) in enumerate(rows):
+            j = kv_head_of(h, nh, nkv)
+            vis, L = visible_mask(b, np.array([s]))
+            if L <= 0:
+                continue
+            sc = (kc[b, j, :L] @ q[b, h, s]) * scale
+            sc = np.where(vis[0], sc, -np.inf)
+            p = softmax(sc[None, :])[0]
+            out[i] = p @ vc[b, j, :L]
+        return out
+
+    out = np.zeros((B, S, nh, hd))
+    for b in range(B):
+        for h in range(nh):
+            j = kv_head_of(h, nh, nkv)
+            L = int(kv_lens[b])
+            if L <= 0:
+                continue
+            K, V = kc[b, j, :L], vc[b, j, :L]
+            for s0 in range(0, S, chunk):
+                s_idx = np.arange(s0, min(S, s0 + chunk))
+                vis, _ = visible_mask(b, s_idx)
+                sc = (q[b, h, s_idx] @ K.T) * scale
+                sc = np.where(vis, sc, -np.inf)
+                out[b, s_idx, h] = softmax(sc) @ V
+    return out
+
+
+def decode_attention(q, k_cache, v_cache, kv_lens, pairs=None):
+    """One new query per sequence over its cached keys ``[0, kv_len)``.
+
+    q ``[B, nh, hd]``; returns O ``[B, nh, hd]`` (or ``[len(pairs), hd]`` for a
+    list of (b, h) pairs).  The split-KV partials and their log-sum-exp merge
+    on the GPU reach this same value, because the merge is exact."""
+    q = np.asarray(q, dtype=np.float64)
+    B, nh, hd = q.shape
+    nkv = k_cache.shape[1]
+    todo = pairs if pairs is not None else [(b, h) for b in range(B) for h in range(nh)]
+    out = np.zeros((len(todo), hd))
+    for i, (b, h) in enumerate(todo):
+        j = kv_head_of(h, nh, nkv)
+        L = int(kv_lens[b])
+        K = np.asarray(k_cache[b, j, :max(L, 0)], dtype=np.float64)
+        V = np.asarray(v_cache[b, j, :max(L, 0)], dtype=np.float64)
+        out[i], _ = attend_row(q[b, h], K, V)
+    if pairs is None:
+        return out.reshape(B, nh, hd)
+    return out

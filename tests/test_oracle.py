@@ -1,0 +1,525 @@
+"""Pins for the float64 oracle (CPU only).
+
+Nothing here compares the oracle with itself.  Each check ties it to
+something the pages or the mathematics fix: the fused-weight slicing printed
+in the fused-QKV pull request, the "fused = three separate projections"
+equivalence argued there, MHA/MQA as the n_kv_heads extremes of GQA (MHA -> GQA
+blog, section 3.2), the exactness of the tiled softmax (FlashAttention-3
+summary, recap section) through closed forms and invariants, and literal
+brute-force loops on tiny shapes.  The last block plants plausible mistakes in
+the oracle and shows that a pin fails for each.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import gqa_ref as ref
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# --------------------------------------------------------------------------
+# literal loops (brute force), written independently of the oracle's numpy
+# --------------------------------------------------------------------------
+def brute_projection(x, w):
+    B, S, D = x.shape
+    N = w.shape[0]
+    y = np.zeros((B, S, N))
+    for b in range(B):
+        for s in range(S):
+            for o in range(N):
+                acc = 0.0
+                for d in range(D):
+                    acc += float(x[b, s, d]) * float(w[o, d])
+                y[b, s, o] = acc
+    return y
+
+
+def brute_attention_row(qv, K, V, visible):
+    hd = len(qv)
+    scores = []
+    for t in range(len(K)):
+        if visible[t]:
+            dot = 0.0
+            for d in range(hd):
+                dot += qv[d] * K[t][d]
+            scores.append((t, dot / math.sqrt(hd)))
+    if not scores:
+        return [0.0] * hd
+    m = max(s for _, s in scores)
+    w = [(t, math.exp(s - m)) for t, s in scores]
+    z = sum(e for _, e in w)
+    out = [0.0] * hd
+    for t, e in w:
+        for d in range(hd):
+            out[d] += e / z * V[t][d]
+    return out
+
+
+# --------------------------------------------------------------------------
+# a1 / a2-split
+# --------------------------------------------------------------------------
+def check_split_matches_page():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "fused_qkv_slices.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert len(rows) >= 8
+    for r in rows:
+        nh, nkv, hd, qlo, qhi, klo, khi, vlo, vhi, N = map(int, r)
+        y = np.arange(N, dtype=np.float64)[None, None, :]
+        q, k, v = ref.split_qkv(y, nh, nkv, hd)
+        assert q.shape == (1, 1, nh, hd) and k.shape == (1, 1, nkv, hd) and v.shape == (1, 1, nkv, hd)
+        assert q[0, 0, 0, 0] == qlo and q[0, 0, -1, -1] == qhi - 1
+        assert k[0, 0, 0, 0] == klo and k[0, 0, -1, -1] == khi - 1
+        assert v[0, 0, 0, 0] == vlo and v[0, 0, -1, -1] == vhi - 1
+        # head j owns features j*hd .. (j+1)*hd-1 inside each block
+        for j in range(nkv):
+            assert k[0, 0, j, 0] == klo + j * hd
+
+
+def test_split_matches_page_slices():
+    check_split_matches_page()
+
+
+def check_fused_equals_separate():
+    r = rng(1)
+    B, S, D, nh, nkv, hd = 2, 5, 12, 4, 2, 4
+    wq = r.standard_normal((nh * hd, D))
+    wk = r.standard_normal((nkv * hd, D))
+    wv = r.standard_normal((nkv * hd, D))
+    x = r.standard_normal((B, S, D))
+    w_qkv = np.concatenate([wq, wk, wv], axis=0)          # the pull request's layout
+    q, k, v = ref.split_qkv(ref.fused_projection(x, w_qkv), nh, nkv, hd)
+    qs = np.einsum("bsd,od->bso", x, wq).reshape(B, S, nh, hd)
+    ks = np.einsum("bsd,od->bso", x, wk).reshape(B, S, nkv, hd)
+    vs = np.einsum("bsd,od->bso", x, wv).reshape(B, S, nkv, hd)
+    np.testing.assert_allclose(q, qs, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(k, ks, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(v, vs, rtol=0, atol=1e-12)
+
+
+def test_fused_equals_separate_projections():
+    check_fused_equals_separate()
+
+
+def test_projection_brute_force():
+    r = rng(2)
+    x = r.standard_normal((2, 3, 7))
+    w = r.standard_normal((9, 7))
+    np.testing.assert_allclose(ref.fused_projection(x, w), brute_projection(x, w), rtol=0, atol=1e-12)
+
+
+def test_projection_exact_on_integers():
+    # one-hot rows pick weight columns exactly
+    D, N = 6, 8
+    w = np.arange(N * D, dtype=np.float64).reshape(N, D) - 20
+    x = np.eye(D)[None]
+    np.testing.assert_array_equal(ref.fused_projection(x, w)[0], w.T)
+
+
+# --------------------------------------------------------------------------
+# a2 RoPE
+# --------------------------------------------------------------------------
+def test_rope_position_zero_is_identity():
+    t = rng(3).standard_normal((2, 4, 3, 16))
+    out = ref.apply_rope(t, np.zeros((2, 4), dtype=np.int64), 10000.0)
+    np.testing.assert_array_equal(out, t)
+
+
+def test_rope_preserves_pair_norms():
+    t = rng(4).standard_normal((1, 5, 2, 8))
+    pos = np.array([[0, 3, 17, 255, 8191]])
+    out = ref.apply_rope(t, pos, 10000.0)
+    n_in = t[..., :4] ** 2 + t[..., 4:] ** 2
+    n_out = out[..., :4] ** 2 + out[..., 4:] ** 2
+    np.testing.assert_allclose(n_out, n_in, rtol=1e-12)
+
+
+def check_rope_hand_example():
+    # hd = 4, theta = 10000: inv_freq = (10000^0, 10000^(-2/4)) = (1, 0.01).
+    # Pairs are (0, 2) and (1, 3).  For x = (1, 2, 3, 4):
+    #   position 1: pair (0,2) turns by 1 rad, pair (1,3) by 0.01 rad
+    #   position 2: by 2 rad and 0.02 rad
+    x = np.array([1.0, 2.0, 3.0, 4.0])
+    for p, (a0, a1) in ((1, (1.0, 0.01)), (2, (2.0, 0.02))):
+        want = np.array([
+            1 * math.cos(a0) - 3 * math.sin(a0),
+            2 * math.cos(a1) - 4 * math.sin(a1),
+            3 * math.cos(a0) + 1 * math.sin(a0),
+            4 * math.cos(a1) + 2 * math.sin(a1),
+        ])
+        got = ref.apply_rope(x[None, None, None, :], np.array([[p]]), 10000.0)[0, 0, 0]
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-14)
+
+
+def test_rope_hand_example():
+    check_rope_hand_example()
+
+
+def test_rope_pairing_plane_and_angle():
+    # A vector with only feature i set stays in span{e_i, e_(i+hd/2)} and turns
+    # by position * theta^(-2i/hd).
+    hd, theta = 16, 10000.0
+    for i in range(hd // 2):
+        e = np.zeros(hd)
+        e[i] = 1.0
+        out = ref.apply_rope(e[None, None, None], np.array([[5]]), theta)[0, 0, 0]
+        others = np.delete(out, [i, i + hd // 2])
+        assert np.all(others == 0.0)
+        ang = math.atan2(out[i + hd // 2], out[i])
+        want = 5 * theta ** (-2 * i / hd)
+        want = math.atan2(math.sin(want), math.cos(want))
+        assert abs(ang - want) < 1e-12
+
+
+def test_rope_relative_position_property():
+    # q(p+c) . k(p'+c) == q(p) . k(p') for every shift c
+    r = rng(5)
+    q = r.standard_normal((1, 1, 1, 32))
+    k = r.standard_normal((1, 1, 1, 32))
+    base = None
+    for c in (0, 1, 7, 100, 4000):
+        qq = ref.apply_rope(q, np.array([[12 + c]]), 10000.0)
+        kk = ref.apply_rope(k, np.array([[3 + c]]), 10000.0)
+        d = float(np.sum(qq * kk))
+        base = d if base is None else base
+        assert abs(d - base) < 1e-9
+
+
+def test_rope_composes():
+    t = rng(6).standard_normal((1, 1, 1, 8))
+    a = ref.apply_rope(ref.apply_rope(t, np.array([[3]]), 500.0), np.array([[4]]), 500.0)
+    b = ref.apply_rope(t, np.array([[7]]), 500.0)
+    np.testing.assert_allclose(a, b, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# a3 scatter into the head-major cache
+# --------------------------------------------------------------------------
+def test_scatter_slots_and_sentinels():
+    B, S, D, nh, nkv, hd, cap = 2, 3, 8, 4, 2, 4, 10
+    w = (np.arange((nh + 2 * nkv) * hd * D).reshape(-1, D) % 7) - 3.0
+    x = np.zeros((B, S, D))
+    for b in range(B):
+        for s in range(S):
+            x[b, s, (b * S + s) % D] = 1.0
+    pos = np.array([[0, 4, 9], [2, 3, 12]])        # 12 >= cap: not written
+    sentinel = -12345.0
+    kc0 = np.full((B, nkv, cap, hd), sentinel)
+    vc0 = np.full((B, nkv, cap, hd), sentinel)
+    q, kc, vc = ref.qkv_rope_project(x, w, pos, nh, nkv, hd, 10000.0, kc0, vc0)
+    assert q.shape == (B, nh, S, hd)
+    written = {(b, int(p)) for b in range(B) for p in pos[b] if p < cap}
+    for b in range(B):
+        for slot in range(cap):
+            if (b, slot) not in written:
+                assert np.all(kc[b, :, slot] == sentinel) and np.all(vc[b, :, slot] == sentinel)
+    # V has no rotation: exact copy of the projected integers at slot = position
+    for b in range(B):
+        for s in range(S):
+            p = int(pos[b, s])
+            if p >= cap:
+                continue
+            col = (b * S + s) % D
+            v_feat = w[(nh + nkv) * hd:, col].reshape(nkv, hd)
+            np.testing.assert_array_equal(vc[b, :, p], v_feat)
+            if p == 0:  # rotation by zero: K and Q exact too
+                np.testing.assert_array_equal(kc[b, :, p], w[nh * hd:(nh + nkv) * hd, col].reshape(nkv, hd))
+                np.testing.assert_array_equal(q[b, :, s], w[:nh * hd, col].reshape(nh, hd))
+
+
+# --------------------------------------------------------------------------
+# a4-a6 attention
+# --------------------------------------------------------------------------
+def _rand_attn(r, B, nh, nkv, S, L, hd, cap=None):
+    cap = cap or L
+    q = r.standard_normal((B, nh, S, hd))
+    kc = r.standard_normal((B, nkv, cap, hd))
+    vc = r.standard_normal((B, nkv, cap, hd))
+    return q, kc, vc
+
+
+def test_softmax_rows_sum_to_one():
+    s = rng(7).standard_normal((50, 33)) * 30
+    p = ref.softmax(s)
+    assert np.all(p >= 0)
+    np.testing.assert_allclose(p.sum(-1), 1.0, atol=1e-13)
+    # invariance to a constant shift per row
+    np.testing.assert_allclose(ref.softmax(s + 1e3), p, atol=1e-13)
+
+
+def check_closed_form_two_keys():
+    # hd = 4: q = (2,0,0,0), k0 = (1,0,0,0), k1 = 0 -> scores (2/sqrt(4), 0) = (1, 0)
+    # so p0 = e/(1+e), p1 = 1/(1+e) and O = p0 v0 + p1 v1.
+    q = np.array([2.0, 0, 0, 0])
+    K = np.array([[1.0, 0, 0, 0], [0, 0, 0, 0]])
+    V = np.array([[1.0, 2, 3, 4], [-1.0, 0, 5, 1]])
+    p0 = math.e / (1 + math.e)
+    want = p0 * V[0] + (1 - p0) * V[1]
+    out, p = ref.attend_row(q, K, V)
+    np.testing.assert_allclose(p, [p0, 1 - p0], atol=1e-15)
+    np.testing.assert_allclose(out, want, atol=1e-15)
+    # the same through the batched prefill / decode entry points
+    qq = q.reshape(1, 1, 1, 4)
+    kc, vc = K.reshape(1, 1, 2, 4), V.reshape(1, 1, 2, 4)
+    o = ref.prefill_attention(qq, kc, vc, np.array([2]), causal=False)
+    np.testing.assert_allclose(o[0, 0, 0], want, atol=1e-15)
+    o = ref.decode_attention(qq[:, :, 0], kc, vc, np.array([2]))
+    np.testing.assert_allclose(o[0, 0], want, atol=1e-15)
+
+
+def test_closed_form_two_keys():
+    check_closed_form_two_keys()
+
+
+def test_identical_keys_give_mean_of_visible_values():
+    r = rng(8)
+    B, nh, nkv, S, hd = 2, 4, 2, 6, 8
+    q = r.standard_normal((B, nh, S, hd))
+    k_row = r.standard_normal(hd)
+    kc = np.broadcast_to(k_row, (B, nkv, S, hd)).copy()
+    vc = r.standard_normal((B, nkv, S, hd))
+    lens = np.array([S, S])
+    o = ref.prefill_attention(q, kc, vc, lens, causal=False)
+    for b in range(B):
+        for h in range(nh):
+            j = h // (nh // nkv)
+            np.testing.assert_allclose(o[b, :, h], np.broadcast_to(vc[b, j].mean(0), (S, hd)), atol=1e-13)
+    o = ref.prefill_attention(q, kc, vc, lens, causal=True)
+    for i in range(S):
+        np.testing.assert_allclose(o[1, i, 3], vc[1, 1, :i + 1].mean(0), atol=1e-13)
+    # q = 0 gives uniform weights whatever the keys are
+    kc2 = r.standard_normal((B, nkv, S, hd))
+    o = ref.prefill_attention(np.zeros_like(q), kc2, vc, lens, causal=True)
+    np.testing.assert_allclose(o[0, 4, 0], vc[0, 0, :5].mean(0), atol=1e-13)
+
+
+def test_single_visible_key_returns_its_value():
+    r = rng(9)
+    q, kc, vc = _rand_attn(r, 1, 2, 1, 5, 5, 8)
+    o = ref.prefill_attention(q, kc, vc, np.array([5]), causal=True)
+    np.testing.assert_allclose(o[0, 0, 0], vc[0, 0, 0], atol=1e-15)
+    np.testing.assert_allclose(o[0, 0, 1], vc[0, 0, 0], atol=1e-15)
+
+
+def test_no_visible_key_gives_zero_row():
+    r = rng(10)
+    q, kc, vc = _rand_attn(r, 1, 2, 1, 3, 4, 8)
+    o = ref.prefill_attention(q, kc, vc, np.array([0]), causal=True)
+    assert np.all(o == 0)
+    o = ref.decode_attention(q[:, :, 0], kc, vc, np.array([0]))
+    assert np.all(o == 0)
+
+
+def test_noncausal_permutation_invariance():
+    r = rng(11)
+    q, kc, vc = _rand_attn(r, 1, 4, 2, 3, 9, 8)
+    perm = r.permutation(9)
+    o1 = ref.prefill_attention(q, kc, vc, np.array([9]), causal=False)
+    o2 = ref.prefill_attention(q, kc[:, :, perm], vc[:, :, perm], np.array([9]), causal=False)
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+
+
+def check_gqa_equals_mha_with_repeated_kv():
+    r = rng(12)
+    B, nh, S, hd = 2, 8, 5, 8
+    for nkv in (1, 2, 4, 8):
+        q, kc, vc = _rand_attn(r, B, nh, nkv, S, S, hd)
+        lens = np.array([S, S - 2])
+        g = nh // nkv
+        kr, vr = np.repeat(kc, g, axis=1), np.repeat(vc, g, axis=1)   # repeat_kv
+        for causal in (True, False):
+            np.testing.assert_allclose(
+                ref.prefill_attention(q, kc, vc, lens, causal),
+                ref.prefill_attention(q, kr, vr, lens, causal), atol=1e-13)
+        np.testing.assert_allclose(
+            ref.decode_attention(q[:, :, -1], kc, vc, lens),
+            ref.decode_attention(q[:, :, -1], kr, vr, lens), atol=1e-13)
+
+
+def test_gqa_equals_mha_with_repeated_kv():
+    check_gqa_equals_mha_with_repeated_kv()
+
+
+def test_mqa_every_head_reads_the_single_kv_head():
+    r = rng(13)
+    q, kc, vc = _rand_attn(r, 1, 6, 1, 4, 4, 8)
+    o = ref.prefill_attention(q, kc, vc, np.array([4]), causal=False)
+    for h in range(6):
+        oh = ref.prefill_attention(q[:, h:h + 1], kc, vc, np.array([4]), causal=False)
+        np.testing.assert_allclose(o[:, :, h], oh[:, :, 0], atol=1e-14)
+
+
+def check_last_causal_row_equals_decode():
+    r = rng(14)
+    B, nh, nkv, S, hd = 2, 4, 2, 7, 16
+    q, kc, vc = _rand_attn(r, B, nh, nkv, S, S, hd)
+    lens = np.array([S, S])
+    o = ref.prefill_attention(q, kc, vc, lens, causal=True)
+    d = ref.decode_attention(q[:, :, -1], kc, vc, lens)
+    np.testing.assert_allclose(o[:, -1], d, atol=1e-13)
+    # and every causal row s equals a decode with kv_len = s + 1
+    for s in range(S):
+        d = ref.decode_attention(q[:, :, s], kc, vc, np.array([s + 1, s + 1]))
+        np.testing.assert_allclose(o[:, s], d, atol=1e-13)
+
+
+def test_last_causal_prefill_row_equals_decode_step():
+    check_last_causal_row_equals_decode()
+
+
+def test_bottom_right_causal_alignment_and_explicit_positions():
+    r = rng(15)
+    B, nh, nkv, S, L, hd = 1, 2, 1, 3, 10, 8
+    q, kc, vc = _rand_attn(r, B, nh, nkv, S, L, hd)
+    lens = np.array([L])
+    o = ref.prefill_attention(q, kc, vc, lens, causal=True)
+    for s in range(S):   # query s sits at position L - S + s and sees keys 0..L-S+s
+        want, _ = ref.attend_row(q[0, 1, s], kc[0, 0], vc[0, 0], L - S + s + 1)
+        np.testing.assert_allclose(o[0, s, 1], want, atol=1e-13)
+    o2 = ref.prefill_attention(q, kc, vc, lens, causal=True, q_positions=np.array([[7, 8, 9]]))
+    np.testing.assert_allclose(o, o2, atol=0)
+
+
+def test_nan_padding_never_reaches_output():
+    r = rng(16)
+    q, kc, vc = _rand_attn(r, 2, 4, 2, 3, 12, 8)
+    lens = np.array([5, 12])
+    kc[0, :, 5:] = np.nan
+    vc[0, :, 5:] = np.nan
+    o = ref.prefill_attention(q, kc, vc, lens, causal=False)
+    d = ref.decode_attention(q[:, :, 0], kc, vc, lens)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(d))
+
+
+def check_brute_force_attention():
+    r = rng(17)
+    for (B, nh, nkv, S, L, hd) in ((1, 2, 1, 3, 5, 4), (2, 4, 2, 6, 6, 8), (2, 4, 1, 4, 6, 2)):
+        q, kc, vc = _rand_attn(r, B, nh, nkv, S, L, hd)
+        lens = np.array([L - 1, L][:B])
+        for causal in (True, False):
+            o = ref.prefill_attention(q, kc, vc, lens, causal)
+            for b in range(B):
+                for h in range(nh):
+                    j = h * nkv // nh
+                    for s in range(S):
+                        p = lens[b] - S + s
+                        vis = [t < lens[b] and (not causal or t <= p) for t in range(L)]
+                        want = brute_attention_row(list(q[b, h, s]), kc[b, j].tolist(), vc[b, j].tolist(), vis)
+                        np.testing.assert_allclose(o[b, s, h], want, rtol=0, atol=1e-12)
+        d = ref.decode_attention(q[:, :, 0], kc, vc, lens)
+        for b in range(B):
+            for h in range(nh):
+                j = h * nkv // nh
+                vis = [t < lens[b] for t in range(L)]
+                want = brute_attention_row(list(q[b, h, 0]), kc[b, j].tolist(), vc[b, j].tolist(), vis)
+                np.testing.assert_allclose(d[b, h], want, rtol=0, atol=1e-12)
+
+
+def test_brute_force_attention():
+    check_brute_force_attention()
+
+
+def test_generation_loop_equals_causal_prefill():
+    """Prompt prefill then one-token decode steps that grow the cache in place
+    give the rows of one causal prefill over all tokens."""
+    r = rng(18)
+    B, D, nh, nkv, hd, P, T = 2, 16, 4, 1, 8, 3, 4
+    cap = P + T
+    w = r.standard_normal(((nh + 2 * nkv) * hd, D)) * 0.3
+    x = r.standard_normal((B, P + T, D))
+    pos = np.broadcast_to(np.arange(P + T), (B, P + T))
+    kc0 = np.full((B, nkv, cap, hd), np.nan)
+    vc0 = np.full((B, nkv, cap, hd), np.nan)
+    q_all, kc_all, vc_all = ref.qkv_rope_project(x, w, pos, nh, nkv, hd, 10000.0, kc0, vc0)
+    full = ref.prefill_attention(q_all, kc_all, vc_all, np.array([cap, cap]), causal=True)
+    q_p, kc, vc = ref.qkv_rope_project(x[:, :P], w, pos[:, :P], nh, nkv, hd, 10000.0, kc0, vc0)
+    o_p = ref.prefill_attention(q_p, kc, vc, np.array([P, P]), causal=True)
+    np.testing.assert_allclose(o_p, full[:, :P], atol=1e-12)
+    for t in range(T):
+        q_t, kc, vc = ref.qkv_rope_project(x[:, P + t:P + t + 1], w, pos[:, P + t:P + t + 1],
+                                           nh, nkv, hd, 10000.0, kc, vc)
+        o_t = ref.decode_attention(q_t[:, :, 0], kc, vc, np.array([P + t + 1] * B))
+        np.testing.assert_allclose(o_t, full[:, P + t], atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: each must make at least one pin fail
+# --------------------------------------------------------------------------
+def _fails(check):
+    try:
+        check()
+    except AssertionError:
+        return True
+    return False
+
+
+def test_planted_wrong_head_map_is_caught(monkeypatch):
+    monkeypatch.setattr(ref, "kv_head_of", lambda h, nh, nkv: h % nkv)
+    assert _fails(check_gqa_equals_mha_with_repeated_kv)
+    assert _fails(check_brute_force_attention)
+
+
+def test_planted_dropped_scale_is_caught(monkeypatch):
+    orig = ref.softmax
+    monkeypatch.setattr(ref, "np", _NumpyNoSqrt())
+    assert _fails(check_closed_form_two_keys)
+    monkeypatch.setattr(ref, "softmax", orig)
+
+
+class _NumpyNoSqrt:
+    """numpy with sqrt replaced by 1 (drops the 1/sqrt(hd) softmax scale)."""
+
+    def __getattr__(self, name):
+        if name == "sqrt":
+            return lambda x: 1.0
+        return getattr(np, name)
+
+
+def test_planted_interleaved_rope_is_caught(monkeypatch):
+    def interleaved(t, positions, theta):
+        t = np.asarray(t, dtype=np.float64)
+        hd = t.shape[-1]
+        ang = np.asarray(positions, dtype=np.float64)[..., None] * ref.rope_inv_freq(hd, theta)
+        c, s = np.cos(ang)[:, :, None, :], np.sin(ang)[:, :, None, :]
+        ev, od = t[..., 0::2], t[..., 1::2]
+        out = np.empty_like(t)
+        out[..., 0::2] = ev * c - od * s
+        out[..., 1::2] = od * c + ev * s
+        return out
+    monkeypatch.setattr(ref, "apply_rope", interleaved)
+    assert _fails(check_rope_hand_example)
+
+
+def test_planted_rope_sign_error_is_caught(monkeypatch):
+    orig = ref.apply_rope
+    monkeypatch.setattr(ref, "apply_rope", lambda t, p, th: orig(t, -np.asarray(p), th))
+    assert _fails(check_rope_hand_example)
+
+
+def test_planted_swapped_kv_slices_is_caught(monkeypatch):
+    orig = ref.split_qkv
+
+    def swapped(y, nh, nkv, hd):
+        q, k, v = orig(y, nh, nkv, hd)
+        return q, v, k
+    monkeypatch.setattr(ref, "split_qkv", swapped)
+    assert _fails(check_split_matches_page)
+    assert _fails(check_fused_equals_separate)
+
+
+def test_planted_transposed_weight_is_caught(monkeypatch):
+    monkeypatch.setattr(ref, "fused_projection",
+                        lambda x, w: np.asarray(x) @ np.asarray(w).reshape(w.shape[1], w.shape[0]))
+    assert _fails(check_fused_equals_separate)
+
+
+def test_planted_off_by_one_causal_is_caught(monkeypatch):
+    orig = ref.default_q_positions
+    monkeypatch.setattr(ref, "default_q_positions", lambda kv, S: orig(kv, S) - 1)
+    assert _fails(check_last_causal_row_equals_decode)
