@@ -1,0 +1,181 @@
+/*
+ * gqa.h - C ABI of the B200 (sm_100a) fused-QKV + grouped-query attention
+ * library (libgqa_b200.so).
+ *
+ * Three calls form the path of one Llama-style attention layer:
+ *
+ *   qkv_rope_project   hidden states -> one fused W_qkv GEMM -> RoPE on q/k ->
+ *                      q written head-major, k/v written into the KV cache
+ *   gqa_attn_prefill   exact (online-softmax) attention of S new queries per
+ *                      sequence over the cache, causal or not
+ *   gqa_attn_decode    one new query per sequence over a ragged-length cache,
+ *                      split along the keys, partials merged by log-sum-exp
+ *
+ * Grouped-query attention: n_heads query heads share n_kv_heads key/value
+ * heads, g = n_heads / n_kv_heads consecutive query heads per KV head (query
+ * head h reads KV head h / g).  MHA is n_kv_heads == n_heads, MQA is
+ * n_kv_heads == 1.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *   never allocates, frees, synchronises or prints.  Every call is
+ *   asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
+ *   legacy default stream) and may be captured in a CUDA graph.
+ * - Tensors are dense, row-major ("C order") with the shapes given below, and
+ *   every tensor pointer must be 16-byte aligned (int32 arrays: 4-byte).
+ * - dtype: GQA_F32 (float32 everywhere, FFMA arithmetic, no TF32) or
+ *   GQA_BF16 (bfloat16 storage, float32 accumulation; P is rounded to bf16
+ *   before the P.V product, outputs are rounded once to nearest-even).
+ * - Return value: GQA_OK (0) or a negative GQA_ERR_* code.  Arguments are
+ *   validated on the host only; device data (positions, kv_lens) is never
+ *   read by the host.  Device-side range problems (a position outside
+ *   [0, cache_cap), a kv_len above cache_cap) are clamped or skipped as
+ *   documented per call and recorded in a device error word that
+ *   gqa_device_error() reads.
+ * - head_dim must be 32, 64 or 128; B == 0 or S == 0 is a valid no-op.
+ * - Runs only on compute capability 10.0 devices (B200, sm_100a).
+ */
+#ifndef GQA_B200_H
+#define GQA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum gqa_dtype { GQA_F32 = 0, GQA_BF16 = 1 };
+
+enum gqa_status {
+  GQA_OK = 0,
+  GQA_ERR_INVALID_ARG = -1,        /* null pointer, negative size, nh % nkv != 0, ... */
+  GQA_ERR_MISALIGNED = -2,         /* a tensor pointer is not 16-byte aligned */
+  GQA_ERR_UNSUPPORTED_DTYPE = -3,  /* dtype is neither GQA_F32 nor GQA_BF16 */
+  GQA_ERR_UNSUPPORTED_ARCH = -4,   /* current device is not compute capability 10.0 */
+  GQA_ERR_WORKSPACE_TOO_SMALL = -5,/* decode workspace smaller than the size query */
+  GQA_ERR_LAUNCH_FAILED = -6,      /* a kernel launch returned a CUDA error */
+  GQA_ERR_UNSUPPORTED_SHAPE = -7,  /* head_dim not in {32, 64, 128} or a size too large */
+  GQA_ERR_NO_DEVICE = -8           /* no CUDA device is current */
+};
+
+/* Device error word bits (gqa_device_error). */
+enum gqa_device_error_bits {
+  GQA_DEVERR_POSITION_RANGE = 1,   /* a position outside [0, cache_cap): K/V row not written */
+  GQA_DEVERR_KVLEN_RANGE = 2,      /* a kv_len above cache_cap (clamped) or below 0 (taken as 0) */
+  GQA_DEVERR_WAIT_TIMEOUT = 4      /* a pipeline wait gave up after its time limit */
+};
+
+/*
+ * qkv_rope_project - steps a1..a3 of the path.
+ *
+ * Source: "Optimize LlamaAttention by fusing QKV projections"
+ * (huggingface/transformers pull request #40092), LlamaAttention.forward:
+ * one qkv_proj linear layer whose output is sliced into query features
+ * [0, nh*hd), key features [nh*hd, (nh+nkv)*hd) and value features
+ * [(nh+nkv)*hd, (nh+2nkv)*hd); head j of a block owns features j*hd..j*hd+hd-1.
+ * RoPE (rotate_half pairing: feature i with i + hd/2, inv_freq_i =
+ * theta^(-2i/hd), angle = position * inv_freq_i) is applied to q and k only
+ * (the fused-QKV toy model of the custom-op overhead gist also applies its
+ * position step to q and k after the split).
+ *
+ *   x          [B, S, hidden]                      dtype
+ *   w_qkv      [(n_heads + 2 n_kv_heads) * head_dim, hidden]  dtype
+ *              (nn.Linear storage: y = x w^T, no bias)
+ *   positions  [B, S] int32: absolute position of each token; it sets the
+ *              rotation angle and the cache slot of its K/V rows
+ *   q_out      [B, n_heads, S, head_dim] dtype (written, head-major)
+ *   k_cache,
+ *   v_cache    [B, n_kv_heads, cache_cap, head_dim] dtype; row positions[b,s]
+ *              of every KV head of sequence b is overwritten, all other rows
+ *              are left untouched.  A position outside [0, cache_cap) writes
+ *              no K/V row and sets GQA_DEVERR_POSITION_RANGE (q is still
+ *              written, rotated by that position).
+ *
+ * The math is float32 (fp32 accumulation of bf16 products for GQA_BF16), with
+ * one final rounding of q/k/v to dtype.
+ */
+int qkv_rope_project(const void* x, const void* w_qkv, const int32_t* positions,
+                     int B, int S, int hidden, int n_heads, int n_kv_heads, int head_dim,
+                     float rope_theta, void* q_out, void* k_cache, void* v_cache,
+                     int cache_cap, int dtype, void* stream);
+
+/*
+ * gqa_attn_prefill - step a4: exact attention of S queries per sequence.
+ *
+ * Source: "FlashAttention-3" (together.ai summary), section
+ * "FlashAttention方式のおさらい": tiled attention with softmax rescaling gives
+ * the exact softmax(Q K^T / sqrt(hd)) V without writing the score matrix;
+ * "MHA -> GQA" blog, section 3.2: g query heads share one KV head.
+ *
+ *   q            [B, n_heads, S, head_dim] dtype (as written by qkv_rope_project)
+ *   k_cache,
+ *   v_cache      [B, n_kv_heads, cache_cap, head_dim] dtype
+ *   q_positions  [B, S] int32 or NULL.  NULL means kv_lens[b] - S + s
+ *                (the S queries are the last S cached tokens).
+ *   kv_lens      [B] int32: keys 0..kv_lens[b]-1 of sequence b are valid;
+ *                values above cache_cap are clamped (GQA_DEVERR_KVLEN_RANGE).
+ *   causal       nonzero: key t is visible to a query at position p iff t <= p
+ *   out          [B, S, n_heads, head_dim] dtype (token-major, ready for an
+ *                output projection).  A query with no visible key gets zeros.
+ *
+ * Scale 1/sqrt(head_dim).  Cache rows at or beyond kv_len are never read
+ * into the result (they may hold anything, NaN included).
+ */
+int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* q_positions, const int32_t* kv_lens,
+                     int B, int S, int n_heads, int n_kv_heads, int head_dim,
+                     int cache_cap, int causal, void* out, int dtype, void* stream);
+
+/*
+ * gqa_attn_decode_workspace_size - bytes of device workspace gqa_attn_decode
+ * needs for these sizes (float32 partial results: a running max, a sum and
+ * an unnormalised output row per sequence, query head and key split).
+ * kv_split: keys per split, 0 = the library's choice, else a multiple of 64.
+ * Returns 0 for invalid arguments.
+ */
+size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int head_dim,
+                                      int cache_cap, int kv_split);
+
+/*
+ * gqa_attn_decode - steps a5..a6: one new query per sequence.
+ *
+ * Source: "MHA -> GQA" blog, sections 3.1-3.2: decode attention is a batched
+ * matrix-vector product over ragged lengths and stays memory-bound; the g
+ * query heads that share a KV head are processed together so that every
+ * K/V byte read serves g heads (arithmetic intensity ~g).  The keys of a
+ * sequence are split into chunks of kv_split; each chunk produces a partial
+ * (max m, sum l, unnormalised o) per head and the partials are merged with a
+ * log-sum-exp combine, which is exact.
+ *
+ *   q          [B, n_heads, head_dim] dtype (the new token, already rotated)
+ *   k_cache,
+ *   v_cache    [B, n_kv_heads, cache_cap, head_dim] dtype
+ *   kv_lens    [B] int32: valid keys including the new token; clamped to
+ *              [0, cache_cap] (GQA_DEVERR_KVLEN_RANGE); 0 gives a zero row
+ *   kv_split   keys per split: 0 = automatic, else a positive multiple of 64
+ *   out        [B, n_heads, head_dim] dtype
+ *   workspace  device scratch of at least gqa_attn_decode_workspace_size()
+ *              bytes, 16-byte aligned; its contents on entry do not matter.
+ */
+int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,
+                    int cache_cap, int kv_split, void* out, void* workspace,
+                    size_t workspace_bytes, int dtype, void* stream);
+
+/* Human-readable text of a gqa_status value (static storage). */
+const char* gqa_status_string(int status);
+
+/*
+ * gqa_device_error - debugging aid: waits for the current device to finish,
+ * copies the device error word (GQA_DEVERR_* bits accumulated by earlier
+ * calls) to *bits and clears it.  Unlike every other call it synchronises.
+ */
+int gqa_device_error(int* bits);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_B200_H */

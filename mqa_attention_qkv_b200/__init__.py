@@ -1,0 +1,184 @@
+"""Python binding of libgqa_b200 (fused-QKV projection + grouped-query
+attention for B200 / sm_100a).
+
+Argument marshalling only: shapes are read from the torch tensors, pointers
+and sizes are passed to the C ABI declared in ``include/gqa.h``, and every step
+of the computation runs in the library's CUDA kernels.  PyTorch provides the
+device memory and the stream.  There is no other code path: if the shared
+library is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "GQA_F32", "GQA_BF16", "GQAError", "library_path", "lib",
+    "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
+    "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
+    "EXPORTED_SYMBOLS",
+]
+
+GQA_F32 = 0
+GQA_BF16 = 1
+
+EXPORTED_SYMBOLS = (
+    "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
+    "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
+)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+
+class GQAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {gqa_status_string(status)} (status {status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libgqa_b200.so")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded shared library (loaded on first use; raises if absent)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run `python -m mqa_attention_qkv_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.qkv_rope_project.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, ctypes.c_float,
+                                   vp, vp, vp, i32, i32, vp]
+    L.qkv_rope_project.restype = i32
+    L.gqa_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+    L.gqa_attn_prefill.restype = i32
+    L.gqa_attn_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.gqa_attn_decode_workspace_size.restype = sz
+    L.gqa_attn_decode.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, sz, i32, vp]
+    L.gqa_attn_decode.restype = i32
+    L.gqa_status_string.argtypes = [i32]
+    L.gqa_status_string.restype = ctypes.c_char_p
+    L.gqa_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    L.gqa_device_error.restype = i32
+    _LIB = L
+    return L
+
+
+def gqa_status_string(status: int) -> str:
+    return lib().gqa_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise GQAError(fn, status)
+
+
+# --------------------------------------------------------------------------
+# tensor marshalling helpers
+# --------------------------------------------------------------------------
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return GQA_BF16
+    if t.dtype == torch.float32:
+        return GQA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _ptr(t, dtype=None, shape=None, name="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+# --------------------------------------------------------------------------
+# the three calls
+# --------------------------------------------------------------------------
+def qkv_rope_project(x, w_qkv, positions, n_heads: int, n_kv_heads: int, head_dim: int,
+                     rope_theta: float, q_out, k_cache, v_cache, stream=None) -> None:
+    """x [B,S,hidden], w_qkv [(nh+2nkv)*hd, hidden], positions [B,S] int32 ->
+    q_out [B,nh,S,hd]; k_cache/v_cache [B,nkv,cap,hd] written at slot=position."""
+    import torch
+    B, S, hidden = x.shape
+    dt = x.dtype
+    cap = k_cache.shape[2]
+    n_qkv = (n_heads + 2 * n_kv_heads) * head_dim
+    args = (
+        _ptr(x, dt, name="x"), _ptr(w_qkv, dt, (n_qkv, hidden), "w_qkv"),
+        _ptr(positions, torch.int32, (B, S), "positions"),
+        B, S, hidden, n_heads, n_kv_heads, head_dim, float(rope_theta),
+        _ptr(q_out, dt, (B, n_heads, S, head_dim), "q_out"),
+        _ptr(k_cache, dt, (B, n_kv_heads, cap, head_dim), "k_cache"),
+        _ptr(v_cache, dt, (B, n_kv_heads, cap, head_dim), "v_cache"),
+        cap, _dtype_code(x), _stream(stream),
+    )
+    _check("qkv_rope_project", lib().qkv_rope_project(*args))
+
+
+def gqa_attn_prefill(q, k_cache, v_cache, kv_lens, causal: bool, out, q_positions=None,
+                     stream=None) -> None:
+    """q [B,nh,S,hd], caches [B,nkv,cap,hd], kv_lens [B] int32 -> out [B,S,nh,hd]."""
+    import torch
+    B, nh, S, hd = q.shape
+    nkv, cap = k_cache.shape[1], k_cache.shape[2]
+    dt = q.dtype
+    args = (
+        _ptr(q, dt, name="q"), _ptr(k_cache, dt, (B, nkv, cap, hd), "k_cache"),
+        _ptr(v_cache, dt, (B, nkv, cap, hd), "v_cache"),
+        _ptr(q_positions, torch.int32, (B, S), "q_positions"),
+        _ptr(kv_lens, torch.int32, (B,), "kv_lens"),
+        B, S, nh, nkv, hd, cap, 1 if causal else 0,
+        _ptr(out, dt, (B, S, nh, hd), "out"), _dtype_code(q), _stream(stream),
+    )
+    _check("gqa_attn_prefill", lib().gqa_attn_prefill(*args))
+
+
+def gqa_attn_decode_workspace_size(B: int, n_heads: int, n_kv_heads: int, head_dim: int,
+                                   cache_cap: int, kv_split: int = 0) -> int:
+    return int(lib().gqa_attn_decode_workspace_size(B, n_heads, n_kv_heads, head_dim, cache_cap, kv_split))
+
+
+def gqa_attn_decode(q, k_cache, v_cache, kv_lens, out, workspace, kv_split: int = 0,
+                    stream=None) -> None:
+    """q [B,nh,hd], caches [B,nkv,cap,hd], kv_lens [B] int32 -> out [B,nh,hd].
+    ``workspace`` is a CUDA tensor of at least gqa_attn_decode_workspace_size bytes."""
+    import torch
+    B, nh, hd = q.shape
+    nkv, cap = k_cache.shape[1], k_cache.shape[2]
+    dt = q.dtype
+    ws_bytes = workspace.numel() * workspace.element_size()
+    args = (
+        _ptr(q, dt, name="q"), _ptr(k_cache, dt, (B, nkv, cap, hd), "k_cache"),
+        _ptr(v_cache, dt, (B, nkv, cap, hd), "v_cache"),
+        _ptr(kv_lens, torch.int32, (B,), "kv_lens"),
+        B, nh, nkv, hd, cap, int(kv_split),
+        _ptr(out, dt, (B, nh, hd), "out"), _ptr(workspace, name="workspace"), ws_bytes,
+        _dtype_code(q), _stream(stream),
+    )
+    _check("gqa_attn_decode", lib().gqa_attn_decode(*args))
+
+
+def gqa_device_error() -> int:
+    """Read and clear the device error word (synchronises the device)."""
+    v = ctypes.c_int(0)
+    _check("gqa_device_error", lib().gqa_device_error(ctypes.byref(v)))
+    return v.value

@@ -1,0 +1,210 @@
+// C ABI of libgqa_b200: host-side argument validation, kernel selection and
+// launch on the caller's stream.  No allocation, no synchronisation, no
+// printing (gqa_device_error, a debugging aid, is the one synchronising call).
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/gqa.h"
+#include "kernels.h"
+
+namespace {
+
+// Device error word: one per device, in the library's static device memory.
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  std::once_flag once;
+  int cc_major = 0, cc_minor = 0, num_sms = 0;
+  int* err = nullptr;
+  cudaError_t status = cudaSuccess;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+// Per-device facts, queried once with that device current.
+const DeviceInfo* device_info(int* status) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    *status = GQA_ERR_NO_DEVICE;
+    return nullptr;
+  }
+  DeviceInfo& d = g_dev[dev];
+  std::call_once(d.once, [&] {
+    cudaError_t e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaGetSymbolAddress(reinterpret_cast<void**>(&d.err), g_device_error);
+    d.status = e;
+    if (e != cudaSuccess) cudaGetLastError();
+  });
+  if (d.status != cudaSuccess) {
+    *status = GQA_ERR_NO_DEVICE;
+    return nullptr;
+  }
+  if (d.cc_major != 10 || d.cc_minor != 0) {
+    *status = GQA_ERR_UNSUPPORTED_ARCH;
+    return nullptr;
+  }
+  *status = GQA_OK;
+  return &d;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool hd_ok(int hd) { return hd == 32 || hd == 64 || hd == 128; }
+
+int launch_status(cudaError_t e) {
+  if (e == cudaSuccess) return GQA_OK;
+  cudaGetLastError();
+  return GQA_ERR_LAUNCH_FAILED;
+}
+
+// Keys per decode split when the caller leaves it to the library: enough
+// (sequence, KV head, split) work units to fill the GPU several times over
+// for a half-full cache, between 64 and 2048 keys, a multiple of 64.
+int auto_split(int B, int nkv, int cap) {
+  const long long units_wanted = 1024;
+  long long s = ((long long)B * nkv * ((cap + 1) / 2) + units_wanted - 1) / units_wanted;
+  s = (s + 63) / 64 * 64;
+  if (s < 64) s = 64;
+  if (s > 2048) s = 2048;
+  return (int)s;
+}
+
+constexpr long long kMaxElems = 1ll << 40;
+
+}  // namespace
+
+extern "C" {
+
+const char* gqa_status_string(int status) {
+  switch (status) {
+    case GQA_OK: return "ok";
+    case GQA_ERR_INVALID_ARG: return "invalid argument";
+    case GQA_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case GQA_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype";
+    case GQA_ERR_UNSUPPORTED_ARCH: return "device is not compute capability 10.0 (sm_100a)";
+    case GQA_ERR_WORKSPACE_TOO_SMALL: return "decode workspace too small";
+    case GQA_ERR_LAUNCH_FAILED: return "kernel launch failed";
+    case GQA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (head_dim must be 32, 64 or 128)";
+    case GQA_ERR_NO_DEVICE: return "no usable CUDA device";
+    default: return "unknown status";
+  }
+}
+
+int gqa_device_error(int* bits) {
+  if (!bits) return GQA_ERR_INVALID_ARG;
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (!d) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return launch_status(cudaErrorUnknown);
+  int v = 0;
+  if (cudaMemcpy(&v, d->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return launch_status(cudaErrorUnknown);
+  const int zero = 0;
+  if (cudaMemcpy(d->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return launch_status(cudaErrorUnknown);
+  *bits = v;
+  return GQA_OK;
+}
+
+int qkv_rope_project(const void* x, const void* w_qkv, const int32_t* positions,
+                     int B, int S, int hidden, int n_heads, int n_kv_heads, int head_dim,
+                     float rope_theta, void* q_out, void* k_cache, void* v_cache,
+                     int cache_cap, int dtype, void* stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || S < 0 || hidden <= 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0)
+    return GQA_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f)) return GQA_ERR_INVALID_ARG;
+  if (!hd_ok(head_dim)) return GQA_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * S * hidden > kMaxElems || (long long)B * S >= (1ll << 31) ||
+      (long long)(n_heads + 2 * n_kv_heads) * head_dim * hidden > kMaxElems)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || S == 0) return GQA_OK;
+  if (!x || !w_qkv || !positions || !q_out || !k_cache || !v_cache) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q_out) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned4(positions))
+    return GQA_ERR_MISALIGNED;
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (!d) return st;
+
+  gqa::QkvParams p{x, w_qkv, positions, B, S, hidden, n_heads, n_kv_heads, head_dim, cache_cap,
+                   (double)rope_theta, q_out, k_cache, v_cache, d->err};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_status(gqa::launch_qkv_simt(p, dtype == GQA_BF16, s));
+}
+
+int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
+                     const int32_t* q_positions, const int32_t* kv_lens,
+                     int B, int S, int n_heads, int n_kv_heads, int head_dim,
+                     int cache_cap, int causal, void* out, int dtype, void* stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || S < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0) return GQA_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
+  if (!hd_ok(head_dim)) return GQA_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems ||
+      (long long)B * n_heads * S * head_dim > kMaxElems || B > 65535 || n_heads > 65535)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || S == 0) return GQA_OK;
+  if (!q || !k_cache || !v_cache || !kv_lens || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned4(kv_lens) || (q_positions && !aligned4(q_positions)))
+    return GQA_ERR_MISALIGNED;
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (!d) return st;
+
+  gqa::PrefillParams p{q, k_cache, v_cache, q_positions, kv_lens, B, S, n_heads, n_kv_heads,
+                       head_dim, cache_cap, causal ? 1 : 0, out, d->err};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_status(gqa::launch_prefill_simt(p, dtype == GQA_BF16, s));
+}
+
+size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int head_dim,
+                                      int cache_cap, int kv_split) {
+  if (B < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0 || n_heads % n_kv_heads) return 0;
+  if (!hd_ok(head_dim)) return 0;
+  if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return 0;
+  const int split = kv_split ? kv_split : auto_split(B, n_kv_heads, cache_cap);
+  const size_t n_split = (size_t)(cache_cap + split - 1) / split;
+  return (size_t)B * n_heads * n_split * (head_dim + gqa::kWsPad) * sizeof(float);
+}
+
+int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,
+                    int cache_cap, int kv_split, void* out, void* workspace,
+                    size_t workspace_bytes, int dtype, void* stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0) return GQA_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
+  if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;
+  if (!hd_ok(head_dim)) return GQA_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems || B > 65535 || n_kv_heads > 65535)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return GQA_OK;
+  if (!q || !k_cache || !v_cache || !kv_lens || !out || !workspace) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      !aligned16(workspace) || !aligned4(kv_lens))
+    return GQA_ERR_MISALIGNED;
+  const size_t need = gqa_attn_decode_workspace_size(B, n_heads, n_kv_heads, head_dim, cache_cap, kv_split);
+  if (workspace_bytes < need) return GQA_ERR_WORKSPACE_TOO_SMALL;
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (!d) return st;
+
+  const int split = kv_split ? kv_split : auto_split(B, n_kv_heads, cache_cap);
+  gqa::DecodeParams p{q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim, cache_cap,
+                      split, (cache_cap + split - 1) / split, static_cast<float*>(workspace), out,
+                      d->err};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf16 = dtype == GQA_BF16;
+  cudaError_t e = gqa::launch_decode_simt(p, bf16, s);
+  if (e == cudaSuccess) e = gqa::launch_decode_combine(p, bf16, s);
+  return launch_status(e);
+}
+
+}  // extern "C"

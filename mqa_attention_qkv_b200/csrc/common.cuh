@@ -1,0 +1,111 @@
+// Device helpers shared by the kernels of libgqa_b200: storage conversion,
+// the device error word, and the bounded waits every pipeline uses.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gqa.h"
+
+namespace gqa {
+
+// ---------------------------------------------------------------------------
+// storage type <-> float
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// ---------------------------------------------------------------------------
+// device error word (bits of gqa_device_error_bits)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void raise_error(int* err, int bits) {
+  if (err) atomicOr(err, bits);
+}
+
+// ---------------------------------------------------------------------------
+// Rotary embedding angle.  inv_freq_i = theta^(-2i/hd) and the angle
+// position * inv_freq_i are formed in double precision and reduced to
+// [-pi, pi] before the float sincos, so the angle error stays ~1e-7 rad even
+// at position 8191 (a float product would carry ~5e-4 rad there).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double rope_inv_freq(int i, int hd, double theta) {
+  return pow(theta, -2.0 * (double)i / (double)hd);
+}
+
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  double a = (double)pos * inv_freq;
+  a -= two_pi * rint(a * (1.0 / two_pi));
+  sincosf((float)a, s, c);
+}
+
+// ---------------------------------------------------------------------------
+// Time-bounded waits.  A wait that has not succeeded after kWaitLimitNs gives
+// up, records GQA_DEVERR_WAIT_TIMEOUT and returns false; the caller then skips
+// the rest of its work and goes straight to its teardown.
+// ---------------------------------------------------------------------------
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier to complete; bounded in time.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+      raise_error(err, GQA_DEVERR_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+}  // namespace gqa

@@ -1,0 +1,54 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gqa {
+
+struct QkvParams {
+  const void* x;          // [T, hidden]      T = B*S
+  const void* w;          // [N, hidden]      N = (nh + 2 nkv) * hd
+  const int32_t* pos;     // [T]
+  int B, S, hidden, nh, nkv, hd, cap;
+  double theta;
+  void* q_out;            // [B, nh, S, hd]
+  void* k_cache;          // [B, nkv, cap, hd]
+  void* v_cache;
+  int* err;
+};
+
+struct PrefillParams {
+  const void* q;          // [B, nh, S, hd]
+  const void* k_cache;    // [B, nkv, cap, hd]
+  const void* v_cache;
+  const int32_t* q_pos;   // [B, S] or nullptr
+  const int32_t* kv_lens; // [B]
+  int B, S, nh, nkv, hd, cap, causal;
+  void* out;              // [B, S, nh, hd]
+  int* err;
+};
+
+struct DecodeParams {
+  const void* q;          // [B, nh, hd]
+  const void* k_cache;    // [B, nkv, cap, hd]
+  const void* v_cache;
+  const int32_t* kv_lens; // [B]
+  int B, nh, nkv, hd, cap;
+  int split;              // keys per split
+  int n_split;            // ceil(cap / split)
+  float* ws;              // [B, nh, n_split, hd + 4]: o[hd], m, l, -, -
+  void* out;              // [B, nh, hd]
+  int* err;
+};
+
+constexpr int kWsPad = 4;  // per-partial row: hd floats of o, then m, l and two pad words
+
+// SIMT kernels (any dtype; the fp32 path and shapes the tensor-core kernels skip)
+cudaError_t launch_qkv_simt(const QkvParams& p, bool bf16, cudaStream_t st);
+cudaError_t launch_prefill_simt(const PrefillParams& p, bool bf16, cudaStream_t st);
+cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, cudaStream_t st);
+cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t st);
+
+}  // namespace gqa

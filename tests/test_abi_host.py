@@ -1,0 +1,128 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+the header declares, and rejects bad arguments on the host before any device
+work (so these calls never touch the fake pointers they are given)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mqa_attention_qkv_b200 as gqa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa.h")
+
+# 16-byte aligned, never dereferenced: every call below fails validation first.
+P = 0x100000
+MIS = P + 8
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|void)\s*\*?\s*(\w+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert set(names) == set(gqa.EXPORTED_SYMBOLS), names
+    L = ctypes.CDLL(gqa.library_path())
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+        s = gqa.gqa_status_string(code)
+        assert s and s != "unknown status"
+    assert gqa.gqa_status_string(12345) == "unknown status"
+
+
+def _qkv(**kw):
+    a = dict(x=P, w=P, pos=P, B=2, S=4, hidden=64, nh=4, nkv=2, hd=64, theta=1e4,
+             q=P, k=P, v=P, cap=16, dtype=1, stream=None)
+    a.update(kw)
+    return gqa.lib().qkv_rope_project(a["x"], a["w"], a["pos"], a["B"], a["S"], a["hidden"], a["nh"],
+                                      a["nkv"], a["hd"], a["theta"], a["q"], a["k"], a["v"], a["cap"],
+                                      a["dtype"], a["stream"])
+
+
+def _prefill(**kw):
+    a = dict(q=P, k=P, v=P, qpos=None, lens=P, B=2, S=4, nh=4, nkv=2, hd=64, cap=16, causal=1,
+             out=P, dtype=1, stream=None)
+    a.update(kw)
+    return gqa.lib().gqa_attn_prefill(a["q"], a["k"], a["v"], a["qpos"], a["lens"], a["B"], a["S"],
+                                      a["nh"], a["nkv"], a["hd"], a["cap"], a["causal"], a["out"],
+                                      a["dtype"], a["stream"])
+
+
+def _decode(**kw):
+    a = dict(q=P, k=P, v=P, lens=P, B=2, nh=4, nkv=2, hd=64, cap=16, split=0, out=P, ws=P,
+             ws_bytes=1 << 30, dtype=1, stream=None)
+    a.update(kw)
+    return gqa.lib().gqa_attn_decode(a["q"], a["k"], a["v"], a["lens"], a["B"], a["nh"], a["nkv"],
+                                     a["hd"], a["cap"], a["split"], a["out"], a["ws"], a["ws_bytes"],
+                                     a["dtype"], a["stream"])
+
+
+INVALID, MISALIGNED, DTYPE, ARCH, WS, LAUNCH, SHAPE, NODEV = -1, -2, -3, -4, -5, -6, -7, -8
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(x=None), INVALID), (dict(w=None), INVALID), (dict(pos=None), INVALID),
+    (dict(q=None), INVALID), (dict(k=None), INVALID), (dict(v=None), INVALID),
+    (dict(nh=6, nkv=4), INVALID), (dict(nkv=0), INVALID), (dict(B=-1), INVALID),
+    (dict(S=-3), INVALID), (dict(hidden=0), INVALID), (dict(cap=0), INVALID),
+    (dict(theta=0.0), INVALID), (dict(hd=96), SHAPE), (dict(hd=256), SHAPE), (dict(dtype=2), DTYPE),
+    (dict(x=MIS), MISALIGNED), (dict(k=MIS), MISALIGNED), (dict(pos=P + 2), MISALIGNED),
+])
+def test_qkv_rejects(kw, code):
+    assert _qkv(**kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), INVALID), (dict(lens=None), INVALID), (dict(out=None), INVALID),
+    (dict(nh=3, nkv=2), INVALID), (dict(cap=0), INVALID), (dict(hd=16), SHAPE),
+    (dict(dtype=-1), DTYPE), (dict(out=MIS), MISALIGNED), (dict(qpos=P + 1), MISALIGNED),
+])
+def test_prefill_rejects(kw, code):
+    assert _prefill(**kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), INVALID), (dict(lens=None), INVALID), (dict(split=100), INVALID),
+    (dict(split=-64), INVALID), (dict(nh=4, nkv=3), INVALID), (dict(hd=48), SHAPE),
+    (dict(ws_bytes=16), WS), (dict(ws=MIS), MISALIGNED), (dict(dtype=7), DTYPE),
+])
+def test_decode_rejects(kw, code):
+    assert _decode(**kw) == code
+
+
+def test_empty_inputs_are_noops():
+    # B == 0 or S == 0 returns OK without launching (pointers may then be NULL)
+    assert _qkv(B=0, x=None, w=None, pos=None, q=None, k=None, v=None) == 0
+    assert _qkv(S=0) == 0
+    assert _prefill(B=0, q=None) == 0
+    assert _prefill(S=0) == 0
+    assert _decode(B=0, q=None, ws=None) == 0
+
+
+def test_workspace_size_query():
+    f = gqa.gqa_attn_decode_workspace_size
+    # B * nh * ceil(cap / split) * (hd + 4) floats
+    assert f(2, 4, 2, 64, 1000, 64) == 2 * 4 * 16 * 68 * 4
+    assert f(64, 32, 8, 128, 8192, 512) == 64 * 32 * 16 * 132 * 4
+    assert f(2, 4, 2, 64, 1000, 0) > 0
+    assert f(2, 4, 2, 64, 1000, 100) == 0      # split not a multiple of 64
+    assert f(2, 4, 3, 64, 1000, 64) == 0       # nh % nkv
+    assert f(2, 4, 2, 80, 1000, 64) == 0       # head_dim
+
+
+def test_valid_call_without_gpu_reports_no_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; this case is for GPU-less hosts")
+    assert _qkv() in (NODEV, ARCH)
+    assert _prefill() in (NODEV, ARCH)
+    assert _decode() in (NODEV, ARCH)

@@ -1,0 +1,250 @@
+"""GPU parity: the CUDA library (called through its C ABI) against the float64
+oracle on the same seeded inputs.  Small cases are compared element by
+element; the five workloads run at their full sizes and are compared on
+sampled rows that the oracle computes one by one."""
+import numpy as np
+import pytest
+import torch
+
+import mqa_attention_qkv_b200 as gqa
+import workloads as W
+from oracle import gqa_ref as ref
+from tests._helpers import bits, dev, dev_i32, gate, host
+
+pytestmark = pytest.mark.gpu
+
+TORCH_DT = {"bf16": torch.bfloat16, "f32": torch.float32}
+SENTINEL = {"bf16": np.uint16(0x7FA5), "f32": np.uint32(0x7FC0_1234)}  # NaN payloads
+
+
+def sentinel_cache(shape, dtype):
+    if dtype == "bf16":
+        return W.Tensor(np.full(shape, SENTINEL["bf16"], dtype=np.uint16), "bf16")
+    return W.Tensor(np.full(shape, SENTINEL["f32"], dtype=np.uint32).view(np.float32), "f32")
+
+
+def nan_padded(B, nkv, cap, hd, lens, seed, tid, dtype):
+    return W.decode_cache(seed, tid, B, nkv, cap, hd, lens, dtype=dtype)
+
+
+def run_project(x, w, pos, nh, nkv, hd, cap, dtype, theta=10000.0, kc=None, vc=None):
+    B, S, _ = x.shape
+    xd, wd = dev(x), dev(w)
+    q = torch.empty((B, nh, S, hd), dtype=TORCH_DT[dtype], device="cuda")
+    kc = kc if kc is not None else dev(sentinel_cache((B, nkv, cap, hd), dtype))
+    vc = vc if vc is not None else dev(sentinel_cache((B, nkv, cap, hd), dtype))
+    gqa.qkv_rope_project(xd, wd, dev_i32(pos), nh, nkv, hd, theta, q, kc, vc)
+    return q, kc, vc
+
+
+# --------------------------------------------------------------------------
+# a1-a3: projection + RoPE + scatter
+# --------------------------------------------------------------------------
+QKV_CASES = [
+    # dtype, B, S, hidden, nh, nkv, hd, cap, scattered positions
+    ("f32", 1, 128, 256, 8, 2, 32, 128, False),
+    ("f32", 2, 19, 96, 4, 4, 64, 40, True),
+    ("bf16", 2, 37, 192, 4, 2, 64, 64, True),
+    ("bf16", 3, 130, 256, 8, 1, 128, 200, True),
+    ("bf16", 1, 5, 64, 2, 1, 32, 8, False),
+    ("bf16", 2, 200, 2048, 32, 4, 64, 256, False),
+    ("bf16", 1, 333, 520, 6, 2, 128, 400, True),
+]
+
+
+@pytest.mark.parametrize("case", QKV_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_qkv_rope_project_parity(case):
+    dtype, B, S, hidden, nh, nkv, hd, cap, scatter = case
+    shape = W.LayerShape(hidden, nh, nkv, hd)
+    x, w, pos = W.layer_inputs(shape, B, S, seed=11, dtype=dtype)
+    if scatter:
+        r = np.random.default_rng(5)
+        pos = np.stack([r.permutation(cap)[:S] for _ in range(B)]).astype(np.int32)
+    q, kc, vc = run_project(x, w, pos, nh, nkv, hd, cap, dtype)
+    sent = sentinel_cache((B, nkv, cap, hd), dtype)
+    q_ref, kc_ref, vc_ref = ref.qkv_rope_project(x.f64, w.f64, pos, nh, nkv, hd, 10000.0,
+                                                 np.zeros((B, nkv, cap, hd)), np.zeros((B, nkv, cap, hd)))
+    gate(host(q), q_ref, dtype, "q_out")
+    written = np.zeros((B, cap), dtype=bool)
+    for b in range(B):
+        written[b, pos[b]] = True
+    kh, vh = host(kc), host(vc)
+    for b in range(B):
+        gate(kh[b][:, written[b]], kc_ref[b][:, written[b]], dtype, "k_cache")
+        gate(vh[b][:, written[b]], vc_ref[b][:, written[b]], dtype, "v_cache")
+    # untouched slots keep their exact bits
+    kb, vb = bits(kc), bits(vc)
+    sb = sent.store.view(np.uint16 if dtype == "bf16" else np.uint32)
+    for b in range(B):
+        assert np.array_equal(kb[b][:, ~written[b]], sb[b][:, ~written[b]])
+        assert np.array_equal(vb[b][:, ~written[b]], sb[b][:, ~written[b]])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("hd", [32, 64, 128])
+def test_kv_cache_layout_bit_exact(dtype, hd):
+    """One-hot hidden states and small-integer weights make every projected
+    value an exact integer: V rows land bit-exactly at slot = position, K and Q
+    too for tokens at position 0 (rotation by zero)."""
+    B, S, D, nh, nkv, cap = 2, 9, 64, 4, 2, 24
+    N = (nh + 2 * nkv) * hd
+    w_int = ((np.arange(N * D).reshape(N, D) * 7919) % 61 - 30).astype(np.float32)
+    x_int = np.zeros((B, S, D), dtype=np.float32)
+    for b in range(B):
+        for s in range(S):
+            x_int[b, s, (3 * b + 5 * s) % D] = 1.0
+    x = W.Tensor(W.bf16_bits(x_int), "bf16") if dtype == "bf16" else W.Tensor(x_int, "f32")
+    w = W.Tensor(W.bf16_bits(w_int), "bf16") if dtype == "bf16" else W.Tensor(w_int, "f32")
+    pos = np.array([[0, 5, 9, 11, 13, 17, 19, 21, 23], [23, 0, 2, 4, 6, 8, 10, 12, 14]], dtype=np.int32)
+    q, kc, vc = run_project(x, w, pos, nh, nkv, hd, cap, dtype)
+    kh, vh, qh = host(kc), host(vc), host(q)
+    for b in range(B):
+        for s in range(S):
+            col = (3 * b + 5 * s) % D
+            p = pos[b, s]
+            v_want = w_int[(nh + nkv) * hd:, col].reshape(nkv, hd)
+            assert np.array_equal(vh[b, :, p], v_want), (b, s)
+            if p == 0:
+                assert np.array_equal(kh[b, :, p], w_int[nh * hd:(nh + nkv) * hd, col].reshape(nkv, hd))
+                assert np.array_equal(qh[b, :, s], w_int[:nh * hd, col].reshape(nh, hd))
+    # unwritten slots keep the sentinel bits
+    kb = bits(kc)
+    sent = SENTINEL[dtype]
+    for b in range(B):
+        free = sorted(set(range(cap)) - set(pos[b].tolist()))
+        assert np.all(kb[b][:, free] == sent)
+
+
+def test_out_of_range_position_sets_error_and_skips_row():
+    dtype, B, S, hidden, nh, nkv, hd, cap = "bf16", 1, 4, 64, 2, 1, 64, 8
+    x, w, _ = W.layer_inputs(W.LayerShape(hidden, nh, nkv, hd), B, S, seed=3, dtype=dtype)
+    pos = np.array([[0, 3, 8, -1]], dtype=np.int32)
+    gqa.gqa_device_error()  # clear
+    q, kc, vc = run_project(x, w, pos, nh, nkv, hd, cap, dtype)
+    assert gqa.gqa_device_error() & 1
+    kb = bits(kc)
+    assert np.all(kb[0, :, [1, 2, 4, 5, 6, 7]] == SENTINEL["bf16"])
+    assert np.all(np.isfinite(host(q)))
+
+
+# --------------------------------------------------------------------------
+# a4: prefill attention
+# --------------------------------------------------------------------------
+def attn_inputs(B, nh, nkv, S, hd, cap, lens, dtype, seed):
+    q = W.normal_tensor((B, nh, S, hd), seed, 0, dtype)
+    kc = nan_padded(B, nkv, cap, hd, lens, seed, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, lens, seed, 2, dtype)
+    return q, kc, vc
+
+
+PREFILL_CASES = []
+for _hd in (32, 64, 128):
+    for _g, _nkv in ((1, 2), (2, 2), (4, 2), (8, 1), (32, 1)):
+        for _S in (1, 7, 64, 129):
+            PREFILL_CASES.append(("bf16", _hd, _g * _nkv, _nkv, _S))
+PREFILL_CASES += [("f32", 32, 8, 2, 128), ("f32", 64, 4, 4, 37), ("f32", 128, 4, 1, 65)]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("case", PREFILL_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_prefill_parity(case, causal):
+    dtype, hd, nh, nkv, S = case
+    B = 2
+    lens = np.array([S + 3, S], dtype=np.int32)        # ragged; first has a 3-key prefix
+    cap = S + 11
+    q, kc, vc = attn_inputs(B, nh, nkv, S, hd, cap, lens, dtype, seed=S + hd)
+    out = torch.empty((B, S, nh, hd), dtype=TORCH_DT[dtype], device="cuda")
+    gqa.gqa_attn_prefill(dev(q), dev(kc), dev(vc), dev_i32(lens), causal, out)
+    want = ref.prefill_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens, causal)
+    gate(host(out), want, dtype, f"prefill {case} causal={causal}")
+
+
+def test_prefill_explicit_positions_and_empty_rows():
+    dtype, B, nh, nkv, S, hd, cap = "bf16", 2, 4, 2, 6, 64, 16
+    lens = np.array([10, 6], dtype=np.int32)
+    q, kc, vc = attn_inputs(B, nh, nkv, S, hd, cap, lens, dtype, seed=99)
+    qpos = np.array([[-1, 0, 2, 4, 9, 12], [5, 4, 3, 2, 1, 0]], dtype=np.int32)  # -1: no key; 12 > len
+    out = torch.empty((B, S, nh, hd), dtype=torch.bfloat16, device="cuda")
+    gqa.gqa_attn_prefill(dev(q), dev(kc), dev(vc), dev_i32(lens), True, out, q_positions=dev_i32(qpos))
+    want = ref.prefill_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens, True, q_positions=qpos)
+    got = host(out)
+    assert np.all(got[0, 0] == 0.0)
+    gate(got[:, 1:], want[:, 1:], dtype, "explicit positions")
+
+
+# --------------------------------------------------------------------------
+# a5-a6: decode
+# --------------------------------------------------------------------------
+def run_decode(q, kc, vc, lens, nh, dtype, kv_split=0):
+    B, _, hd = q.shape
+    nkv, cap = kc.shape[1], kc.shape[2]
+    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap, kv_split) // 4 + 1,
+                     dtype=torch.float32, device="cuda")
+    out = torch.empty((B, nh, hd), dtype=TORCH_DT[dtype], device="cuda")
+    gqa.gqa_attn_decode(dev(q), dev(kc), dev(vc), dev_i32(lens), out, ws, kv_split=kv_split)
+    return out
+
+
+DECODE_CASES = [(dt, hd, g, nkv) for dt in ("bf16",) for hd in (32, 64, 128)
+                for g, nkv in ((1, 4), (2, 2), (4, 2), (8, 1), (32, 1))]
+DECODE_CASES += [("f32", 32, 4, 2), ("f32", 128, 1, 2), ("f32", 64, 8, 1)]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_decode_parity(case):
+    dtype, hd, g, nkv = case
+    nh = g * nkv
+    lens = np.array([1, 63, 64, 65, 300, 1000, 7, 513], dtype=np.int32)
+    B, cap = len(lens), 1024
+    q = W.normal_tensor((B, nh, hd), 7, 0, dtype)
+    kc = nan_padded(B, nkv, cap, hd, lens, 7, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, lens, 7, 2, dtype)
+    want = ref.decode_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens)
+    for split in (0, 64, 192):
+        out = run_decode(q, kc, vc, lens, nh, dtype, kv_split=split)
+        gate(host(out), want, dtype, f"decode {case} split={split}")
+
+
+def test_decode_split_count_invariance():
+    """n_split in {1, 2, 7, max} agree to float32 rounding of the merge."""
+    dtype, hd, nh, nkv = "bf16", 128, 8, 1
+    lens = np.array([448, 448], dtype=np.int32)
+    B, cap = 2, 448
+    q = W.normal_tensor((B, nh, hd), 8, 0, dtype)
+    kc = nan_padded(B, nkv, cap, hd, lens, 8, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, lens, 8, 2, dtype)
+    outs = [host(run_decode(q, kc, vc, lens, nh, dtype, kv_split=s)) for s in (448, 256, 64)]
+    for o in outs[1:]:
+        assert np.max(np.abs(o - outs[0])) <= 2 ** -7 * np.max(np.abs(outs[0]))
+
+
+def test_decode_zero_and_clamped_lengths():
+    dtype, hd, nh, nkv, cap = "bf16", 64, 4, 2, 128
+    lens = np.array([0, 128, 5], dtype=np.int32)
+    q = W.normal_tensor((3, nh, hd), 9, 0, dtype)
+    kc = nan_padded(3, nkv, cap, hd, lens, 9, 1, dtype)
+    vc = nan_padded(3, nkv, cap, hd, lens, 9, 2, dtype)
+    gqa.gqa_device_error()
+    out = run_decode(q, kc, vc, lens, nh, dtype)
+    assert gqa.gqa_device_error() == 0
+    got = host(out)
+    assert np.all(got[0] == 0)
+    want = ref.decode_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens)
+    gate(got[1:], want[1:], dtype, "decode lens")
+    # a length above cap is clamped and flagged
+    over = run_decode(q, kc, vc, np.array([0, 500, 5], dtype=np.int32), nh, dtype)
+    assert gqa.gqa_device_error() & 2
+    gate(host(over)[1:], want[1:], dtype, "clamped")
+
+
+def test_prefill_last_row_equals_decode_on_gpu():
+    dtype, B, nh, nkv, S, hd = "bf16", 2, 8, 2, 77, 128
+    lens = np.array([S, S], dtype=np.int32)
+    q, kc, vc = attn_inputs(B, nh, nkv, S, hd, S, lens, dtype, seed=5)
+    out = torch.empty((B, S, nh, hd), dtype=torch.bfloat16, device="cuda")
+    gqa.gqa_attn_prefill(dev(q), dev(kc), dev(vc), dev_i32(lens), True, out)
+    qd = W.Tensor(np.ascontiguousarray(q.store[:, :, -1]), "bf16")
+    d = run_decode(qd, kc, vc, lens, nh, dtype)
+    want = ref.decode_attention(qd.f64, kc.f64, vc.f64, lens)
+    gate(host(d), want, dtype, "decode")
+    gate(host(out)[:, -1], want, dtype, "prefill last row")
