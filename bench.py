@@ -1,0 +1,436 @@
+"""Benchmark of the fused-QKV + grouped-query attention path on B200.
+
+One step = the whole path over one batch of the TinyLlama-1.1B-shaped layer
+(hidden 2048, 32 query heads, 4 KV heads, head_dim 64, bf16, RoPE theta 1e4):
+
+  1. qkv_rope_project   prompt  x [4, 2048, 2048] -> q, K/V cache slots 0..2047
+  2. gqa_attn_prefill   causal, 4 x 2048 queries over their 2048 keys
+  3. qkv_rope_project   one new token per sequence at position 2048
+  4. gqa_attn_decode    4 sequences x 32 heads over 2049 cached keys
+                        (split-KV partials + log-sum-exp combine)
+
+value = tokens processed per second (8192 prompt + 4 decode tokens per step,
+summed over all GPUs).  Inputs are seeded synthetic tensors resident in HBM;
+4 rotating input/output sets (~0.5 GB) keep every step's data out of L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the float64 CPU oracle (the correctness reference)
+on a bounded sample of the same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill attn TFLOPS & % BF16 peak; decode KV GB/s & % HBM; tokens/s per layer"
+WORKLOAD = dict(name="tinyllama-1.1b-layer-prefill4x2048+decode", B=4, S=2048, hidden=2048,
+                n_heads=32, n_kv_heads=4, head_dim=64, theta=10000.0, cap=2112, causal=True)
+N_ROT = 4
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_traffic():
+    """DRAM bytes per launch from an ncu capture (profiles/dram_traffic.txt),
+    valid only while the kernel source is unchanged (sha256 prefix)."""
+    out = {}
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return out
+    for line in open(p):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#"):
+            name, src, sha, nbytes = parts[:4]
+            fp = os.path.join(ROOT, "mqa_attention_qkv_b200", "csrc", src)
+            if os.path.exists(fp) and hashlib.sha256(open(fp, "rb").read()).hexdigest()[:12] == sha:
+                out[name] = float(nbytes)
+    return out
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], swp=f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        loaded = [r["sm"] for r in rows if r["power"] > 0.3 * max(x["power"] for x in rows)] or [r["sm"] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import mqa_attention_qkv_b200 as gqa
+    import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    wl = WORKLOAD
+    B, S, D, nh, nkv, hd, cap = (wl[k] for k in ("B", "S", "hidden", "n_heads", "n_kv_heads", "head_dim", "cap"))
+    shape = W.LayerShape(D, nh, nkv, hd, wl["theta"])
+    bf = torch.bfloat16
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+
+    def randn(*s, std=1.0):
+        return (torch.randn(*s, generator=gen, device=dev, dtype=torch.float32) * std).to(bf)
+
+    sets = []
+    for _ in range(N_ROT):
+        st = dict(
+            x=randn(B, S, D), w=randn(shape.n_qkv, D, std=0.02), x_dec=randn(B, 1, D),
+            q=torch.empty(B, nh, S, hd, dtype=bf, device=dev),
+            kc=torch.zeros(B, nkv, cap, hd, dtype=bf, device=dev),
+            vc=torch.zeros(B, nkv, cap, hd, dtype=bf, device=dev),
+            o=torch.empty(B, S, nh, hd, dtype=bf, device=dev),
+            q_dec=torch.empty(B, nh, 1, hd, dtype=bf, device=dev),
+            o_dec=torch.empty(B, nh, hd, dtype=bf, device=dev),
+        )
+        sets.append(st)
+    pos = torch.arange(S, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+    pos_dec = torch.full((B, 1), S, dtype=torch.int32, device=dev)
+    lens = torch.full((B,), S, dtype=torch.int32, device=dev)
+    lens_dec = torch.full((B,), S + 1, dtype=torch.int32, device=dev)
+    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    names = ("qkv_prefill", "attn_prefill", "qkv_decode", "attn_decode")
+
+    def step(st, evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        mark(0)
+        gqa.qkv_rope_project(st["x"], st["w"], pos, nh, nkv, hd, wl["theta"], st["q"], st["kc"], st["vc"], stream)
+        mark(1)
+        gqa.gqa_attn_prefill(st["q"], st["kc"], st["vc"], lens, True, st["o"], stream=stream)
+        mark(2)
+        gqa.qkv_rope_project(st["x_dec"], st["w"], pos_dec, nh, nkv, hd, wl["theta"], st["q_dec"], st["kc"], st["vc"], stream)
+        mark(3)
+        gqa.gqa_attn_decode(st["q_dec"].view(B, nh, hd), st["kc"], st["vc"], lens_dec, st["o_dec"], ws, stream=stream)
+        mark(4)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up
+    for i in range(args.warmup):
+        step(sets[i % N_ROT])
+    barrier()
+
+    # timed region: K steps; per-kernel events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    n0 = gqa.gqa_launch_count()
+    barrier()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(sets[i % N_ROT], evs[i])
+    t_end.record(stream)
+    barrier()
+    launches = gqa.gqa_launch_count() - n0
+    clk = clocks.stop()
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
+    per_kernel = {n: [evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)]
+                  for k, n in enumerate(names)}
+
+    tokens_per_step = B * S + B
+    ms_step = ms_total / args.steps
+    value = tokens_per_step * world * args.steps / (ms_total / 1e3)
+
+    # algorithmic work per launch
+    peaks, peak_src = load_peaks()
+    flops = {
+        "qkv_prefill": 2.0 * B * S * D * shape.n_qkv,
+        "attn_prefill": 4.0 * B * nh * S * S * hd / 2,           # causal counted as half
+    }
+    bytes_ = {
+        "qkv_decode": 2.0 * (shape.n_qkv * D + B * D + B * shape.n_qkv),
+        "attn_decode": 2.0 * (2 * B * nkv * (S + 1) * hd + 2 * B * nh * hd),
+    }
+    mean_ms = {n: statistics.mean(v) for n, v in per_kernel.items()}
+    dominant = max(mean_ms, key=mean_ms.get)
+    traffic = kernel_traffic()
+    bf16_peak = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+    hbm_peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+
+    def roof(n):
+        if n in flops:
+            a = flops[n] / (mean_ms[n] / 1e3) / 1e12
+            return {"bound": "tensor", "achieved": round(a, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                    "frac": round(a / bf16_peak, 4), "traffic": traffic.get(n), "kernel": n,
+                    "peak_source": f"{peak_src} bf16_tflops (burst)"}
+        a = bytes_[n] / (mean_ms[n] / 1e3) / 1e9
+        return {"bound": "hbm", "achieved": round(a, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(a / hbm_peak, 4), "traffic": traffic.get(n), "kernel": n,
+                "peak_source": f"{peak_src} hbm_gbs"}
+
+    roofline = roof(dominant)
+    kernels = {n: {"ms": round(mean_ms[n], 4), **{k: v for k, v in roof(n).items() if k in ("achieved", "unit", "frac")}}
+               for n in names}
+
+    # end to end through the public API: pinned host inputs -> device -> path -> host outputs
+    e2e = None
+    if not args.no_e2e:
+        hx = [sets[i]["x"].cpu().pin_memory() for i in range(N_ROT)]
+        hxd = [sets[i]["x_dec"].cpu().pin_memory() for i in range(N_ROT)]
+        ho = torch.empty(B, S, nh, hd, dtype=bf).pin_memory()
+        hod = torch.empty(B, nh, hd, dtype=bf).pin_memory()
+        hpos = pos.cpu().pin_memory()
+
+        def e2e_step(i):
+            st = sets[i % N_ROT]
+            st["x"].copy_(hx[i % N_ROT], non_blocking=True)
+            st["x_dec"].copy_(hxd[i % N_ROT], non_blocking=True)
+            pos.copy_(hpos, non_blocking=True)
+            step(st)
+            ho.copy_(st["o"], non_blocking=True)
+            hod.copy_(st["o_dec"], non_blocking=True)
+
+        for i in range(args.warmup):
+            e2e_step(i)
+        barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(args.steps):
+            e2e_step(i)
+        b_.record(stream)
+        barrier()
+        ms_e2e = max_over_ranks(a.elapsed_time(b_))
+        h2d = hx[0].numel() * 2 + hxd[0].numel() * 2 + hpos.numel() * 4
+        d2h = ho.numel() * 2 + hod.numel() * 2
+        e2e = {"value": round(tokens_per_step * world * args.steps / (ms_e2e / 1e3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(ms_e2e / args.steps, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(budget_s=args.cpu_budget)
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    attn = kernels["attn_prefill"]
+    dec = kernels["attn_decode"]
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) hidden states, N(0,0.02) weights)",
+        "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": S, "hidden": D,
+                   "n_heads": nh, "n_kv_heads": nkv, "head_dim": hd, "causal": True,
+                   "decode_kv_len": S + 1, "parallelism": f"replicas x{world}",
+                   "l2": f"{N_ROT} rotating input/output sets of ~{_set_mb(sets[0]):.0f} MB (> 126 MB L2)"},
+        "prefill_attn_tflops": attn["achieved"], "prefill_attn_frac_bf16_peak": attn["frac"],
+        "decode_kv_gbs": dec["achieved"], "decode_frac_hbm": dec["frac"],
+        "kernels": kernels, "roofline": roofline, "gpu_launches": int(launches),
+        "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+    }
+    print(json.dumps(line))
+
+
+def _set_mb(st):
+    return sum(t.numel() * t.element_size() for t in st.values()) / 1e6
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample_step(rows_per_seq: int, seed: int = 1):
+    """The float64 oracle on one of the workload's sequences: projection of its
+    2048 prompt tokens, causal attention for `rows_per_seq` evenly spaced query
+    rows (all 32 heads), then the decode step.  Returns tokens covered."""
+    import numpy as np
+
+    import workloads as W
+    from oracle import gqa_ref as ref
+    wl = WORKLOAD
+    S, nh, nkv, hd, cap = wl["S"], wl["n_heads"], wl["n_kv_heads"], wl["head_dim"], wl["cap"]
+    shape = W.LayerShape(wl["hidden"], nh, nkv, hd, wl["theta"])
+    x, w, pos = W.layer_inputs(shape, 1, S, seed=seed, dtype="bf16")
+    xd = W.hidden_states(shape, 1, 1, seed=seed, stream=1, dtype="bf16")
+    zeros = np.zeros((1, nkv, cap, hd))
+    q, kc, vc = ref.qkv_rope_project(x.f64, w.f64, pos, nh, nkv, hd, wl["theta"], zeros, zeros)
+    srows = np.linspace(0, S - 1, rows_per_seq).round().astype(int)
+    rows = [(0, h, int(s)) for h in range(nh) for s in srows]
+    ref.prefill_attention(q, kc, vc, np.array([S]), True, rows=rows)
+    qd, kc, vc = ref.qkv_rope_project(xd.f64, w.f64, np.array([[S]], dtype=np.int32), nh, nkv, hd,
+                                      wl["theta"], kc, vc)
+    ref.decode_attention(qd[:, :, 0], kc, vc, np.array([S + 1]))
+    return rows_per_seq + 1
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        th = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        th = 1
+    return th, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def cpu_baseline(budget_s: float = 20.0, rows_per_seq: int | None = None):
+    if rows_per_seq is None:
+        t0 = time.perf_counter()
+        oracle_sample_step(64)
+        dt = time.perf_counter() - t0
+        rows_per_seq = int(max(64, min(WORKLOAD["S"], 64 * budget_s / max(dt, 1e-3))))
+    t0 = time.perf_counter()
+    tok = oracle_sample_step(rows_per_seq)
+    dt = time.perf_counter() - t0
+    threads, affinity = _cores()
+    return {"value": round(tok / dt, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": (f"float64 numpy oracle, 1 of 4 sequences: projection of its 2048 prompt tokens, "
+                       f"causal attention of {rows_per_seq} evenly spaced query rows x 32 heads, "
+                       f"1 decode token; {dt:.1f} s; host affinity {affinity} cores"),
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    # size each step so that warm-up + timed steps stay within ~3 minutes
+    per_step_budget = max(1.0, 180.0 / max(1, args.steps + args.warmup))
+    t0 = time.perf_counter()
+    oracle_sample_step(16)
+    dt = time.perf_counter() - t0
+    rows = int(max(16, min(WORKLOAD["S"], 16 * per_step_budget / max(dt, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample_step(rows)
+    times, tok = [], 0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        tok += oracle_sample_step(rows)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = tok / total
+    threads, affinity = _cores()
+    cpu = {"value": round(value, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": (f"float64 numpy oracle per step: 1 sequence, projection of 2048 prompt tokens, "
+                      f"causal attention of {rows} evenly spaced query rows x 32 heads, 1 decode token; "
+                      f"host affinity {affinity} cores")}
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / max(1, args.steps), 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD["name"], "global_batch": WORKLOAD["B"], "seq_len": WORKLOAD["S"],
+                   "parallelism": "host cores"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, always
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -174,6 +174,13 @@ const char* gqa_status_string(int status);
  */
 int gqa_device_error(int* bits);
 
+/*
+ * gqa_launch_count - number of kernels this library has launched in this
+ * process (all devices, all streams).  A host-side counter: reading it does
+ * not touch the device.
+ */
+uint64_t gqa_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -16,7 +16,7 @@ __all__ = [
     "GQA_F32", "GQA_BF16", "GQAError", "library_path", "lib",
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
-    "EXPORTED_SYMBOLS",
+    "gqa_launch_count", "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -25,6 +25,7 @@ GQA_BF16 = 1
 EXPORTED_SYMBOLS = (
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
+    "gqa_launch_count",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -64,6 +65,8 @@ def lib() -> ctypes.CDLL:
     L.gqa_status_string.restype = ctypes.c_char_p
     L.gqa_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
     L.gqa_device_error.restype = i32
+    L.gqa_launch_count.argtypes = []
+    L.gqa_launch_count.restype = ctypes.c_uint64
     _LIB = L
     return L
 
@@ -182,3 +185,8 @@ def gqa_device_error() -> int:
     v = ctypes.c_int(0)
     _check("gqa_device_error", lib().gqa_device_error(ctypes.byref(v)))
     return v.value
+
+
+def gqa_launch_count() -> int:
+    """Kernels launched by the library so far in this process (host counter)."""
+    return int(lib().gqa_launch_count())

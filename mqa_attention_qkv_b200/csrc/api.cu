@@ -23,6 +23,7 @@ struct DeviceInfo {
   cudaError_t status = cudaSuccess;
 };
 DeviceInfo g_dev[kMaxDevices];
+std::atomic<unsigned long long> g_launches{0};
 
 // Per-device facts, queried once with that device current.
 const DeviceInfo* device_info(int* status) {
@@ -57,7 +58,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool hd_ok(int hd) { return hd == 32 || hd == 64 || hd == 128; }
 
-int launch_status(cudaError_t e) {
+int launch_status(cudaError_t e, int n_launched = 1) {
+  g_launches.fetch_add((unsigned long long)n_launched, std::memory_order_relaxed);
   if (e == cudaSuccess) return GQA_OK;
   cudaGetLastError();
   return GQA_ERR_LAUNCH_FAILED;
@@ -101,11 +103,14 @@ int gqa_device_error(int* bits) {
   int st;
   const DeviceInfo* d = device_info(&st);
   if (!d) return st;
-  if (cudaDeviceSynchronize() != cudaSuccess) return launch_status(cudaErrorUnknown);
   int v = 0;
-  if (cudaMemcpy(&v, d->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return launch_status(cudaErrorUnknown);
   const int zero = 0;
-  if (cudaMemcpy(d->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return launch_status(cudaErrorUnknown);
+  if (cudaDeviceSynchronize() != cudaSuccess ||
+      cudaMemcpy(&v, d->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(d->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_LAUNCH_FAILED;
+  }
   *bits = v;
   return GQA_OK;
 }
@@ -204,7 +209,9 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
   const bool bf16 = dtype == GQA_BF16;
   cudaError_t e = gqa::launch_decode_simt(p, bf16, s);
   if (e == cudaSuccess) e = gqa::launch_decode_combine(p, bf16, s);
-  return launch_status(e);
+  return launch_status(e, 2);
 }
+
+uint64_t gqa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

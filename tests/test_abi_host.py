@@ -20,7 +20,7 @@ MIS = P + 8
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|size_t|char\s*\*|void)\s*\*?\s*(\w+)\s*\(",
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|size_t|uint64_t|char\s*\*|void)\s*\*?\s*(\w+)\s*\(",
                                  src, flags=re.M)))
 
 
