@@ -164,6 +164,31 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                     int cache_cap, int kv_split, void* out, void* workspace,
                     size_t workspace_bytes, int dtype, void* stream);
 
+/*
+ * gqa_attn_decode_noalloc - gqa_attn_decode without a workspace argument.
+ *
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory where they run decode: a serving loop whose
+ * device memory is all pre-reserved by another allocator, a plugin that its
+ * host framework hands only the op's tensors (no allocator interface), or a
+ * latency-critical path on which an allocation, which may synchronise the
+ * device, is not allowed.  The caller still passes every input and output;
+ * arguments, layouts, results and errors are those of gqa_attn_decode.
+ *
+ * The split-KV partials live in a fixed 64 MiB array of static device memory
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits.  A problem whose partials (gqa_attn_decode_workspace_size)
+ * exceed 64 MiB is rejected with GQA_ERR_WORKSPACE_TOO_SMALL; a larger
+ * kv_split needs fewer partials.  The first call on each device looks up the
+ * array's device address (with that device current), so make that first call
+ * before any stream capture.  All calls share the array and nothing in it has
+ * to start at zero; calls that overlap on the GPU (e.g. on two streams) race,
+ * so order them on one stream or with events.  It allocates nothing.
+ */
+int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,
+                            int cache_cap, int kv_split, void* out, int dtype, void* stream);
+
 /* Human-readable text of a gqa_status value (static storage). */
 const char* gqa_status_string(int status);
 

@@ -16,7 +16,7 @@ __all__ = [
     "GQA_F32", "GQA_BF16", "GQAError", "library_path", "lib",
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
-    "gqa_launch_count", "EXPORTED_SYMBOLS",
+    "gqa_launch_count", "gqa_attn_decode_noalloc", "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -25,7 +25,7 @@ GQA_BF16 = 1
 EXPORTED_SYMBOLS = (
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
-    "gqa_launch_count",
+    "gqa_launch_count", "gqa_attn_decode_noalloc",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
     L.gqa_device_error.restype = i32
     L.gqa_launch_count.argtypes = []
     L.gqa_launch_count.restype = ctypes.c_uint64
+    L.gqa_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+    L.gqa_attn_decode_noalloc.restype = i32
     _LIB = L
     return L
 
@@ -190,3 +192,21 @@ def gqa_device_error() -> int:
 def gqa_launch_count() -> int:
     """Kernels launched by the library so far in this process (host counter)."""
     return int(lib().gqa_launch_count())
+
+
+def gqa_attn_decode_noalloc(q, k_cache, v_cache, kv_lens, out, kv_split: int = 0, stream=None) -> None:
+    """gqa_attn_decode for callers that cannot allocate device memory: the
+    split-KV scratch is a fixed 64 MiB static array inside the library (see
+    include/gqa.h).  Same shapes and results as gqa_attn_decode."""
+    import torch
+    B, nh, hd = q.shape
+    nkv, cap = k_cache.shape[1], k_cache.shape[2]
+    dt = q.dtype
+    args = (
+        _ptr(q, dt, name="q"), _ptr(k_cache, dt, (B, nkv, cap, hd), "k_cache"),
+        _ptr(v_cache, dt, (B, nkv, cap, hd), "v_cache"),
+        _ptr(kv_lens, torch.int32, (B,), "kv_lens"),
+        B, nh, nkv, hd, cap, int(kv_split),
+        _ptr(out, dt, (B, nh, hd), "out"), _dtype_code(q), _stream(stream),
+    )
+    _check("gqa_attn_decode_noalloc", lib().gqa_attn_decode_noalloc(*args))

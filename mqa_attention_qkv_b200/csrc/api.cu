@@ -81,6 +81,23 @@ constexpr long long kMaxElems = 1ll << 40;
 
 }  // namespace
 
+namespace gqa {
+
+int device_check(int** err) {
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (d && err) *err = d->err;
+  return st;
+}
+
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+int decode_split_len(int B, int n_kv_heads, int cache_cap, int kv_split) {
+  return kv_split ? kv_split : auto_split(B, n_kv_heads, cache_cap);
+}
+
+}  // namespace gqa
+
 extern "C" {
 
 const char* gqa_status_string(int status) {

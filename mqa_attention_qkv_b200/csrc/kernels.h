@@ -51,4 +51,9 @@ cudaError_t launch_prefill_simt(const PrefillParams& p, bool bf16, cudaStream_t 
 cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t st);
 
+// Shared by the C-ABI translation units (defined in api.cu).
+int device_check(int** err);  // GQA_OK, or the status for the current device
+void count_launches(int n);
+int decode_split_len(int B, int n_kv_heads, int cache_cap, int kv_split);
+
 }  // namespace gqa
