@@ -157,6 +157,8 @@ int qkv_rope_project(const void* x, const void* w_qkv, const int32_t* positions,
   gqa::QkvParams p{x, w_qkv, positions, B, S, hidden, n_heads, n_kv_heads, head_dim, cache_cap,
                    (double)rope_theta, q_out, k_cache, v_cache, d->err};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Tensor-core path: bf16 with 16-byte-aligned rows (TMA row stride).
+  if (dtype == GQA_BF16 && hidden % 8 == 0) return launch_status(gqa::launch_qkv_tc(p, d->num_sms, s));
   return launch_status(gqa::launch_qkv_simt(p, dtype == GQA_BF16, s));
 }
 

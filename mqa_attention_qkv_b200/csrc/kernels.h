@@ -51,6 +51,14 @@ cudaError_t launch_prefill_simt(const PrefillParams& p, bool bf16, cudaStream_t 
 cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t st);
 
+// Tensor-core (tcgen05 + TMA) kernels, bf16 only.
+cudaError_t launch_qkv_tc(const QkvParams& p, int num_sms, cudaStream_t st);
+
+// 2-D bf16 TMA descriptor with 128-byte swizzle; `map` points at a CUtensorMap.
+// Zero fill outside [0, inner) x [0, outer).  False if encoding fails.
+bool make_tmap_bf16_2d(void* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                       uint32_t box_inner, uint32_t box_outer);
+
 // Shared by the C-ABI translation units (defined in api.cu).
 int device_check(int** err);  // GQA_OK, or the status for the current device
 void count_launches(int n);

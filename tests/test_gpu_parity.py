@@ -49,6 +49,9 @@ QKV_CASES = [
     ("bf16", 1, 5, 64, 2, 1, 32, 8, False),
     ("bf16", 2, 200, 2048, 32, 4, 64, 256, False),
     ("bf16", 1, 333, 520, 6, 2, 128, 400, True),
+    ("bf16", 3, 150, 136, 3, 1, 64, 160, True),     # N = 320 (partial 256-tile), K tail, T = 450
+    ("bf16", 2, 300, 256, 12, 2, 32, 320, False),   # hd 32: 8 heads per tile
+    ("bf16", 2, 70, 100, 4, 2, 64, 80, True),       # hidden % 8 != 0: the SIMT path
 ]
 
 
