@@ -185,6 +185,8 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
   gqa::PrefillParams p{q, k_cache, v_cache, q_positions, kv_lens, B, S, n_heads, n_kv_heads,
                        head_dim, cache_cap, causal ? 1 : 0, out, d->err};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == GQA_BF16 && (head_dim == 64 || head_dim == 128))
+    return launch_status(gqa::launch_prefill_tc(p, s));
   return launch_status(gqa::launch_prefill_simt(p, dtype == GQA_BF16, s));
 }
 

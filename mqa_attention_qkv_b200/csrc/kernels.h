@@ -53,6 +53,7 @@ cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t
 
 // Tensor-core (tcgen05 + TMA) kernels, bf16 only.
 cudaError_t launch_qkv_tc(const QkvParams& p, int num_sms, cudaStream_t st);
+cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t st);  // head_dim 64 or 128
 
 // 2-D bf16 TMA descriptor with 128-byte swizzle; `map` points at a CUtensorMap.
 // Zero fill outside [0, inner) x [0, outer).  False if encoding fails.
