@@ -41,8 +41,21 @@ import numpy as np
 __all__ = [
     "fused_projection", "split_qkv", "rope_inv_freq", "apply_rope",
     "qkv_rope_project", "kv_head_of", "softmax", "attend_row",
-    "prefill_attention", "decode_attention", "default_q_positions",
+    "prefill_attention", "decode_attention", "default_q_positions", "round_bf16",
 ]
+
+
+# --------------------------------------------------------------------------
+# storage type between calls
+# --------------------------------------------------------------------------
+def round_bf16(a: np.ndarray) -> np.ndarray:
+    """Round to the nearest bfloat16 value (8 significant bits, ties to even).
+
+    The path stores q, K and V in the call's dtype between calls; chained
+    expectations apply this to what one call stores before the next reads it."""
+    a = np.asarray(a, dtype=np.float64)
+    m, e = np.frexp(a)                       # a = m * 2**e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
 
 
 # --------------------------------------------------------------------------

@@ -523,3 +523,27 @@ def test_planted_off_by_one_causal_is_caught(monkeypatch):
     orig = ref.default_q_positions
     monkeypatch.setattr(ref, "default_q_positions", lambda kv, S: orig(kv, S) - 1)
     assert _fails(check_last_causal_row_equals_decode)
+
+
+# --------------------------------------------------------------------------
+# bf16 storage rounding used for chained expectations
+# --------------------------------------------------------------------------
+def test_round_bf16_matches_bit_level_rounding():
+    """Independent route: float32 bits rounded to nearest-even in the input
+    module (integer arithmetic) versus frexp/rint here."""
+    import workloads as W
+    r = rng(30)
+    a = np.concatenate([r.standard_normal(200000), r.standard_normal(1000) * 1e4,
+                        r.standard_normal(1000) * 1e-4]).astype(np.float32)
+    want = W.bf16_to_f32(W.bf16_bits(a)).astype(np.float64)
+    np.testing.assert_array_equal(ref.round_bf16(a.astype(np.float64)), want)
+
+
+def test_round_bf16_exact_and_ties_to_even():
+    exact = np.array([1.0, -2.0, 1.5, 0.00390625, 3.0 * 2 ** 40, 1 + 2 ** -7])
+    np.testing.assert_array_equal(ref.round_bf16(exact), exact)
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: ties go to the even mantissa (1.0)
+    assert ref.round_bf16(np.array([1 + 2 ** -8]))[0] == 1.0
+    assert ref.round_bf16(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
+    a = rng(31).standard_normal(10000) * 37
+    assert np.max(np.abs(ref.round_bf16(a) - a) / np.abs(a)) <= 2 ** -8
