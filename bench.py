@@ -165,6 +165,7 @@ def run_ours(args):
             o_dec=torch.empty(B, nh, hd, dtype=bf, device=dev),
         )
         sets.append(st)
+    set_mb = _set_mb(sets[0])
     pos = torch.arange(S, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
     pos_dec = torch.full((B, 1), S, dtype=torch.int32, device=dev)
     lens = torch.full((B,), S, dtype=torch.int32, device=dev)
@@ -295,6 +296,10 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(budget_s=args.cpu_budget)
+    wls = None
+    if rank == 0 and world == 1 and not args.no_workloads:
+        del sets
+        wls = measure_workloads(dev, {"hbm_gbs": hbm_peak, "bf16_tflops": bf16_peak})
 
     if world > 1:
         dist.barrier(device_ids=[local])
@@ -311,17 +316,152 @@ def run_ours(args):
         "config": {"workload": wl["name"], "global_batch": B * world, "seq_len": S, "hidden": D,
                    "n_heads": nh, "n_kv_heads": nkv, "head_dim": hd, "causal": True,
                    "decode_kv_len": S + 1, "parallelism": f"replicas x{world}",
-                   "l2": f"{N_ROT} rotating input/output sets of ~{_set_mb(sets[0]):.0f} MB (> 126 MB L2)"},
+                   "l2": f"{N_ROT} rotating input/output sets of ~{set_mb:.0f} MB (> 126 MB L2)"},
         "prefill_attn_tflops": attn["achieved"], "prefill_attn_frac_bf16_peak": attn["frac"],
         "decode_kv_gbs": dec["achieved"], "decode_frac_hbm": dec["frac"],
         "kernels": kernels, "roofline": roofline, "gpu_launches": int(launches),
-        "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+        "clocks": clk, "e2e": e2e, "cpu_baseline": cpu, "workloads": wls,
     }
     print(json.dumps(line))
 
 
 def _set_mb(st):
     return sum(t.numel() * t.element_size() for t in st.values()) / 1e6
+
+
+# ---------------------------------------------------------------------------
+# the other workloads of the metric, measured kernel by kernel
+# ---------------------------------------------------------------------------
+def measure_workloads(dev, peaks, iters=10):
+    """Llama-2-7B-shaped batched decode (B 64, 32 query heads, hd 128, ragged
+    KV 512..8192, MHA/GQA/MQA caches): KV GB/s; 8K-token prefill (B 2, 16
+    heads, hd 128, KV heads 16/4, causal and not): TFLOP/s; the MQA generation
+    loop (B 8, hidden 6144, 48 heads, 1 KV head, prompt 16 + 1024 steps):
+    tokens/s.  Each kernel is timed alone with CUDA events, L2 flushed before
+    every timed call (a 512 MB write), median of `iters`."""
+    import numpy as np
+    import torch
+
+    import mqa_attention_qkv_b200 as gqa
+    import workloads as W
+
+    bf = torch.bfloat16
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+
+    def timed(fn):
+        ts = []
+        for i in range(iters + 2):
+            flush.fill_(i & 0xFF)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            if i >= 2:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    out = {}
+    hbm, bf16_peak = peaks["hbm_gbs"], peaks["bf16_tflops"]
+
+    # ---- batched decode
+    wl = W.LLAMA2_DECODE
+    e = wl.extra
+    B, nh, hd, cap = e["batch"], wl.shape.n_heads, wl.shape.head_dim, e["cap"]
+    lens_np = W.ragged_lengths(B, e["kv_lo"], e["kv_hi"], wl.seed)
+    lens = torch.from_numpy(lens_np).to(dev)
+    q = torch.randn(B, nh, hd, generator=gen, device=dev).to(bf)
+    dec = {}
+    for nkv in e["n_kv_heads_cases"]:
+        kc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
+        vc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
+        o = torch.empty(B, nh, hd, dtype=bf, device=dev)
+        ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: gqa.gqa_attn_decode(q, kc, vc, lens, o, ws, stream=stream))
+        nbytes = 2.0 * (2 * nkv * hd * float(lens_np.sum()) + 2 * B * nh * hd)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        dec[f"nkv{nkv}"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                            "bytes": int(nbytes)}
+        del kc, vc
+    out["llama2_decode_b64"] = dec
+
+    # ---- long-context prefill
+    wl = W.LONG_PREFILL
+    B, S = wl.batch_seq[0]
+    nh, hd = wl.shape.n_heads, wl.shape.head_dim
+    lp = {}
+    for nkv in wl.extra["n_kv_heads_cases"]:
+        q = torch.randn(B, nh, S, hd, generator=gen, device=dev).to(bf)
+        k = torch.randn(B, nkv, S, hd, generator=gen, device=dev).to(bf)
+        v = torch.randn(B, nkv, S, hd, generator=gen, device=dev).to(bf)
+        o = torch.empty(B, S, nh, hd, dtype=bf, device=dev)
+        ln = torch.full((B,), S, dtype=torch.int32, device=dev)
+        for causal in (True, False):
+            ms = timed(lambda: gqa.gqa_attn_prefill(q, k, v, ln, causal, o, stream=stream))
+            fl = 4.0 * B * nh * S * S * hd * (0.5 if causal else 1.0)
+            tf = fl / (ms / 1e3) / 1e12
+            lp[f"nkv{nkv}_{'causal' if causal else 'full'}"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                                                 "frac_bf16": round(tf / bf16_peak, 4)}
+    out["long_prefill_2x8192"] = lp
+
+    # ---- MQA generation loop (prompt 16, 1024 steps), one timed region
+    wl = W.MQA_GENERATE
+    sh, e = wl.shape, wl.extra
+    B, P, T, cap = e["batch"], e["prompt"], e["steps"], e["cap"]
+    nh, nkv, hd = sh.n_heads, sh.n_kv_heads, sh.head_dim
+    w = (torch.randn(sh.n_qkv, sh.hidden, generator=gen, device=dev) * 0.02).to(bf)
+    xp = torch.randn(B, P, sh.hidden, generator=gen, device=dev).to(bf)
+    xs = torch.randn(T, B, 1, sh.hidden, generator=gen, device=dev).to(bf)
+    kc = torch.zeros(B, nkv, cap, hd, dtype=bf, device=dev)
+    vc = torch.zeros_like(kc)
+    qp = torch.empty(B, nh, P, hd, dtype=bf, device=dev)
+    op = torch.empty(B, P, nh, hd, dtype=bf, device=dev)
+    qt = torch.empty(B, nh, 1, hd, dtype=bf, device=dev)
+    ot = torch.empty(T, B, nh, hd, dtype=bf, device=dev)
+    posp = torch.arange(P, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+    pos_steps = (P + torch.arange(T, dtype=torch.int32, device=dev)).view(T, 1, 1).expand(T, B, 1).contiguous()
+    len_steps = (P + 1 + torch.arange(T, dtype=torch.int32, device=dev)).view(T, 1).expand(T, B).contiguous()
+    lp_ = torch.full((B,), P, dtype=torch.int32, device=dev)
+    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
+
+    def gen_loop():
+        st = torch.cuda.current_stream(dev)   # the capture stream while a graph is being recorded
+        gqa.qkv_rope_project(xp, w, posp, nh, nkv, hd, sh.rope_theta, qp, kc, vc, st)
+        gqa.gqa_attn_prefill(qp, kc, vc, lp_, True, op, stream=st)
+        for t in range(T):
+            gqa.qkv_rope_project(xs[t], w, pos_steps[t], nh, nkv, hd, sh.rope_theta, qt, kc, vc, st)
+            gqa.gqa_attn_decode(qt.view(B, nh, hd), kc, vc, len_steps[t], ot[t], ws, stream=st)
+
+    gen_loop()
+    ms_direct = timed_once(gen_loop, stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        gen_loop()
+    graph.replay()
+    ms_graph = timed_once(graph.replay, stream)
+    toks = B * (P + T)
+    per_step_bytes = 2.0 * sh.n_qkv * sh.hidden
+    out["mqa_generate_b8_p16_g1024"] = {
+        "ms_direct": round(ms_direct, 3), "ms_graph": round(ms_graph, 3),
+        "tokens_per_s_direct": round(toks / (ms_direct / 1e3), 1),
+        "tokens_per_s_graph": round(toks / (ms_graph / 1e3), 1),
+        "weight_stream_GB/s_graph": round(per_step_bytes * T / (ms_graph / 1e3) / 1e9, 1),
+        "note": "W_qkv (78.6 MB) is re-read every step and may stay partly L2-resident across steps"}
+    del graph
+    return out
+
+
+def timed_once(fn, stream):
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    fn()
+    b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b)
 
 
 # ---------------------------------------------------------------------------
@@ -423,6 +563,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-kernel measurements of the decode, 8K-prefill and generation workloads")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, always

@@ -185,8 +185,8 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
   gqa::PrefillParams p{q, k_cache, v_cache, q_positions, kv_lens, B, S, n_heads, n_kv_heads,
                        head_dim, cache_cap, causal ? 1 : 0, out, d->err};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dtype == GQA_BF16 && (head_dim == 64 || head_dim == 128))
-    return launch_status(gqa::launch_prefill_tc(p, s));
+  if (dtype == GQA_BF16 && head_dim == 64) return launch_status(gqa::launch_prefill_pair(p, s));
+  if (dtype == GQA_BF16 && head_dim == 128) return launch_status(gqa::launch_prefill_tc(p, s));
   return launch_status(gqa::launch_prefill_simt(p, dtype == GQA_BF16, s));
 }
 
@@ -228,9 +228,7 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                       d->err};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == GQA_BF16;
-  cudaError_t e = gqa::launch_decode_simt(p, bf16, s);
-  if (e == cudaSuccess) e = gqa::launch_decode_combine(p, bf16, s);
-  return launch_status(e, 2);
+  return launch_status(gqa::launch_decode(p, bf16, s), 2);
 }
 
 uint64_t gqa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

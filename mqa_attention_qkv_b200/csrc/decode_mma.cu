@@ -1,0 +1,322 @@
+// Split-KV decode attention (step a5, bf16, head_dim 64 or 128).
+//
+// Decode reads each cached K/V row once per new token and does g
+// multiply-adds per byte: it is HBM-bound (MHA -> GQA blog, sections
+// 3.1-3.2).  The g query heads that share a KV head are stacked as the rows
+// of one tensor-core tile, so one pass over a K/V row serves all g heads and
+// GQA's arithmetic intensity ~g is actually used.  tcgen05 wants M >= 64; for
+// g <= 16 that would multiply the tensor work 4-16x for nothing, and this
+// kernel's tensor work is far below the tensor roofline anyway, so it uses
+// mma.sync m16n8k16 with the (up to 16) heads as M.
+//
+// CTA = (sequence b, KV head j, key split c, group of <= 16 heads).  5 warps:
+//   warp 4     TMA producer: 64-key K and V tiles (128-byte swizzle, so the
+//              ldmatrix reads below are conflict free) into a 3-4 stage ring
+//   warps 0-3  each takes 16 keys of every tile: S = Q K^T (Q fragments in
+//              registers), mask keys >= the split end, online softmax in
+//              log2 units, P kept in registers as the A fragment of
+//              O += P V (V through ldmatrix.trans).  V rows past the valid
+//              keys are zeroed first so NaN padding never meets a zero P.
+// At the end the 4 warps' (m, l, O) are merged through shared memory and one
+// partial (o unnormalised, m, l) per head is written for the combine.
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr int KT = 64;          // keys per tile
+constexpr int THREADS = 160;    // 4 consumer warps + 1 producer warp
+
+template <int HD>
+struct DCfg {
+  static constexpr int STAGES = HD == 128 ? 3 : 4;
+  static constexpr int NBOX = HD / 64;
+  static constexpr int BOX_BYTES = KT * 128;               // 64 rows x 128 bytes
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;      // one K or V tile
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int RED_STRIDE = HD + 4;                // fp32 merge rows
+  static constexpr int RED_BYTES = 4 * 16 * RED_STRIDE * 4;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES > RED_BYTES ? STAGES * STAGE_BYTES : RED_BYTES;
+  static constexpr int SMEM = RING_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// byte offset of element (row, col) inside a tile of 64-row x 64-column
+// swizzled boxes (128-byte rows, 16-byte chunk c stored at c ^ (row & 7))
+__device__ __forceinline__ uint32_t swz(int row, int col) {
+  return (uint32_t)((col >> 6) * (KT * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
+}
+
+struct Bars {
+  uint64_t full[4], empty[4];
+  float ml[4][16][2];
+};
+
+template <int HD>
+__global__ void __launch_bounds__(THREADS)
+decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                  DecodeParams p, int n_hgrp) {
+  using C = DCfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::RING_BYTES);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int b = blockIdx.z, j = blockIdx.y;
+  const int split = blockIdx.x / n_hgrp, hg = blockIdx.x % n_hgrp;
+  const int g = p.nh / p.nkv;
+  int* err = p.err;
+
+  int kv_len = p.kv_lens[b];
+  if (kv_len > p.cap || kv_len < 0) {
+    if (threadIdx.x == 0 && split == 0 && hg == 0) raise_error(err, GQA_DEVERR_KVLEN_RANGE);
+    kv_len = kv_len > p.cap ? p.cap : 0;
+  }
+  const int k_lo = split * p.split;
+  if (k_lo >= kv_len) return;  // no key of this sequence in this split (whole block)
+  const int k_hi = min(kv_len, k_lo + p.split);
+  const int n_t = (k_hi - k_lo + KT - 1) / KT;
+  const int h0 = j * g + hg * 16;
+  const int rows = min(16, g - hg * 16);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 4);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmk);
+      tc::prefetch_tmap(&tmv);
+      const int row0 = (b * p.nkv + j) * p.cap + k_lo;
+      for (int t = 0; t < n_t; ++t) {
+        const int s = t % C::STAGES;
+        if (!mbar_wait(&bars->empty[s], ((t / C::STAGES) & 1) ^ 1, err)) break;
+        mbar_arrive_expect_tx(&bars->full[s], C::STAGE_BYTES);
+        uint8_t* kt = smem + s * C::STAGE_BYTES;
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          tc::tma_load_2d(kt + bx * C::BOX_BYTES, &tmk, bx * 64, row0 + t * KT, &bars->full[s]);
+          tc::tma_load_2d(kt + C::TILE_BYTES + bx * C::BOX_BYTES, &tmv, bx * 64, row0 + t * KT, &bars->full[s]);
+        }
+      }
+      // every issued load has landed before the block may exit
+      for (int t = max(0, n_t - C::STAGES); t < n_t; ++t)
+        mbar_wait(&bars->full[t % C::STAGES], (t / C::STAGES) & 1, err);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int gr = lane >> 2, tq = lane & 3;  // fragment row group / thread in quad
+  // Q fragments for all K steps (rows gr and gr + 8 of this head group)
+  uint32_t qa[HD / 16][4];
+  {
+    const uint32_t* q32 = static_cast<const uint32_t*>(p.q);
+    const size_t r0 = ((size_t)b * p.nh + h0 + gr) * (HD / 2), r1 = r0 + 8 * (HD / 2);
+#pragma unroll
+    for (int ks = 0; ks < HD / 16; ++ks) {
+      const int c = ks * 8 + tq;  // bf16x2 column index
+      qa[ks][0] = gr < rows ? q32[r0 + c] : 0u;
+      qa[ks][1] = gr + 8 < rows ? q32[r1 + c] : 0u;
+      qa[ks][2] = gr < rows ? q32[r0 + c + 4] : 0u;
+      qa[ks][3] = gr + 8 < rows ? q32[r1 + c + 4] : 0u;
+    }
+  }
+  const float scale_log2 = 1.4426950408889634f * rsqrtf((float)HD);
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float o[HD / 8][4];
+#pragma unroll
+  for (int n = 0; n < HD / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+
+  const int mrow = lane & 7, mat = lane >> 3;  // ldmatrix: row within matrix, matrix index
+  for (int t = 0; t < n_t; ++t) {
+    const int s = t % C::STAGES;
+    const bool ok = mbar_wait(&bars->full[s], (t / C::STAGES) & 1, err);
+    if (!__all_sync(0xffffffffu, ok)) break;
+    const uint32_t kbase = smem_u32(smem + s * C::STAGE_BYTES);
+    const uint32_t vbase = kbase + C::TILE_BYTES;
+    const int slab = warp * 16;                         // first tile row of this warp
+    const int nvalid = min(16, max(0, k_hi - (k_lo + t * KT + slab)));
+    if (nvalid > 0) {
+      if (nvalid < 16) {
+        // zero V rows [nvalid, 16) of this warp's slab (whole 128-byte rows)
+        for (int e = lane; e < (16 - nvalid) * 8 * C::NBOX; e += 32) {
+          const int r = slab + nvalid + e / (8 * C::NBOX);
+          const int rem = e % (8 * C::NBOX);
+          tc::st_shared_v4(vbase + (rem / 8) * C::BOX_BYTES + r * 128 + (rem % 8) * 16, 0u, 0u, 0u, 0u);
+        }
+        tc::fence_proxy_async_smem();  // ordered before the next TMA write into this stage
+        __syncwarp();
+      }
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < HD / 16; ++ks) {
+        // matrices: (keys 0-7, k lo), (keys 0-7, k hi), (keys 8-15, k lo), (keys 8-15, k hi)
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kbase + swz(slab + (mat >> 1) * 8 + mrow, ks * 16 + (mat & 1) * 8), b0, b1, b2, b3);
+        mma16816(sc[0], qa[ks], b0, b1);
+        mma16816(sc[1], qa[ks], b2, b3);
+      }
+      // scale to log2 units and mask keys past the valid range
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = nt * 8 + 2 * tq + (e & 1);
+          const float v = key < nvalid ? sc[nt][e] * scale_log2 : -INFINITY;
+          sc[nt][e] = v;
+          if (e < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+        }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);   // finite: key 0 of the slab is valid
+      const float al0 = tc::ex2(m0 - mn0), al1 = tc::ex2(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        sc[nt][0] = tc::ex2(sc[nt][0] - mn0);
+        sc[nt][1] = tc::ex2(sc[nt][1] - mn0);
+        sc[nt][2] = tc::ex2(sc[nt][2] - mn1);
+        sc[nt][3] = tc::ex2(sc[nt][3] - mn1);
+        s0 += sc[nt][0] + sc[nt][1];
+        s1 += sc[nt][2] + sc[nt][3];
+      }
+      s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+      s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+      l0 = l0 * al0 + s0;
+      l1 = l1 * al1 + s1;
+#pragma unroll
+      for (int n = 0; n < HD / 8; ++n) {
+        o[n][0] *= al0;
+        o[n][1] *= al0;
+        o[n][2] *= al1;
+        o[n][3] *= al1;
+      }
+      const uint32_t pa[4] = {pack_bf16x2(sc[0][0], sc[0][1]), pack_bf16x2(sc[0][2], sc[0][3]),
+                              pack_bf16x2(sc[1][0], sc[1][1]), pack_bf16x2(sc[1][2], sc[1][3])};
+#pragma unroll
+      for (int np = 0; np < HD / 16; ++np) {
+        // matrices: (keys 0-7, cols 0-7), (keys 8-15, cols 0-7), (keys 0-7, cols 8-15), (keys 8-15, cols 8-15)
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vbase + swz(slab + (mat & 1) * 8 + mrow, np * 16 + (mat >> 1) * 8), b0, b1, b2, b3);
+        mma16816(o[2 * np], pa, b0, b1);
+        mma16816(o[2 * np + 1], pa, b2, b3);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->empty[s]);
+  }
+
+  // ------------------------------------------------------------------ merge the 4 warps
+  if (tq == 0) {
+    bars->ml[warp][gr][0] = m0;
+    bars->ml[warp][gr][1] = l0;
+    bars->ml[warp][gr + 8][0] = m1;
+    bars->ml[warp][gr + 8][1] = l1;
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");   // consumers only; the ring is idle now
+  float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    M0 = fmaxf(M0, bars->ml[w][gr][0]);
+    M1 = fmaxf(M1, bars->ml[w][gr + 8][0]);
+  }
+  const float f0 = m0 == -INFINITY ? 0.f : tc::ex2(m0 - M0);
+  const float f1 = m1 == -INFINITY ? 0.f : tc::ex2(m1 - M1);
+  float* red = reinterpret_cast<float*>(smem);
+#pragma unroll
+  for (int n = 0; n < HD / 8; ++n) {
+    const int c = n * 8 + 2 * tq;
+    red[(warp * 16 + gr) * C::RED_STRIDE + c] = o[n][0] * f0;
+    red[(warp * 16 + gr) * C::RED_STRIDE + c + 1] = o[n][1] * f0;
+    red[(warp * 16 + gr + 8) * C::RED_STRIDE + c] = o[n][2] * f1;
+    red[(warp * 16 + gr + 8) * C::RED_STRIDE + c + 1] = o[n][3] * f1;
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  const int tid = threadIdx.x;
+  for (int e = tid; e < 16 * HD; e += 128) {
+    const int r = e / HD, c = e % HD;
+    if (r >= rows) continue;
+    const float v = red[(0 * 16 + r) * C::RED_STRIDE + c] + red[(1 * 16 + r) * C::RED_STRIDE + c] +
+                    red[(2 * 16 + r) * C::RED_STRIDE + c] + red[(3 * 16 + r) * C::RED_STRIDE + c];
+    float* row = p.ws + (((size_t)b * p.nh + h0 + r) * p.n_split + split) * (HD + kWsPad);
+    row[c] = v;
+    if (c == 0) {
+      float M = -INFINITY, L = 0.f;
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, bars->ml[w][r][0]);
+      for (int w = 0; w < 4; ++w) {
+        const float mw = bars->ml[w][r][0];
+        if (mw != -INFINITY) L += bars->ml[w][r][1] * tc::ex2(mw - M);
+      }
+      row[HD] = M;
+      row[HD + 1] = L;
+    }
+  }
+}
+
+template <int HD>
+cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
+  using C = DCfg<HD>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tk, tv;
+  const uint64_t rows = (uint64_t)p.B * p.nkv * p.cap;
+  if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
+  const int g = p.nh / p.nkv;
+  const int n_hgrp = (g + 15) / 16;
+  dim3 grid((unsigned)(p.n_split * n_hgrp), p.nkv, p.B);
+  decode_mma_kernel<HD><<<grid, THREADS, C::SMEM, st>>>(tk, tv, p, n_hgrp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
+  switch (p.hd) {
+    case 64: return launch_hd<64>(p, st);
+    case 128: return launch_hd<128>(p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st) {
+  cudaError_t e = (bf16 && (p.hd == 64 || p.hd == 128)) ? launch_decode_mma(p, st) : launch_decode_simt(p, bf16, st);
+  if (e == cudaSuccess) e = launch_decode_combine(p, bf16, st);
+  return e;
+}
+
+}  // namespace gqa

@@ -94,8 +94,7 @@ int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
                       split, (cache_cap + split - 1) / split, static_cast<float*>(ws), out, err};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = dtype == GQA_BF16;
-  cudaError_t e = gqa::launch_decode_simt(p, bf16, s);
-  if (e == cudaSuccess) e = gqa::launch_decode_combine(p, bf16, s);
+  const cudaError_t e = gqa::launch_decode(p, bf16, s);
   gqa::count_launches(2);
   if (e != cudaSuccess) {
     cudaGetLastError();

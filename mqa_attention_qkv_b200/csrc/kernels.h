@@ -54,6 +54,12 @@ cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t
 // Tensor-core (tcgen05 + TMA) kernels, bf16 only.
 cudaError_t launch_qkv_tc(const QkvParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t st);  // head_dim 64 or 128
+cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
+cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128
+
+// Decode partials (tensor-core kernel for bf16 head_dim 64/128, else SIMT)
+// followed by the log-sum-exp combine; partial m is in log2 units.
+cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st);
 
 // 2-D bf16 TMA descriptor with 128-byte swizzle; `map` points at a CUtensorMap.
 // Zero fill outside [0, inner) x [0, outer).  False if encoding fails.

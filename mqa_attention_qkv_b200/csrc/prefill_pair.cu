@@ -1,0 +1,358 @@
+// Prefill attention for head_dim 64, two CTAs per SM (step a4, bf16).
+//
+// Same algorithm as prefill_tc.cu (exact tiled online softmax, FlashAttention-3
+// summary, recap section; GQA head map h -> h / g), laid out so that two CTAs
+// share each SM: at head_dim 64 a KV tile costs the tensor cores half of what
+// its 16K exponentials cost the MUFU unit, so the softmax of one CTA has to
+// run while the other CTA's MMAs do.  Per CTA:
+//   * TMEM: 256 columns = S (128 fp32 columns) + O (64).  P is written back
+//     over the first 64 columns of S as packed bf16 pairs and fed to the
+//     P.V MMA straight from TMEM (A operand in tensor memory), so P needs no
+//     shared memory.
+//   * shared memory: Q 16 KB + 3 K stages + 2 V stages = 96 KB.
+//   * warp 0 TMA, warp 1 MMA issuer, warps 2-5 softmax (thread = query row).
+// Softmax uses packed f32x2 FMA/ADD (two scores per instruction), 3-input
+// max and independent accumulators so the per-row chains stay short.  O is
+// rescaled in TMEM only when a row max grows by more than 2^8.
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace gqa {
+namespace {
+
+constexpr int HD = 64, BQ = 128, BKV = 128, THREADS = 192;
+constexpr int KS = 3, VS = 2;
+constexpr int TILE = 128 * HD * 2;             // 16 KB
+constexpr int Q_OFF = 0, K_OFF = TILE, V_OFF = K_OFF + KS * TILE, BAR_OFF = V_OFF + VS * TILE;
+constexpr int SMEM = BAR_OFF + 1024 + 1024;
+constexpr uint32_t kTmemCols = 256, kOCol = 128;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false, false);
+constexpr uint32_t IDESC_O = tc::idesc_bf16(128, HD, false, true);
+
+struct Bars {
+  uint64_t q_full, v_clean, drain, s_full, p_full, o_done;
+  uint64_t k_full[KS], k_empty[KS], v_full[VS], v_empty[VS];
+  uint32_t tmem_base;
+  int lim_max;
+};
+
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (a0, a1) * s + (c, c) on the packed f32x2 pipe
+__device__ __forceinline__ void fma2(float& a0, float& a1, float s, float c) {
+  uint64_t x, y, z;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(y) : "f"(s));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(z) : "f"(c));
+  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(x) : "l"(y), "l"(z));
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(x));
+}
+
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  uint64_t x, y;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1,%2};" : "=l"(y) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(x) : "l"(y));
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(x));
+}
+
+__global__ void __launch_bounds__(THREADS, 2)
+prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                    const __grid_constant__ CUtensorMap tmv, PrefillParams p, int n_qt) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + BAR_OFF);
+  int* err = p.err;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  const int bh_count = p.B * p.nh;
+  const int u = blockIdx.x;
+  const int qt = n_qt - 1 - u / bh_count;
+  const int b = (u % bh_count) / p.nh;
+  const int h = u % p.nh;
+  const int j = h / (p.nh / p.nkv);
+  const int s0 = qt * BQ;
+
+  int kv_len = p.kv_lens[b];
+  if (kv_len > p.cap || kv_len < 0) {
+    if (threadIdx.x == 0) raise_error(err, GQA_DEVERR_KVLEN_RANGE);
+    kv_len = kv_len > p.cap ? p.cap : 0;
+  }
+
+  const int row = (warp & 3) * 32 + lane;
+  int my_lim = 0;
+  bool my_valid = false;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->v_clean, 1);
+    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->o_done, 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(&bars->k_full[i], 1);
+      mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(&bars->v_full[i], 1);
+      mbar_init(&bars->v_empty[i], 1);
+    }
+    bars->lim_max = -1;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tc::prefetch_tmap(&tmq);
+    tc::prefetch_tmap(&tmk);
+    tc::prefetch_tmap(&tmv);
+  }
+  if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
+  __syncthreads();
+  if (warp >= 2) {
+    const int s = s0 + row;
+    my_valid = s < p.S;
+    if (my_valid) {
+      const int pos = p.q_pos ? p.q_pos[(size_t)b * p.S + s] : kv_len - p.S + s;
+      my_lim = p.causal ? max(0, min(kv_len, pos + 1)) : kv_len;
+      atomicMax(&bars->lim_max, my_lim);
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+  const int kv_hi = bars->lim_max < 0 ? 0 : bars->lim_max;
+  const int n_kv = (kv_hi + BKV - 1) / BKV;
+  const bool sanitize = n_kv > 0 && kv_len < n_kv * BKV;
+  const int kv_row0 = (b * p.nkv + j) * p.cap;
+  uint8_t* sQ = smem + Q_OFF;
+  uint8_t* sK = smem + K_OFF;
+  uint8_t* sV = smem + V_OFF;
+
+  if (warp == 0) {
+    // ================================================================ TMA
+    bool ok = true;
+    if (lane == 0 && n_kv > 0) {
+      mbar_arrive_expect_tx(&bars->q_full, TILE);
+      tc::tma_load_2d(sQ, &tmq, 0, (b * p.nh + h) * p.S + s0, &bars->q_full);
+      auto load_k = [&](int t) {
+        const int st = t % KS;
+        if (!mbar_wait(&bars->k_empty[st], ((t / KS) & 1) ^ 1, err)) return false;
+        mbar_arrive_expect_tx(&bars->k_full[st], TILE);
+        tc::tma_load_2d(sK + st * TILE, &tmk, 0, kv_row0 + t * BKV, &bars->k_full[st]);
+        return true;
+      };
+      auto load_v = [&](int t) {
+        const int st = t % VS;
+        if (!mbar_wait(&bars->v_empty[st], ((t / VS) & 1) ^ 1, err)) return false;
+        mbar_arrive_expect_tx(&bars->v_full[st], TILE);
+        tc::tma_load_2d(sV + st * TILE, &tmv, 0, kv_row0 + t * BKV, &bars->v_full[st]);
+        return true;
+      };
+      ok = load_k(0);
+      if (ok && n_kv > 1) ok = load_k(1);
+      for (int t = 0; ok && t < n_kv; ++t) {
+        if (t + 2 < n_kv) ok = load_k(t + 2);
+        if (ok) ok = load_v(t);
+      }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok && sanitize) {
+      const int t = n_kv - 1, st = t % VS;
+      const bool landed = mbar_wait(&bars->v_full[st], (t / VS) & 1, err);
+      if (__all_sync(0xffffffffu, landed)) {
+        const int r0 = max(0, kv_len - t * BKV);
+        uint8_t* vt = sV + st * TILE;
+        for (int r = r0 + lane / 8; r < BKV; r += 4)
+          *reinterpret_cast<uint4*>(vt + r * 128 + (lane % 8) * 16) = make_uint4(0, 0, 0, 0);
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->v_clean);
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA
+    if (lane == 0 && n_kv > 0) {
+      bool ok = mbar_wait(&bars->q_full, 0, err);
+      const uint32_t q_addr = smem_u32(sQ);
+      for (int t = 0; ok && t < n_kv; ++t) {
+        const int ks = t % KS, vs = t % VS;
+        if (!mbar_wait(&bars->k_full[ks], (t / KS) & 1, err)) { ok = false; break; }
+        // S/P columns are free once PV_{t-1} has read P_{t-1}
+        if (t > 0 && !mbar_wait(&bars->o_done, (t - 1) & 1, err)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t k_addr = smem_u32(sK + ks * TILE);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k)
+          tc::mma_bf16_ss(tmem, tc::sdesc_sw128(q_addr + k * 32, 16, 1024), tc::sdesc_sw128(k_addr + k * 32, 16, 1024),
+                          IDESC_S, k != 0);
+        tc::mma_commit(&bars->k_empty[ks]);
+        tc::mma_commit(&bars->s_full);
+        if (!mbar_wait(&bars->p_full, t & 1, err)) { ok = false; break; }
+        if (!mbar_wait(&bars->v_full[vs], (t / VS) & 1, err)) { ok = false; break; }
+        if (sanitize && t == n_kv - 1 && !mbar_wait(&bars->v_clean, 0, err)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t v_addr = smem_u32(sV + vs * TILE);
+#pragma unroll
+        for (int k = 0; k < BKV / 16; ++k)
+          mma_bf16_ts(tmem + kOCol, tmem + k * 8, tc::sdesc_sw128(v_addr + k * 2048, 16384, 1024), IDESC_O,
+                      (t | k) != 0);
+        tc::mma_commit(&bars->v_empty[vs]);
+        tc::mma_commit(&bars->o_done);
+      }
+      tc::mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, err);
+    }
+  } else {
+    // ================================================================ softmax
+    const float scale_log2 = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < n_kv; ++t) {
+      const int k0 = t * BKV;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full, t & 1, err));
+      if (!ok) break;
+      tc::fence_after_sync();
+      float s[BKV];
+#pragma unroll
+      for (int c = 0; c < BKV / 16; ++c) {
+        uint32_t r[16];
+        tc::tmem_ld16(tmem + lane_base + c * 16, r);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s[c * 16 + i] = __uint_as_float(r[i]);
+      }
+      tc::tmem_ld_wait();
+      if (k0 + BKV > my_lim) {
+#pragma unroll
+        for (int i = 0; i < BKV; ++i)
+          if (k0 + i >= my_lim) s[i] = -INFINITY;
+      }
+      // row max of the raw scores (scale > 0 commutes with max)
+      float ma = -INFINITY, mb = -INFINITY, mc = -INFINITY, md = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < BKV; i += 8) {
+        ma = max3(ma, s[i], s[i + 1]);
+        mb = max3(mb, s[i + 2], s[i + 3]);
+        mc = max3(mc, s[i + 4], s[i + 5]);
+        md = max3(md, s[i + 6], s[i + 7]);
+      }
+      const float mx = fmaxf(fmaxf(ma, mb), fmaxf(mc, md)) * scale_log2;
+      float alpha = 1.f;
+      if (m_used == -INFINITY) {
+        m_used = mx;
+      } else if (mx > m_used + kRescaleThreshold) {
+        alpha = tc::ex2(m_used - mx);
+        l *= alpha;
+        m_used = mx;
+      }
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (t - 1) & 1, err));
+        if (!ok) break;
+        tc::fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < HD / 16; ++c) {
+          uint32_t r[16];
+          tc::tmem_ld16(tmem + lane_base + kOCol + c * 16, r);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tc::tmem_st16(tmem + lane_base + kOCol + c * 16, r);
+        }
+      }
+      // P = 2^(s * scale - m) -> bf16 pairs over the first 64 columns of S
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+      float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < BKV / 32; ++c) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float p0 = s[c * 32 + 2 * i], p1 = s[c * 32 + 2 * i + 1];
+          fma2(p0, p1, scale_log2, neg_m);
+          p0 = tc::ex2(p0);
+          p1 = tc::ex2(p1);
+          if (i & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
+          w[i] = pack_bf16x2(p0, p1);
+        }
+        tc::tmem_st16(tmem + lane_base + c * 16, w);
+      }
+      l += (sa0 + sa1) + (sb0 + sb1);
+      tc::tmem_st_wait();
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full);
+    }
+
+    if (ok && n_kv > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (n_kv - 1) & 1, err));
+    tc::fence_after_sync();
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + (((size_t)b * p.S + (s0 + row)) * p.nh + h) * HD;
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+    for (int c = 0; c < HD / 16; ++c) {
+      uint32_t r[16];
+      if (ok && n_kv > 0) {
+        __syncwarp();
+        tc::tmem_ld16(tmem + lane_base + kOCol + c * 16, r);
+        tc::tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = 0u;
+      }
+      if (my_valid) {
+        uint32_t o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          o[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+        tc::st_global_v4(dst + c * 16, o[0], o[1], o[2], o[3]);
+        tc::st_global_v4(dst + c * 16 + 8, o[4], o[5], o[6], o[7]);
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st) {
+  if (p.hd != HD) return cudaErrorInvalidValue;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tq, tk, tv;
+  const uint64_t q_rows = (uint64_t)p.B * p.nh * p.S, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
+  if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+  const int n_qt = (p.S + BQ - 1) / BQ;
+  const long long grid = (long long)n_qt * p.B * p.nh;
+  prefill_pair_kernel<<<(unsigned)grid, THREADS, SMEM, st>>>(tq, tk, tv, p, n_qt);
+  return cudaGetLastError();
+}
+
+}  // namespace gqa

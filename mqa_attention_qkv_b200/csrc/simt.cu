@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(PrefillParams pp, Decode
 #pragma unroll
       for (int d = 0; d < PER; ++d) row[lane + 32 * d] = acc[rr][d];
       if (lane == 0) {
-        row[HD] = m_r[rr];
+        row[HD] = m_r[rr] * 1.4426950408889634f;  // partial max in log2 units
         row[HD + 1] = l_r[rr];
       }
     } else {
@@ -274,8 +274,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(PrefillParams pp, Decode
 
 // ---------------------------------------------------------------------------
 // decode_combine: one warp per (b, h).  Partials c = 0..n-1 with n =
-// ceil(kv_len / split); M = max m_c, L = sum l_c e^(m_c - M),
-// O = sum o_c e^(m_c - M) / L.
+// ceil(kv_len / split), their maxima m_c in log2 units of the scaled score;
+// M = max m_c, L = sum l_c 2^(m_c - M), O = sum o_c 2^(m_c - M) / L.
 // ---------------------------------------------------------------------------
 template <typename T, int HD>
 __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p) {
@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p) {
   if (M != -INFINITY) {
     for (int c = 0; c < n; ++c) {
       const float* part = ws + (size_t)c * (HD + kWsPad);
-      const float e = expf(part[HD] - M);
+      const float e = exp2f(part[HD] - M);
       L += part[HD + 1] * e;
 #pragma unroll
       for (int d = 0; d < PER; ++d) o[d] = fmaf(part[lane + 32 * d], e, o[d]);
