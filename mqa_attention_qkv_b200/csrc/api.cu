@@ -158,7 +158,11 @@ int qkv_rope_project(const void* x, const void* w_qkv, const int32_t* positions,
                    (double)rope_theta, q_out, k_cache, v_cache, d->err};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Tensor-core path: bf16 with 16-byte-aligned rows (TMA row stride).
-  if (dtype == GQA_BF16 && hidden % 8 == 0) return launch_status(gqa::launch_qkv_tc(p, d->num_sms, s));
+  if (dtype == GQA_BF16 && hidden % 8 == 0) {
+    // a few tokens: W-streaming kernel spread over every SM; else 128-token tiles
+    if ((long long)B * S <= 64) return launch_status(gqa::launch_qkv_smallm(p, s));
+    return launch_status(gqa::launch_qkv_tc(p, d->num_sms, s));
+  }
   return launch_status(gqa::launch_qkv_simt(p, dtype == GQA_BF16, s));
 }
 

@@ -53,6 +53,7 @@ cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t
 
 // Tensor-core (tcgen05 + TMA) kernels, bf16 only.
 cudaError_t launch_qkv_tc(const QkvParams& p, int num_sms, cudaStream_t st);
+cudaError_t launch_qkv_smallm(const QkvParams& p, cudaStream_t st);  // B*S <= 64
 cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t st);  // head_dim 64 or 128
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128

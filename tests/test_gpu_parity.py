@@ -52,6 +52,12 @@ QKV_CASES = [
     ("bf16", 3, 150, 136, 3, 1, 64, 160, True),     # N = 320 (partial 256-tile), K tail, T = 450
     ("bf16", 2, 300, 256, 12, 2, 32, 320, False),   # hd 32: 8 heads per tile
     ("bf16", 2, 70, 100, 4, 2, 64, 80, True),       # hidden % 8 != 0: the SIMT path
+    # few tokens (the W-streaming kernel), every token-count variant
+    ("bf16", 3, 1, 2048, 32, 4, 64, 16, True),
+    ("bf16", 4, 3, 520, 8, 2, 128, 8, True),
+    ("bf16", 2, 10, 1000, 6, 1, 128, 16, True),
+    ("bf16", 8, 5, 256, 12, 2, 32, 9, True),
+    ("bf16", 1, 64, 136, 4, 4, 64, 64, False),
 ]
 
 
