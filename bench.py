@@ -170,7 +170,7 @@ def run_ours(args):
     pos_dec = torch.full((B, 1), S, dtype=torch.int32, device=dev)
     lens = torch.full((B,), S, dtype=torch.int32, device=dev)
     lens_dec = torch.full((B,), S + 1, dtype=torch.int32, device=dev)
-    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     names = ("qkv_prefill", "attn_prefill", "qkv_decode", "attn_decode")
@@ -379,7 +379,7 @@ def measure_workloads(dev, peaks, iters=10):
         kc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
         vc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
         o = torch.empty(B, nh, hd, dtype=bf, device=dev)
-        ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
         ms = timed(lambda: gqa.gqa_attn_decode(q, kc, vc, lens, o, ws, stream=stream))
         nbytes = 2.0 * (2 * nkv * hd * float(lens_np.sum()) + 2 * B * nh * hd)
         gbs = nbytes / (ms / 1e3) / 1e9
@@ -425,7 +425,7 @@ def measure_workloads(dev, peaks, iters=10):
     pos_steps = (P + torch.arange(T, dtype=torch.int32, device=dev)).view(T, 1, 1).expand(T, B, 1).contiguous()
     len_steps = (P + 1 + torch.arange(T, dtype=torch.int32, device=dev)).view(T, 1).expand(T, B).contiguous()
     lp_ = torch.full((B,), P, dtype=torch.int32, device=dev)
-    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
 
     def gen_loop():
         st = torch.cuda.current_stream(dev)   # the capture stream while a graph is being recorded

@@ -130,8 +130,10 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
 
 /*
  * gqa_attn_decode_workspace_size - bytes of device workspace gqa_attn_decode
- * needs for these sizes (float32 partial results: a running max, a sum and
- * an unnormalised output row per sequence, query head and key split).
+ * needs for these sizes: a block of split counters (one 32-bit word per
+ * sequence, KV head and group of up to 16 query heads, rounded up to 256
+ * bytes) followed by float32 partial results (a running max, a sum and an
+ * unnormalised output row per sequence, query head and key split).
  * kv_split: keys per split, 0 = the library's choice, else a multiple of 64.
  * Returns 0 for invalid arguments.
  */
@@ -147,7 +149,10 @@ size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int he
  * K/V byte read serves g heads (arithmetic intensity ~g).  The keys of a
  * sequence are split into chunks of kv_split; each chunk produces a partial
  * (max m, sum l, unnormalised o) per head and the partials are merged with a
- * log-sum-exp combine, which is exact.
+ * log-sum-exp combine, which is exact.  On the tensor-core path (bf16,
+ * head_dim 64/128) the last chunk of a (sequence, KV head) to finish does the
+ * merge, found through a counter in the workspace; a sequence with a single
+ * chunk is written directly.
  *
  *   q          [B, n_heads, head_dim] dtype (the new token, already rotated)
  *   k_cache,
@@ -155,9 +160,14 @@ size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int he
  *   kv_lens    [B] int32: valid keys including the new token; clamped to
  *              [0, cache_cap] (GQA_DEVERR_KVLEN_RANGE); 0 gives a zero row
  *   kv_split   keys per split: 0 = automatic, else a positive multiple of 64
+ *              giving at most 1024 splits of cache_cap
  *   out        [B, n_heads, head_dim] dtype
  *   workspace  device scratch of at least gqa_attn_decode_workspace_size()
- *              bytes, 16-byte aligned; its contents on entry do not matter.
+ *              bytes, 16-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE
+ *              (e.g. cudaMemset once after allocating it).  Every call leaves
+ *              the counter block at zero again, so a workspace can be reused
+ *              by any later call; calls that may run at the same time on the
+ *              GPU need workspaces of their own.
  */
 int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,
@@ -180,10 +190,12 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
  * process exits.  A problem whose partials (gqa_attn_decode_workspace_size)
  * exceed 64 MiB is rejected with GQA_ERR_WORKSPACE_TOO_SMALL; a larger
  * kv_split needs fewer partials.  The first call on each device looks up the
- * array's device address (with that device current), so make that first call
- * before any stream capture.  All calls share the array and nothing in it has
- * to start at zero; calls that overlap on the GPU (e.g. on two streams) race,
- * so order them on one stream or with events.  It allocates nothing.
+ * array's device address (with that device current) and zeroes the array
+ * once (a synchronous cudaMemset), so make that first call before any stream
+ * capture.  All calls share the array; each leaves its counter block at zero,
+ * as the next call needs it.  Calls that overlap on the GPU (e.g. on two
+ * streams) race, so order them on one stream or with events.  It allocates
+ * nothing.
  */
 int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,

@@ -65,15 +65,20 @@ int launch_status(cudaError_t e, int n_launched = 1) {
   return GQA_ERR_LAUNCH_FAILED;
 }
 
-// Keys per decode split when the caller leaves it to the library: enough
-// (sequence, KV head, split) work units to fill the GPU several times over
-// for a half-full cache, between 64 and 2048 keys, a multiple of 64.
-int auto_split(int B, int nkv, int cap) {
-  const long long units_wanted = 1024;
-  long long s = ((long long)B * nkv * ((cap + 1) / 2) + units_wanted - 1) / units_wanted;
+// Keys per decode split when the caller leaves it to the library: about two
+// work units (sequence x KV head x group of 16 query heads x split) per SM of
+// a B200 (148 SMs) for a full cache, at least 128 keys (2 tiles) and at most
+// 2048, a multiple of 64, and never more than kMaxSplits splits.
+constexpr long long kUnitsWanted = 2 * 148;
+constexpr int kMaxSplits = 1024;
+int auto_split(int B, int nkv, int n_hgrp, int cap) {
+  const long long groups = (long long)B * nkv * n_hgrp;
+  long long s = (groups * cap + kUnitsWanted - 1) / kUnitsWanted;
   s = (s + 63) / 64 * 64;
-  if (s < 64) s = 64;
+  if (s < 128) s = 128;
   if (s > 2048) s = 2048;
+  const long long min_s = ((cap + kMaxSplits - 1) / kMaxSplits + 63) / 64 * 64;
+  if (s < min_s) s = min_s;
   return (int)s;
 }
 
@@ -92,8 +97,19 @@ int device_check(int** err) {
 
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
-int decode_split_len(int B, int n_kv_heads, int cache_cap, int kv_split) {
-  return kv_split ? kv_split : auto_split(B, n_kv_heads, cache_cap);
+int decode_split_len(int B, int nh, int nkv, int cache_cap, int kv_split) {
+  return kv_split ? kv_split : auto_split(B, nkv, decode_n_hgrp(nh, nkv), cache_cap);
+}
+
+DecodeParams decode_params(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens,
+                           int B, int nh, int nkv, int hd, int cap, int kv_split, void* out, void* workspace,
+                           int* err) {
+  const int split = decode_split_len(B, nh, nkv, cap, kv_split);
+  const int n_hgrp = decode_n_hgrp(nh, nkv);
+  unsigned* counters = static_cast<unsigned*>(workspace);
+  float* partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_counter_bytes(B, nkv, n_hgrp));
+  return DecodeParams{q, k_cache, v_cache, kv_lens, B, nh, nkv, hd, cap, split, (cap + split - 1) / split,
+                      partials, out, err, counters, n_hgrp};
 }
 
 }  // namespace gqa
@@ -199,9 +215,11 @@ size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int he
   if (B < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0 || n_heads % n_kv_heads) return 0;
   if (!hd_ok(head_dim)) return 0;
   if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return 0;
-  const int split = kv_split ? kv_split : auto_split(B, n_kv_heads, cache_cap);
+  const int split = gqa::decode_split_len(B, n_heads, n_kv_heads, cache_cap, kv_split);
   const size_t n_split = (size_t)(cache_cap + split - 1) / split;
-  return (size_t)B * n_heads * n_split * (head_dim + gqa::kWsPad) * sizeof(float);
+  if (n_split > (size_t)kMaxSplits) return 0;
+  return gqa::decode_counter_bytes(B, n_kv_heads, gqa::decode_n_hgrp(n_heads, n_kv_heads)) +
+         (size_t)B * n_heads * n_split * (head_dim + gqa::kWsPad) * sizeof(float);
 }
 
 int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -212,6 +230,7 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
   if (B < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0) return GQA_ERR_INVALID_ARG;
   if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
   if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;
+  if (kv_split > 0 && (cache_cap + kv_split - 1) / kv_split > kMaxSplits) return GQA_ERR_INVALID_ARG;
   if (!hd_ok(head_dim)) return GQA_ERR_UNSUPPORTED_SHAPE;
   if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems || B > 65535 || n_kv_heads > 65535)
     return GQA_ERR_UNSUPPORTED_SHAPE;
@@ -226,13 +245,12 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
   const DeviceInfo* d = device_info(&st);
   if (!d) return st;
 
-  const int split = kv_split ? kv_split : auto_split(B, n_kv_heads, cache_cap);
-  gqa::DecodeParams p{q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim, cache_cap,
-                      split, (cache_cap + split - 1) / split, static_cast<float*>(workspace), out,
-                      d->err};
+  const gqa::DecodeParams p = gqa::decode_params(q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim,
+                                                 cache_cap, kv_split, out, workspace, d->err);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool bf16 = dtype == GQA_BF16;
-  return launch_status(gqa::launch_decode(p, bf16, s), 2);
+  cudaError_t e;
+  const int n = gqa::launch_decode(p, dtype == GQA_BF16, s, &e);
+  return launch_status(e, n);
 }
 
 uint64_t gqa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -65,7 +65,9 @@ __device__ __forceinline__ uint32_t swz(int row, int col) {
 
 struct Bars {
   uint64_t full[4], empty[4];
-  float ml[4][16][2];
+  float ml[4][16][2];   // per warp, per head row: max, sum
+  float cm[16][2];      // per head row: merged max, sum (or 1/sum)
+  int last;
 };
 
 template <int HD>
@@ -88,11 +90,17 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     kv_len = kv_len > p.cap ? p.cap : 0;
   }
   const int k_lo = split * p.split;
-  if (k_lo >= kv_len) return;  // no key of this sequence in this split (whole block)
-  const int k_hi = min(kv_len, k_lo + p.split);
-  const int n_t = (k_hi - k_lo + KT - 1) / KT;
   const int h0 = j * g + hg * 16;
   const int rows = min(16, g - hg * 16);
+  if (k_lo >= kv_len) {  // no key of this sequence in this split (whole block)
+    if (split == 0) {    // no key at all: the output rows are zero
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * p.nh + h0) * HD;
+      for (int e = threadIdx.x; e < rows * HD; e += blockDim.x) out[e] = __float2bfloat16_rn(0.f);
+    }
+    return;
+  }
+  const int k_hi = min(kv_len, k_lo + p.split);
+  const int n_t = (k_hi - k_lo + KT - 1) / KT;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -259,26 +267,95 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     red[(warp * 16 + gr + 8) * C::RED_STRIDE + c] = o[n][2] * f1;
     red[(warp * 16 + gr + 8) * C::RED_STRIDE + c + 1] = o[n][3] * f1;
   }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
   const int tid = threadIdx.x;
-  for (int e = tid; e < 16 * HD; e += 128) {
+  if (tid < 16) {  // this CTA's max and sum per head row, over its 4 warps
+    float M = -INFINITY, L = 0.f;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, bars->ml[w][tid][0]);
+    for (int w = 0; w < 4; ++w) {
+      const float mw = bars->ml[w][tid][0];
+      if (mw != -INFINITY) L += bars->ml[w][tid][1] * tc::ex2(mw - M);
+    }
+    bars->cm[tid][0] = M;
+    bars->cm[tid][1] = L;
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  auto red_sum = [&](int r, int c) {
+    return red[(0 * 16 + r) * C::RED_STRIDE + c] + red[(1 * 16 + r) * C::RED_STRIDE + c] +
+           red[(2 * 16 + r) * C::RED_STRIDE + c] + red[(3 * 16 + r) * C::RED_STRIDE + c];
+  };
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+  const int n_active = (kv_len + p.split - 1) / p.split;   // splits that hold keys of this sequence
+  if (n_active == 1) {
+    // the only split: normalise and write the output directly
+    for (int e = tid; e < rows * HD; e += 128) {
+      const int r = e / HD, c = e % HD;
+      const float L = bars->cm[r][1];
+      out[((size_t)b * p.nh + h0 + r) * HD + c] = __float2bfloat16_rn(L > 0.f ? red_sum(r, c) / L : 0.f);
+    }
+    return;
+  }
+  // write this split's partial (o unnormalised, m in log2 units, l)
+  for (int e = tid; e < rows * HD; e += 128) {
     const int r = e / HD, c = e % HD;
-    if (r >= rows) continue;
-    const float v = red[(0 * 16 + r) * C::RED_STRIDE + c] + red[(1 * 16 + r) * C::RED_STRIDE + c] +
-                    red[(2 * 16 + r) * C::RED_STRIDE + c] + red[(3 * 16 + r) * C::RED_STRIDE + c];
     float* row = p.ws + (((size_t)b * p.nh + h0 + r) * p.n_split + split) * (HD + kWsPad);
-    row[c] = v;
+    row[c] = red_sum(r, c);
     if (c == 0) {
-      float M = -INFINITY, L = 0.f;
-      for (int w = 0; w < 4; ++w) M = fmaxf(M, bars->ml[w][r][0]);
-      for (int w = 0; w < 4; ++w) {
-        const float mw = bars->ml[w][r][0];
-        if (mw != -INFINITY) L += bars->ml[w][r][1] * tc::ex2(mw - M);
-      }
-      row[HD] = M;
-      row[HD + 1] = L;
+      row[HD] = bars->cm[r][0];
+      row[HD + 1] = bars->cm[r][1];
     }
   }
+  // the last split of this (sequence, KV head, head group) to finish merges them all
+  __threadfence();
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  unsigned* counter = p.counters + ((size_t)b * p.nkv + j) * n_hgrp + hg;
+  if (tid == 0) bars->last = atomicAdd(counter, 1u) == (unsigned)(n_active - 1);
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (!bars->last) return;
+  __threadfence();
+  // merge: per head row, lanes take the splits -> max, sum and one weight
+  // 2^(m_s - M) / L per split (kept in shared memory); then every thread
+  // takes float4 output columns and sums the splits with independent loads.
+  const size_t stride = HD + kWsPad;
+  float* wgt = red;  // [16][n_active]
+  for (int r = warp; r < rows; r += 4) {
+    const float* part = p.ws + ((size_t)b * p.nh + h0 + r) * p.n_split * stride;
+    float M = -INFINITY;
+    for (int s = lane; s < n_active; s += 32) M = fmaxf(M, __ldcg(part + s * stride + HD));
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+    float L = 0.f;
+    for (int s = lane; s < n_active; s += 32) {
+      const float ms = __ldcg(part + s * stride + HD);
+      const float e = ms == -INFINITY ? 0.f : tc::ex2(ms - M);
+      wgt[r * n_active + s] = e;
+      L += __ldcg(part + s * stride + HD + 1) * e;
+    }
+#pragma unroll
+    for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o2);
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __syncwarp();
+    for (int s = lane; s < n_active; s += 32) wgt[r * n_active + s] *= inv;
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  for (int e = tid; e < rows * (HD / 4); e += 128) {
+    const int r = e / (HD / 4), c = (e % (HD / 4)) * 4;
+    const float* part = p.ws + ((size_t)b * p.nh + h0 + r) * p.n_split * stride + c;
+    const float* w = wgt + r * n_active;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = 0; s < n_active; ++s) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(part + s * stride));
+      const float ws_ = w[s];
+      acc.x = fmaf(v.x, ws_, acc.x);
+      acc.y = fmaf(v.y, ws_, acc.y);
+      acc.z = fmaf(v.z, ws_, acc.z);
+      acc.w = fmaf(v.w, ws_, acc.w);
+    }
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * p.nh + h0 + r) * HD + c);
+    dst[0] = __floats2bfloat162_rn(acc.x, acc.y);
+    dst[1] = __floats2bfloat162_rn(acc.z, acc.w);
+  }
+  if (tid == 0) atomicExch(counter, 0u);  // leave the counter at zero for the next call
 }
 
 template <int HD>
@@ -313,10 +390,15 @@ cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
   }
 }
 
-cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st) {
-  cudaError_t e = (bf16 && (p.hd == 64 || p.hd == 128)) ? launch_decode_mma(p, st) : launch_decode_simt(p, bf16, st);
+int launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st, cudaError_t* err) {
+  if (bf16 && (p.hd == 64 || p.hd == 128)) {  // merges its splits itself
+    *err = launch_decode_mma(p, st);
+    return 1;
+  }
+  cudaError_t e = launch_decode_simt(p, bf16, st);
   if (e == cudaSuccess) e = launch_decode_combine(p, bf16, st);
-  return e;
+  *err = e;
+  return 2;
 }
 
 }  // namespace gqa

@@ -48,6 +48,8 @@ void* scratch_ptr() {
   ScratchSlot& s = g_slot[dev];
   std::call_once(s.once, [&] {
     s.status = cudaGetSymbolAddress(&s.ptr, g_decode_scratch);
+    // the split counters at the front must start at zero; every call leaves them so
+    if (s.status == cudaSuccess) s.status = cudaMemset(s.ptr, 0, kNoAllocScratchBytes);
     if (s.status != cudaSuccess) {
       s.ptr = nullptr;
       cudaGetLastError();
@@ -85,17 +87,17 @@ int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
   void* ws = scratch_ptr();
   if (!ws) return GQA_ERR_NO_DEVICE;
 
-  // Nothing in the scratch has to start at zero: the merge reads only the
-  // partials of splits that hold keys, and this call writes each of them
-  // first.  Calls that overlap on the GPU (other streams) share the array and
-  // race; order them on one stream or with events.
-  const int split = gqa::decode_split_len(B, n_kv_heads, cache_cap, kv_split);
-  gqa::DecodeParams p{q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim, cache_cap,
-                      split, (cache_cap + split - 1) / split, static_cast<float*>(ws), out, err};
+  // The scratch starts with the per-(sequence, KV head) split counters, which
+  // must be zero: the set-up above zeroes the array once and every call leaves
+  // the counters at zero again.  The partials need no clearing (each one the
+  // merge reads is written by the same call first).  Calls that overlap on the
+  // GPU (other streams) share the array and race; order them on one stream or
+  // with events.
+  const gqa::DecodeParams p = gqa::decode_params(q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim,
+                                                 cache_cap, kv_split, out, ws, err);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool bf16 = dtype == GQA_BF16;
-  const cudaError_t e = gqa::launch_decode(p, bf16, s);
-  gqa::count_launches(2);
+  cudaError_t e;
+  gqa::count_launches(gqa::launch_decode(p, dtype == GQA_BF16, s, &e));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GQA_ERR_LAUNCH_FAILED;

@@ -41,9 +41,17 @@ struct DecodeParams {
   float* ws;              // [B, nh, n_split, hd + 4]: o[hd], m, l, -, -
   void* out;              // [B, nh, hd]
   int* err;
+  unsigned* counters;     // [B, nkv, n_hgrp]: finished splits (zero between calls)
+  int n_hgrp;             // groups of <= 16 query heads per KV head
 };
 
 constexpr int kWsPad = 4;  // per-partial row: hd floats of o, then m, l and two pad words
+
+// Decode workspace: the counters (rounded up to 256 bytes), then the partials.
+inline size_t decode_counter_bytes(int B, int nkv, int n_hgrp) {
+  return ((size_t)B * nkv * n_hgrp * sizeof(unsigned) + 255) / 256 * 256;
+}
+inline int decode_n_hgrp(int nh, int nkv) { return (nh / nkv + 15) / 16; }
 
 // SIMT kernels (any dtype; the fp32 path and shapes the tensor-core kernels skip)
 cudaError_t launch_qkv_simt(const QkvParams& p, bool bf16, cudaStream_t st);
@@ -58,9 +66,11 @@ cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t st);  // head
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128
 
-// Decode partials (tensor-core kernel for bf16 head_dim 64/128, else SIMT)
-// followed by the log-sum-exp combine; partial m is in log2 units.
-cudaError_t launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st);
+// Decode: the tensor-core kernel for bf16 head_dim 64/128 (the last split of
+// each (sequence, KV head, head group) merges the partials itself, using the
+// counters), else SIMT partials + the log-sum-exp combine kernel.  Partial m
+// is in log2 units.  Returns the number of kernels launched; *err the status.
+int launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st, cudaError_t* err);
 
 // 2-D bf16 TMA descriptor with 128-byte swizzle; `map` points at a CUtensorMap.
 // Zero fill outside [0, inner) x [0, outer).  False if encoding fails.
@@ -70,6 +80,10 @@ bool make_tmap_bf16_2d(void* map, const void* base, uint64_t inner, uint64_t out
 // Shared by the C-ABI translation units (defined in api.cu).
 int device_check(int** err);  // GQA_OK, or the status for the current device
 void count_launches(int n);
-int decode_split_len(int B, int n_kv_heads, int cache_cap, int kv_split);
+int decode_split_len(int B, int nh, int nkv, int cache_cap, int kv_split);
+// Decode parameters over a workspace laid out as counters, then partials.
+DecodeParams decode_params(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens,
+                           int B, int nh, int nkv, int hd, int cap, int kv_split, void* out, void* workspace,
+                           int* err);
 
 }  // namespace gqa

@@ -110,9 +110,11 @@ def test_empty_inputs_are_noops():
 
 def test_workspace_size_query():
     f = gqa.gqa_attn_decode_workspace_size
-    # B * nh * ceil(cap / split) * (hd + 4) floats
-    assert f(2, 4, 2, 64, 1000, 64) == 2 * 4 * 16 * 68 * 4
-    assert f(64, 32, 8, 128, 8192, 512) == 64 * 32 * 16 * 132 * 4
+    # split counters (B * nkv * ceil(g / 16) words, rounded up to 256 bytes)
+    # then B * nh * ceil(cap / split) * (hd + 4) floats
+    assert f(2, 4, 2, 64, 1000, 64) == 256 + 2 * 4 * 16 * 68 * 4
+    assert f(64, 32, 8, 128, 8192, 512) == 2048 + 64 * 32 * 16 * 132 * 4
+    assert f(64, 32, 1, 128, 8192, 512) == 512 + 64 * 32 * 16 * 132 * 4   # g = 32: 2 head groups
     assert f(2, 4, 2, 64, 1000, 0) > 0
     assert f(2, 4, 2, 64, 1000, 100) == 0      # split not a multiple of 64
     assert f(2, 4, 3, 64, 1000, 64) == 0       # nh % nkv

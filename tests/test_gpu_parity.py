@@ -187,7 +187,7 @@ def test_prefill_explicit_positions_and_empty_rows():
 def run_decode(q, kc, vc, lens, nh, dtype, kv_split=0):
     B, _, hd = q.shape
     nkv, cap = kc.shape[1], kc.shape[2]
-    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap, kv_split) // 4 + 1,
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap, kv_split) // 4 + 1,
                      dtype=torch.float32, device="cuda")
     out = torch.empty((B, nh, hd), dtype=TORCH_DT[dtype], device="cuda")
     gqa.gqa_attn_decode(dev(q), dev(kc), dev(vc), dev_i32(lens), out, ws, kv_split=kv_split)
@@ -212,6 +212,26 @@ def test_decode_parity(case):
     for split in (0, 64, 192):
         out = run_decode(q, kc, vc, lens, nh, dtype, kv_split=split)
         gate(host(out), want, dtype, f"decode {case} split={split}")
+
+
+def test_decode_workspace_reuse_leaves_counters_zero():
+    """One zero-filled workspace serves calls of different shapes in a row; the
+    merge counters at its front are back at zero after each call."""
+    ws = torch.zeros(8 << 20, dtype=torch.uint8, device="cuda")
+    for seed, (B, nh, nkv, hd, cap, lens) in enumerate([
+            (3, 32, 4, 128, 900, [900, 70, 511]),
+            (5, 48, 1, 128, 700, [1, 700, 64, 65, 333]),
+            (2, 8, 8, 64, 300, [300, 129])]):
+        lens = np.array(lens, dtype=np.int32)
+        q = W.normal_tensor((B, nh, hd), 40 + seed, 0, "bf16")
+        kc = nan_padded(B, nkv, cap, hd, lens, 40 + seed, 1, "bf16")
+        vc = nan_padded(B, nkv, cap, hd, lens, 40 + seed, 2, "bf16")
+        out = torch.empty((B, nh, hd), dtype=torch.bfloat16, device="cuda")
+        gqa.gqa_attn_decode(dev(q), dev(kc), dev(vc), dev_i32(lens), out, ws, kv_split=64)
+        want = ref.decode_attention(q.f64, kc.f64, vc.f64, lens)
+        gate(host(out), want, "bf16", f"reused workspace, case {seed}")
+        n_counters = B * nkv * ((nh // nkv + 15) // 16)
+        assert int(ws[:4 * n_counters].view(torch.int32).abs().sum()) == 0
 
 
 def test_decode_split_count_invariance():

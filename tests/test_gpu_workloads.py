@@ -68,7 +68,7 @@ def test_tinyllama_prefill_and_decode_step(bs):
     posd = np.full((B, 1), S, dtype=np.int32)
     gqa.qkv_rope_project(dev(xd), wd, dev_i32(posd), nh, nkv, hd, sh.rope_theta, qd, kc, vc)
     od = torch.empty((B, nh, hd), dtype=BF, device="cuda")
-    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device="cuda")
     gqa.gqa_attn_decode(qd.view(B, nh, hd), kc, vc, dev_i32(np.full(B, S + 1)), od, ws)
     torch.cuda.synchronize()
 
@@ -106,7 +106,7 @@ def test_llama2_decode_full(nkv):
     vc = W.decode_cache(wl.seed, 2, B, nkv, cap, hd, lens)
     vd = dev(vc)
     del vc
-    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device="cuda")
     out = torch.empty((B, nh, hd), dtype=BF, device="cuda")
     gqa.gqa_attn_decode(dev(q), kd, vd, dev_i32(lens), out, ws)
     got = host(out)
@@ -143,7 +143,7 @@ def test_mqa_generation_loop_full():
     posp = np.broadcast_to(np.arange(P, dtype=np.int32), (B, P)).copy()
     gqa.qkv_rope_project(dev(xp), wd, dev_i32(posp), nh, nkv, hd, sh.rope_theta, q, kc, vc)
     gqa.gqa_attn_prefill(q, kc, vc, dev_i32(np.full(B, P)), True, o_p)
-    ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device="cuda")
     check = {0, 1, 2, 100, 511, 1022, 1023}
     outs = {}
     qt = torch.empty((B, nh, 1, hd), dtype=BF, device="cuda")

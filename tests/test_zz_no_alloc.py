@@ -38,7 +38,7 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls():
     ]
     for seed, B, nh, nkv, hd, cap, lens, split in cases:
         q, kc, vc, ln = _problem(seed, B, nh, nkv, hd, cap, lens)
-        ws = torch.empty(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap, split),
+        ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap, split),
                          dtype=torch.uint8, device="cuda")
         want = torch.empty((B, nh, hd), dtype=torch.bfloat16, device="cuda")
         got = torch.full((B, nh, hd), float("nan"), dtype=torch.bfloat16, device="cuda")
