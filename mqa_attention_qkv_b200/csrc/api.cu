@@ -68,7 +68,8 @@ int launch_status(cudaError_t e, int n_launched = 1) {
 // Keys per decode split when the caller leaves it to the library: about two
 // work units (sequence x KV head x group of 16 query heads x split) per SM of
 // a B200 (148 SMs) for a full cache, at least 128 keys (2 tiles) and at most
-// 2048, a multiple of 64, and never more than kMaxSplits splits.
+// 2048, a multiple of 64, and never more than kMaxSplits splits.  (Eight
+// units per SM, tried for ragged MQA batches, measured slower on B200.)
 constexpr long long kUnitsWanted = 2 * 148;
 constexpr int kMaxSplits = 1024;
 int auto_split(int B, int nkv, int n_hgrp, int cap) {
@@ -205,8 +206,9 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
   gqa::PrefillParams p{q, k_cache, v_cache, q_positions, kv_lens, B, S, n_heads, n_kv_heads,
                        head_dim, cache_cap, causal ? 1 : 0, out, d->err};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // head_dim 64: two CTAs per SM (measured fastest there); 128: two query tiles per CTA
   if (dtype == GQA_BF16 && head_dim == 64) return launch_status(gqa::launch_prefill_pair(p, s));
-  if (dtype == GQA_BF16 && head_dim == 128) return launch_status(gqa::launch_prefill_tc(p, s));
+  if (dtype == GQA_BF16 && head_dim == 128) return launch_status(gqa::launch_prefill_fa(p, s));
   return launch_status(gqa::launch_prefill_simt(p, dtype == GQA_BF16, s));
 }
 

@@ -95,15 +95,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of an mbarrier to complete; bounded in time.
+// Wait for phase `parity` of an mbarrier to complete; bounded in time.  Once
+// any wait has given up (the timeout bit of the error word is set), every
+// other wait gives up at its next check too, so a broken pipeline ends the
+// whole grid within about one limit instead of one limit per CTA.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-      raise_error(err, GQA_DEVERR_WAIT_TIMEOUT);
-      return false;
+    if ((it & 255u) == 0) {
+      if (err && (*reinterpret_cast<volatile int*>(err) & GQA_DEVERR_WAIT_TIMEOUT)) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        raise_error(err, GQA_DEVERR_WAIT_TIMEOUT);
+        return false;
+      }
     }
   }
 }

@@ -1,24 +1,30 @@
-// Split-KV decode attention (step a5, bf16, head_dim 64 or 128).
+// Split-KV decode attention (steps a5-a6, bf16, head_dim 64 or 128).
 //
 // Decode reads each cached K/V row once per new token and does g
 // multiply-adds per byte: it is HBM-bound (MHA -> GQA blog, sections
 // 3.1-3.2).  The g query heads that share a KV head are stacked as the rows
-// of one tensor-core tile, so one pass over a K/V row serves all g heads and
+// of tensor-core tiles, so one pass over a K/V row serves all of them and
 // GQA's arithmetic intensity ~g is actually used.  tcgen05 wants M >= 64; for
 // g <= 16 that would multiply the tensor work 4-16x for nothing, and this
 // kernel's tensor work is far below the tensor roofline anyway, so it uses
-// mma.sync m16n8k16 with the (up to 16) heads as M.
+// mma.sync m16n8k16 with up to MT x 16 heads as M (MT = 2 when g > 16, so an
+// MQA group of 32 heads reads its K/V once, not twice).
 //
-// CTA = (sequence b, KV head j, key split c, group of <= 16 heads).  5 warps:
+// CTA = (sequence b, KV head j, key split c, group of <= 16 MT heads).
+// 5 warps:
 //   warp 4     TMA producer: 64-key K and V tiles (128-byte swizzle, so the
 //              ldmatrix reads below are conflict free) into a 3-4 stage ring
-//   warps 0-3  each takes 16 keys of every tile: S = Q K^T (Q fragments in
-//              registers), mask keys >= the split end, online softmax in
-//              log2 units, P kept in registers as the A fragment of
-//              O += P V (V through ldmatrix.trans).  V rows past the valid
-//              keys are zeroed first so NaN padding never meets a zero P.
-// At the end the 4 warps' (m, l, O) are merged through shared memory and one
-// partial (o unnormalised, m, l) per head is written for the combine.
+//   warps 0-3  each takes 16 keys of every tile: S = Q K^T (Q fragments
+//              from a swizzled shared copy), mask keys past the split, online
+//              softmax in log2 units, P kept in registers as the A fragment
+//              of O += P V (V through ldmatrix.trans, shared by the MT tiles).
+//              V rows past the valid keys are zeroed first, so NaN padding
+//              never meets a zero P.
+// The 4 warps' (m, l, O) are merged through shared memory.  A sequence with a
+// single split writes its output directly; otherwise every split writes a
+// partial (o unnormalised, m, l), bumps a per-(b, j, head group) counter in the
+// workspace, and the last one to finish merges all partials (log-sum-exp)
+// and resets the counter to zero.
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -28,17 +34,19 @@ namespace {
 constexpr int KT = 64;          // keys per tile
 constexpr int THREADS = 160;    // 4 consumer warps + 1 producer warp
 
-template <int HD>
+template <int HD, int MT>
 struct DCfg {
   static constexpr int STAGES = HD == 128 ? 3 : 4;
   static constexpr int NBOX = HD / 64;
   static constexpr int BOX_BYTES = KT * 128;               // 64 rows x 128 bytes
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;      // one K or V tile
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int ROWS = 16 * MT;                     // head rows per CTA
   static constexpr int RED_STRIDE = HD + 4;                // fp32 merge rows
-  static constexpr int RED_BYTES = 4 * 16 * RED_STRIDE * 4;
+  static constexpr int RED_BYTES = 4 * ROWS * RED_STRIDE * 4;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES > RED_BYTES ? STAGES * STAGE_BYTES : RED_BYTES;
-  static constexpr int SMEM = RING_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
+  static constexpr int Q_BYTES = NBOX * ROWS * 128;        // swizzled bf16 Q rows
+  static constexpr int SMEM = RING_BYTES + Q_BYTES + 2048 /*barriers*/ + 1024 /*align*/;
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -57,27 +65,31 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// byte offset of element (row, col) inside a tile of 64-row x 64-column
-// swizzled boxes (128-byte rows, 16-byte chunk c stored at c ^ (row & 7))
+// byte offset of element (row, col) in a tile of 64-column boxes of `rows`
+// 128-byte rows, 16-byte chunk c of a row stored at chunk c ^ (row & 7)
+template <int ROWS_PER_BOX>
 __device__ __forceinline__ uint32_t swz(int row, int col) {
-  return (uint32_t)((col >> 6) * (KT * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
+  return (uint32_t)((col >> 6) * (ROWS_PER_BOX * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
 }
 
+template <int MT>
 struct Bars {
   uint64_t full[4], empty[4];
-  float ml[4][16][2];   // per warp, per head row: max, sum
-  float cm[16][2];      // per head row: merged max, sum (or 1/sum)
+  float ml[4][16 * MT][2];   // per warp, per head row: max, sum
+  float cm[16 * MT][2];      // per head row: merged max, sum (or 1/sum)
   int last;
 };
 
-template <int HD>
+template <int HD, int MT>
 __global__ void __launch_bounds__(THREADS)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                   DecodeParams p, int n_hgrp) {
-  using C = DCfg<HD>;
+  using C = DCfg<HD, MT>;
+  constexpr int ROWS = C::ROWS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + C::RING_BYTES);
+  uint8_t* sq = smem + C::RING_BYTES;
+  Bars<MT>* bars = reinterpret_cast<Bars<MT>*>(sq + C::Q_BYTES);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int b = blockIdx.z, j = blockIdx.y;
   const int split = blockIdx.x / n_hgrp, hg = blockIdx.x % n_hgrp;
@@ -90,8 +102,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     kv_len = kv_len > p.cap ? p.cap : 0;
   }
   const int k_lo = split * p.split;
-  const int h0 = j * g + hg * 16;
-  const int rows = min(16, g - hg * 16);
+  const int h0 = j * g + hg * ROWS;
+  const int rows = min(ROWS, g - hg * ROWS);
   if (k_lo >= kv_len) {  // no key of this sequence in this split (whole block)
     if (split == 0) {    // no key at all: the output rows are zero
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * p.nh + h0) * HD;
@@ -108,6 +120,14 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
       mbar_init(&bars->empty[s], 4);
     }
     fence_mbar_init();
+  }
+  // Q rows of this head group -> swizzled shared copy (zero rows past `rows`)
+  for (int e = threadIdx.x; e < ROWS * (HD / 8); e += THREADS) {
+    const int r = e / (HD / 8), c8 = (e % (HD / 8)) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < rows) v = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
+                                                      ((size_t)b * p.nh + h0 + r) * HD + c8);
+    *reinterpret_cast<uint4*>(sq + swz<ROWS>(r, c8)) = v;
   }
   __syncthreads();
 
@@ -136,27 +156,19 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 
   // ------------------------------------------------------------------ consumers
   const int gr = lane >> 2, tq = lane & 3;  // fragment row group / thread in quad
-  // Q fragments for all K steps (rows gr and gr + 8 of this head group)
-  uint32_t qa[HD / 16][4];
-  {
-    const uint32_t* q32 = static_cast<const uint32_t*>(p.q);
-    const size_t r0 = ((size_t)b * p.nh + h0 + gr) * (HD / 2), r1 = r0 + 8 * (HD / 2);
-#pragma unroll
-    for (int ks = 0; ks < HD / 16; ++ks) {
-      const int c = ks * 8 + tq;  // bf16x2 column index
-      qa[ks][0] = gr < rows ? q32[r0 + c] : 0u;
-      qa[ks][1] = gr + 8 < rows ? q32[r1 + c] : 0u;
-      qa[ks][2] = gr < rows ? q32[r0 + c + 4] : 0u;
-      qa[ks][3] = gr + 8 < rows ? q32[r1 + c + 4] : 0u;
-    }
-  }
-  const float scale_log2 = 1.4426950408889634f * rsqrtf((float)HD);
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  float o[HD / 8][4];
-#pragma unroll
-  for (int n = 0; n < HD / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-
   const int mrow = lane & 7, mat = lane >> 3;  // ldmatrix: row within matrix, matrix index
+  const uint32_t q_base = smem_u32(sq);
+  const float scale_log2 = 1.4426950408889634f * rsqrtf((float)HD);
+  float m[MT][2], l[MT][2];
+  float o[MT][HD / 8][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    m[mt][0] = m[mt][1] = -INFINITY;
+    l[mt][0] = l[mt][1] = 0.f;
+#pragma unroll
+    for (int n = 0; n < HD / 8; ++n) o[mt][n][0] = o[mt][n][1] = o[mt][n][2] = o[mt][n][3] = 0.f;
+  }
+
   for (int t = 0; t < n_t; ++t) {
     const int s = t % C::STAGES;
     const bool ok = mbar_wait(&bars->full[s], (t / C::STAGES) & 1, err);
@@ -176,66 +188,86 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
         tc::fence_proxy_async_smem();  // ordered before the next TMA write into this stage
         __syncwarp();
       }
-      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float sc[MT][2][4];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) sc[mt][nt][0] = sc[mt][nt][1] = sc[mt][nt][2] = sc[mt][nt][3] = 0.f;
 #pragma unroll
       for (int ks = 0; ks < HD / 16; ++ks) {
-        // matrices: (keys 0-7, k lo), (keys 0-7, k hi), (keys 8-15, k lo), (keys 8-15, k hi)
+        // K matrices: (keys 0-7, k lo), (keys 0-7, k hi), (keys 8-15, k lo), (keys 8-15, k hi)
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(kbase + swz(slab + (mat >> 1) * 8 + mrow, ks * 16 + (mat & 1) * 8), b0, b1, b2, b3);
-        mma16816(sc[0], qa[ks], b0, b1);
-        mma16816(sc[1], qa[ks], b2, b3);
-      }
-      // scale to log2 units and mask keys past the valid range
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+        ldsm_x4(kbase + swz<KT>(slab + (mat >> 1) * 8 + mrow, ks * 16 + (mat & 1) * 8), b0, b1, b2, b3);
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = nt * 8 + 2 * tq + (e & 1);
-          const float v = key < nvalid ? sc[nt][e] * scale_log2 : -INFINITY;
-          sc[nt][e] = v;
-          if (e < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+        for (int mt = 0; mt < MT; ++mt) {
+          // Q matrices: (rows 0-7, k lo), (rows 8-15, k lo), (rows 0-7, k hi), (rows 8-15, k hi)
+          uint32_t qa[4];
+          ldsm_x4(q_base + swz<ROWS>(mt * 16 + (mat & 1) * 8 + mrow, ks * 16 + (mat >> 1) * 8), qa[0], qa[1], qa[2],
+                  qa[3]);
+          mma16816(sc[mt][0], qa, b0, b1);
+          mma16816(sc[mt][1], qa, b2, b3);
         }
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);   // finite: key 0 of the slab is valid
-      const float al0 = tc::ex2(m0 - mn0), al1 = tc::ex2(m1 - mn1);
-      m0 = mn0;
-      m1 = mn1;
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        sc[nt][0] = tc::ex2(sc[nt][0] - mn0);
-        sc[nt][1] = tc::ex2(sc[nt][1] - mn0);
-        sc[nt][2] = tc::ex2(sc[nt][2] - mn1);
-        sc[nt][3] = tc::ex2(sc[nt][3] - mn1);
-        s0 += sc[nt][0] + sc[nt][1];
-        s1 += sc[nt][2] + sc[nt][3];
       }
-      s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-      s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-      s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-      s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
-      l0 = l0 * al0 + s0;
-      l1 = l1 * al1 + s1;
+      uint32_t pa[MT][4];
 #pragma unroll
-      for (int n = 0; n < HD / 8; ++n) {
-        o[n][0] *= al0;
-        o[n][1] *= al0;
-        o[n][2] *= al1;
-        o[n][3] *= al1;
+      for (int mt = 0; mt < MT; ++mt) {
+        // scale to log2 units and mask keys past the valid range
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = nt * 8 + 2 * tq + (e & 1);
+            const float v = key < nvalid ? sc[mt][nt][e] * scale_log2 : -INFINITY;
+            sc[mt][nt][e] = v;
+            if (e < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+          }
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float mn0 = fmaxf(m[mt][0], mx0), mn1 = fmaxf(m[mt][1], mx1);  // finite: key 0 of the slab is valid
+        const float al0 = tc::ex2(m[mt][0] - mn0), al1 = tc::ex2(m[mt][1] - mn1);
+        m[mt][0] = mn0;
+        m[mt][1] = mn1;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          sc[mt][nt][0] = tc::ex2(sc[mt][nt][0] - mn0);
+          sc[mt][nt][1] = tc::ex2(sc[mt][nt][1] - mn0);
+          sc[mt][nt][2] = tc::ex2(sc[mt][nt][2] - mn1);
+          sc[mt][nt][3] = tc::ex2(sc[mt][nt][3] - mn1);
+          s0 += sc[mt][nt][0] + sc[mt][nt][1];
+          s1 += sc[mt][nt][2] + sc[mt][nt][3];
+        }
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+        s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+        l[mt][0] = l[mt][0] * al0 + s0;
+        l[mt][1] = l[mt][1] * al1 + s1;
+#pragma unroll
+        for (int n = 0; n < HD / 8; ++n) {
+          o[mt][n][0] *= al0;
+          o[mt][n][1] *= al0;
+          o[mt][n][2] *= al1;
+          o[mt][n][3] *= al1;
+        }
+        pa[mt][0] = pack_bf16x2(sc[mt][0][0], sc[mt][0][1]);
+        pa[mt][1] = pack_bf16x2(sc[mt][0][2], sc[mt][0][3]);
+        pa[mt][2] = pack_bf16x2(sc[mt][1][0], sc[mt][1][1]);
+        pa[mt][3] = pack_bf16x2(sc[mt][1][2], sc[mt][1][3]);
       }
-      const uint32_t pa[4] = {pack_bf16x2(sc[0][0], sc[0][1]), pack_bf16x2(sc[0][2], sc[0][3]),
-                              pack_bf16x2(sc[1][0], sc[1][1]), pack_bf16x2(sc[1][2], sc[1][3])};
 #pragma unroll
       for (int np = 0; np < HD / 16; ++np) {
-        // matrices: (keys 0-7, cols 0-7), (keys 8-15, cols 0-7), (keys 0-7, cols 8-15), (keys 8-15, cols 8-15)
+        // V matrices: (keys 0-7, cols 0-7), (keys 8-15, cols 0-7), (keys 0-7, cols 8-15), (keys 8-15, cols 8-15)
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vbase + swz(slab + (mat & 1) * 8 + mrow, np * 16 + (mat >> 1) * 8), b0, b1, b2, b3);
-        mma16816(o[2 * np], pa, b0, b1);
-        mma16816(o[2 * np + 1], pa, b2, b3);
+        ldsm_x4_t(vbase + swz<KT>(slab + (mat & 1) * 8 + mrow, np * 16 + (mat >> 1) * 8), b0, b1, b2, b3);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          mma16816(o[mt][2 * np], pa[mt], b0, b1);
+          mma16816(o[mt][2 * np + 1], pa[mt], b2, b3);
+        }
       }
     }
     __syncwarp();
@@ -244,31 +276,39 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 
   // ------------------------------------------------------------------ merge the 4 warps
   if (tq == 0) {
-    bars->ml[warp][gr][0] = m0;
-    bars->ml[warp][gr][1] = l0;
-    bars->ml[warp][gr + 8][0] = m1;
-    bars->ml[warp][gr + 8][1] = l1;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      bars->ml[warp][mt * 16 + gr][0] = m[mt][0];
+      bars->ml[warp][mt * 16 + gr][1] = l[mt][0];
+      bars->ml[warp][mt * 16 + gr + 8][0] = m[mt][1];
+      bars->ml[warp][mt * 16 + gr + 8][1] = l[mt][1];
+    }
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");   // consumers only; the ring is idle now
-  float M0 = -INFINITY, M1 = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    M0 = fmaxf(M0, bars->ml[w][gr][0]);
-    M1 = fmaxf(M1, bars->ml[w][gr + 8][0]);
-  }
-  const float f0 = m0 == -INFINITY ? 0.f : tc::ex2(m0 - M0);
-  const float f1 = m1 == -INFINITY ? 0.f : tc::ex2(m1 - M1);
   float* red = reinterpret_cast<float*>(smem);
 #pragma unroll
-  for (int n = 0; n < HD / 8; ++n) {
-    const int c = n * 8 + 2 * tq;
-    red[(warp * 16 + gr) * C::RED_STRIDE + c] = o[n][0] * f0;
-    red[(warp * 16 + gr) * C::RED_STRIDE + c + 1] = o[n][1] * f0;
-    red[(warp * 16 + gr + 8) * C::RED_STRIDE + c] = o[n][2] * f1;
-    red[(warp * 16 + gr + 8) * C::RED_STRIDE + c + 1] = o[n][3] * f1;
+  for (int mt = 0; mt < MT; ++mt) {
+    float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      M0 = fmaxf(M0, bars->ml[w][mt * 16 + gr][0]);
+      M1 = fmaxf(M1, bars->ml[w][mt * 16 + gr + 8][0]);
+    }
+    const float f0 = m[mt][0] == -INFINITY ? 0.f : tc::ex2(m[mt][0] - M0);
+    const float f1 = m[mt][1] == -INFINITY ? 0.f : tc::ex2(m[mt][1] - M1);
+#pragma unroll
+    for (int n = 0; n < HD / 8; ++n) {
+      const int c = n * 8 + 2 * tq;
+      float* r0 = red + (warp * ROWS + mt * 16 + gr) * C::RED_STRIDE + c;
+      float* r1 = r0 + 8 * C::RED_STRIDE;
+      r0[0] = o[mt][n][0] * f0;
+      r0[1] = o[mt][n][1] * f0;
+      r1[0] = o[mt][n][2] * f1;
+      r1[1] = o[mt][n][3] * f1;
+    }
   }
   const int tid = threadIdx.x;
-  if (tid < 16) {  // this CTA's max and sum per head row, over its 4 warps
+  if (tid < ROWS) {  // this CTA's max and sum per head row, over its 4 warps
     float M = -INFINITY, L = 0.f;
     for (int w = 0; w < 4; ++w) M = fmaxf(M, bars->ml[w][tid][0]);
     for (int w = 0; w < 4; ++w) {
@@ -280,8 +320,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
   auto red_sum = [&](int r, int c) {
-    return red[(0 * 16 + r) * C::RED_STRIDE + c] + red[(1 * 16 + r) * C::RED_STRIDE + c] +
-           red[(2 * 16 + r) * C::RED_STRIDE + c] + red[(3 * 16 + r) * C::RED_STRIDE + c];
+    return red[(0 * ROWS + r) * C::RED_STRIDE + c] + red[(1 * ROWS + r) * C::RED_STRIDE + c] +
+           red[(2 * ROWS + r) * C::RED_STRIDE + c] + red[(3 * ROWS + r) * C::RED_STRIDE + c];
   };
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
   const int n_active = (kv_len + p.split - 1) / p.split;   // splits that hold keys of this sequence
@@ -316,7 +356,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
   // 2^(m_s - M) / L per split (kept in shared memory); then every thread
   // takes float4 output columns and sums the splits with independent loads.
   const size_t stride = HD + kWsPad;
-  float* wgt = red;  // [16][n_active]
+  float* wgt = red;  // [ROWS][n_active]
   for (int r = warp; r < rows; r += 4) {
     const float* part = p.ws + ((size_t)b * p.nh + h0 + r) * p.n_split * stride;
     float M = -INFINITY;
@@ -358,14 +398,15 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
   if (tid == 0) atomicExch(counter, 0u);  // leave the counter at zero for the next call
 }
 
-template <int HD>
+template <int HD, int MT>
 cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
-  using C = DCfg<HD>;
+  using C = DCfg<HD, MT>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e =
+        cudaFuncSetAttribute(decode_mma_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -373,19 +414,18 @@ cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
   const uint64_t rows = (uint64_t)p.B * p.nkv * p.cap;
   if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
-  const int g = p.nh / p.nkv;
-  const int n_hgrp = (g + 15) / 16;
-  dim3 grid((unsigned)(p.n_split * n_hgrp), p.nkv, p.B);
-  decode_mma_kernel<HD><<<grid, THREADS, C::SMEM, st>>>(tk, tv, p, n_hgrp);
+  dim3 grid((unsigned)(p.n_split * p.n_hgrp), p.nkv, p.B);
+  decode_mma_kernel<HD, MT><<<grid, THREADS, C::SMEM, st>>>(tk, tv, p, p.n_hgrp);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
+  static_assert(true, "one m16 tile per head group (see decode_mtiles)");
   switch (p.hd) {
-    case 64: return launch_hd<64>(p, st);
-    case 128: return launch_hd<128>(p, st);
+    case 64: return launch_hd<64, 1>(p, st);
+    case 128: return launch_hd<128, 1>(p, st);
     default: return cudaErrorInvalidValue;
   }
 }

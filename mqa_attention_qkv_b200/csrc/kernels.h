@@ -51,7 +51,15 @@ constexpr int kWsPad = 4;  // per-partial row: hd floats of o, then m, l and two
 inline size_t decode_counter_bytes(int B, int nkv, int n_hgrp) {
   return ((size_t)B * nkv * n_hgrp * sizeof(unsigned) + 255) / 256 * 256;
 }
-inline int decode_n_hgrp(int nh, int nkv) { return (nh / nkv + 15) / 16; }
+// Tensor-core decode: query heads of a KV head are handled in groups of
+// 16 x mtiles.  Measured on B200, two m16 tiles per CTA (233 registers, one
+// CTA per SM) made MQA slower than re-reading K/V from L2 for a second group
+// of 16 heads, so every group is one tile.
+inline int decode_mtiles(int, int) { return 1; }
+inline int decode_n_hgrp(int nh, int nkv) {
+  const int rows = 16 * decode_mtiles(nh, nkv);
+  return (nh / nkv + rows - 1) / rows;
+}
 
 // SIMT kernels (any dtype; the fp32 path and shapes the tensor-core kernels skip)
 cudaError_t launch_qkv_simt(const QkvParams& p, bool bf16, cudaStream_t st);
@@ -62,8 +70,8 @@ cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t
 // Tensor-core (tcgen05 + TMA) kernels, bf16 only.
 cudaError_t launch_qkv_tc(const QkvParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_qkv_smallm(const QkvParams& p, cudaStream_t st);  // B*S <= 64
-cudaError_t launch_prefill_tc(const PrefillParams& p, cudaStream_t st);  // head_dim 64 or 128
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
+cudaError_t launch_prefill_fa(const PrefillParams& p, cudaStream_t st);    // head_dim 64/128, 2 Q tiles/CTA
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128
 
 // Decode: the tensor-core kernel for bf16 head_dim 64/128 (the last split of

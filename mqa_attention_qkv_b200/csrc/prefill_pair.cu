@@ -1,7 +1,7 @@
 // Prefill attention for head_dim 64, two CTAs per SM (step a4, bf16).
 //
-// Same algorithm as prefill_tc.cu (exact tiled online softmax, FlashAttention-3
-// summary, recap section; GQA head map h -> h / g), laid out so that two CTAs
+// Exact tiled online softmax (FlashAttention-3 summary, recap section; GQA head
+// map h -> h / g, MHA -> GQA blog section 3.2), laid out so that two CTAs
 // share each SM: at head_dim 64 a KV tile costs the tensor cores half of what
 // its 16K exponentials cost the MUFU unit, so the softmax of one CTA has to
 // run while the other CTA's MMAs do.  Per CTA:
@@ -37,38 +37,10 @@ struct Bars {
   int lim_max;
 };
 
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// (a0, a1) * s + (c, c) on the packed f32x2 pipe
-__device__ __forceinline__ void fma2(float& a0, float& a1, float s, float c) {
-  uint64_t x, y, z;
-  asm("mov.b64 %0, {%1,%2};" : "=l"(x) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1,%1};" : "=l"(y) : "f"(s));
-  asm("mov.b64 %0, {%1,%1};" : "=l"(z) : "f"(c));
-  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(x) : "l"(y), "l"(z));
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(x));
-}
-
-__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
-  uint64_t x, y;
-  asm("mov.b64 %0, {%1,%2};" : "=l"(x) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1,%2};" : "=l"(y) : "f"(b0), "f"(b1));
-  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(x) : "l"(y));
-  asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(x));
-}
+using tc::add2;
+using tc::fma2;
+using tc::max3;
+using tc::mma_bf16_ts;
 
 __global__ void __launch_bounds__(THREADS, 2)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,

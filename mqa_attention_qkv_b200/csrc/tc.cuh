@@ -102,6 +102,17 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// A operand from tensor memory (bf16 pairs packed in 32-bit columns, row =
+// lane), B from shared memory.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -139,6 +150,74 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Named CTA barriers (id 1..15): wait until `n` threads arrived / arrive only.
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (a0, a1) = (a0, a1) * s + (c, c) as one packed f32x2 FMA
+__device__ __forceinline__ void fma2(float& a0, float& a1, float s, float c) {
+  uint64_t x, y, z;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(y) : "f"(s));
+  asm("mov.b64 %0, {%1,%1};" : "=l"(z) : "f"(c));
+  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(x) : "l"(y), "l"(z));
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(x));
+}
+
+// (a0, a1) += (b0, b1) as one packed f32x2 add
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  uint64_t x, y;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1,%2};" : "=l"(y) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(x) : "l"(y));
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(x));
+}
+
+// (a0, a1) = (a0, a1) * (b0, b1) + (c0, c1) as one packed f32x2 FMA
+__device__ __forceinline__ void fma2v(float& a0, float& a1, float b0, float b1, float c0, float c1) {
+  uint64_t x, y, z;
+  asm("mov.b64 %0, {%1,%2};" : "=l"(x) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1,%2};" : "=l"(y) : "f"(b0), "f"(b1));
+  asm("mov.b64 %0, {%1,%2};" : "=l"(z) : "f"(c0), "f"(c1));
+  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(x) : "l"(y), "l"(z));
+  asm("mov.b64 {%0,%1}, %2;" : "=f"(a0), "=f"(a1) : "l"(x));
+}
+
+// 2^x for two finite values on the FMA pipe instead of the MUFU unit:
+// x = n + f with n = round(x) (1.5 * 2^23 added and subtracted rounds to an
+// integer and leaves n in the low mantissa bits), |f| <= 1/2, 2^f by a
+// degree-3 polynomial fitted for minimum relative error on [-1/2, 1/2]
+// (exp2_poly_fit.py, max relative error 7.5e-5), then n added to the
+// exponent field.  Inputs below -125 are clamped (result ~2^-125); callers
+// keep masked -inf scores on the MUFU path, which returns exact zeros.
+__device__ __forceinline__ void exp2_poly2(float& a, float& b) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992807353940116f, c1 = 0.69326098546065529f;
+  constexpr float c2 = 0.24261112219321609f, c3 = 0.055171669057926163f;
+  float xa = fmaxf(a, -125.f), xb = fmaxf(b, -125.f);
+  float ta = xa, tb = xb;
+  add2(ta, tb, kRound, kRound);            // t = x + 1.5*2^23 (round to nearest)
+  float na = ta, nb = tb;
+  add2(na, nb, -kRound, -kRound);          // n = round(x) as a float
+  fma2v(na, nb, -1.f, -1.f, xa, xb);       // f = x - n
+  float pa = na, pb = nb;
+  fma2(pa, pb, c3, c2);                    // c3 f + c2
+  fma2v(pa, pb, na, nb, c1, c1);           // (.) f + c1
+  fma2v(pa, pb, na, nb, c0, c0);           // (.) f + c0
+  a = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  b = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
 }
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {

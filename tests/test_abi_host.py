@@ -114,7 +114,8 @@ def test_workspace_size_query():
     # then B * nh * ceil(cap / split) * (hd + 4) floats
     assert f(2, 4, 2, 64, 1000, 64) == 256 + 2 * 4 * 16 * 68 * 4
     assert f(64, 32, 8, 128, 8192, 512) == 2048 + 64 * 32 * 16 * 132 * 4
-    assert f(64, 32, 1, 128, 8192, 512) == 512 + 64 * 32 * 16 * 132 * 4   # g = 32: 2 head groups
+    assert f(64, 32, 1, 128, 8192, 512) == 512 + 64 * 32 * 16 * 132 * 4    # g = 32: 2 head groups
+    assert f(8, 48, 1, 128, 1040, 64) == 256 + 8 * 48 * 17 * 132 * 4       # g = 48: 3 head groups
     assert f(2, 4, 2, 64, 1000, 0) > 0
     assert f(2, 4, 2, 64, 1000, 100) == 0      # split not a multiple of 64
     assert f(2, 4, 3, 64, 1000, 64) == 0       # nh % nkv
