@@ -160,7 +160,7 @@ size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int he
  *   kv_lens    [B] int32: valid keys including the new token; clamped to
  *              [0, cache_cap] (GQA_DEVERR_KVLEN_RANGE); 0 gives a zero row
  *   kv_split   keys per split: 0 = automatic, else a positive multiple of 64
- *              giving at most 1024 splits of cache_cap
+ *              giving at most 512 splits of cache_cap
  *   out        [B, n_heads, head_dim] dtype
  *   workspace  device scratch of at least gqa_attn_decode_workspace_size()
  *              bytes, 16-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE

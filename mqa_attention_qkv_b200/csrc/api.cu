@@ -71,7 +71,7 @@ int launch_status(cudaError_t e, int n_launched = 1) {
 // 2048, a multiple of 64, and never more than kMaxSplits splits.  (Eight
 // units per SM, tried for ragged MQA batches, measured slower on B200.)
 constexpr long long kUnitsWanted = 2 * 148;
-constexpr int kMaxSplits = 1024;
+using gqa::kMaxSplits;
 int auto_split(int B, int nkv, int n_hgrp, int cap) {
   const long long groups = (long long)B * nkv * n_hgrp;
   long long s = (groups * cap + kUnitsWanted - 1) / kUnitsWanted;
@@ -110,7 +110,7 @@ DecodeParams decode_params(const void* q, const void* k_cache, const void* v_cac
   unsigned* counters = static_cast<unsigned*>(workspace);
   float* partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_counter_bytes(B, nkv, n_hgrp));
   return DecodeParams{q, k_cache, v_cache, kv_lens, B, nh, nkv, hd, cap, split, (cap + split - 1) / split,
-                      partials, out, err, counters, n_hgrp};
+                      partials, out, err, counters, n_hgrp, kv_split == 0, 0};
 }
 
 }  // namespace gqa
@@ -177,7 +177,7 @@ int qkv_rope_project(const void* x, const void* w_qkv, const int32_t* positions,
   // Tensor-core path: bf16 with 16-byte-aligned rows (TMA row stride).
   if (dtype == GQA_BF16 && hidden % 8 == 0) {
     // a few tokens: W-streaming kernel spread over every SM; else 128-token tiles
-    if ((long long)B * S <= 64) return launch_status(gqa::launch_qkv_smallm(p, s));
+    if ((long long)B * S <= 64) return launch_status(gqa::launch_qkv_smallm(p, d->num_sms, s));
     return launch_status(gqa::launch_qkv_tc(p, d->num_sms, s));
   }
   return launch_status(gqa::launch_qkv_simt(p, dtype == GQA_BF16, s));

@@ -7,10 +7,10 @@
 // GQA's arithmetic intensity ~g is actually used.  tcgen05 wants M >= 64; for
 // g <= 16 that would multiply the tensor work 4-16x for nothing, and this
 // kernel's tensor work is far below the tensor roofline anyway, so it uses
-// mma.sync m16n8k16 with up to MT x 16 heads as M (MT = 2 when g > 16, so an
-// MQA group of 32 heads reads its K/V once, not twice).
+// mma.sync m16n8k16 with 16 heads as M (g > 16: several head groups, each
+// reading the K/V rows, the second time mostly from L2).
 //
-// CTA = (sequence b, KV head j, key split c, group of <= 16 MT heads).
+// CTA = (sequence b, KV head j, key split c, group of <= 16 heads).
 // 5 warps:
 //   warp 4     TMA producer: 64-key K and V tiles (128-byte swizzle, so the
 //              ldmatrix reads below are conflict free) into a 3-4 stage ring
@@ -21,10 +21,17 @@
 //              V rows past the valid keys are zeroed first, so NaN padding
 //              never meets a zero P.
 // The 4 warps' (m, l, O) are merged through shared memory.  A sequence with a
-// single split writes its output directly; otherwise every split writes a
-// partial (o unnormalised, m, l), bumps a per-(b, j, head group) counter in the
-// workspace, and the last one to finish merges all partials (log-sum-exp)
-// and resets the counter to zero.
+// single split writes its output directly.  Splits are then merged
+// (log-sum-exp) in one of two ways:
+//   cluster mode (the library picks the split, <= 8 per group): the splits of
+//     a (b, j, head group) are one thread-block cluster; each sequence's
+//     64-key tiles are dealt out evenly over its CTAs, and the CTAs read one
+//     another's partials from distributed shared memory -- no workspace round
+//     trip, which is what a small decode step's latency is made of;
+//   workspace mode (fixed kv_split keys per split, or longer caches): every
+//     split writes a partial (o unnormalised, m, l) to the workspace, bumps a
+//     per-(b, j, head group) counter, and the last one to finish merges all
+//     partials and resets the counter to zero.
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -32,6 +39,7 @@ namespace gqa {
 namespace {
 
 constexpr int KT = 64;          // keys per tile
+constexpr int kMaxClusterSplits = 8;  // portable cluster size
 constexpr int THREADS = 160;    // 4 consumer warps + 1 producer warp
 
 template <int HD, int MT>
@@ -47,6 +55,8 @@ struct DCfg {
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES > RED_BYTES ? STAGES * STAGE_BYTES : RED_BYTES;
   static constexpr int Q_BYTES = NBOX * ROWS * 128;        // swizzled bf16 Q rows
   static constexpr int SMEM = RING_BYTES + Q_BYTES + 2048 /*barriers*/ + 1024 /*align*/;
+  // the final merge keeps (m, l) of every (head row, split) pair in the ring
+  static_assert(ROWS * kMaxSplits * 8 <= RING_BYTES, "split merge does not fit in shared memory");
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -80,7 +90,7 @@ struct Bars {
   int last;
 };
 
-template <int HD, int MT>
+template <int HD, int MT, bool CL>
 __global__ void __launch_bounds__(THREADS)
 decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                   DecodeParams p, int n_hgrp) {
@@ -92,7 +102,10 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
   Bars<MT>* bars = reinterpret_cast<Bars<MT>*>(sq + C::Q_BYTES);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int b = blockIdx.z, j = blockIdx.y;
-  const int split = blockIdx.x / n_hgrp, hg = blockIdx.x % n_hgrp;
+  // cluster mode: the n_split CTAs of one (sequence, KV head, head group)
+  // are consecutive in x and form one cluster
+  const int split = CL ? blockIdx.x % p.n_split : blockIdx.x / n_hgrp;
+  const int hg = CL ? blockIdx.x / p.n_split : blockIdx.x % n_hgrp;
   const int g = p.nh / p.nkv;
   int* err = p.err;
 
@@ -101,18 +114,29 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     if (threadIdx.x == 0 && split == 0 && hg == 0) raise_error(err, GQA_DEVERR_KVLEN_RANGE);
     kv_len = kv_len > p.cap ? p.cap : 0;
   }
-  const int k_lo = split * p.split;
   const int h0 = j * g + hg * ROWS;
   const int rows = min(ROWS, g - hg * ROWS);
-  if (k_lo >= kv_len) {  // no key of this sequence in this split (whole block)
-    if (split == 0) {    // no key at all: the output rows are zero
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * p.nh + h0) * HD;
-      for (int e = threadIdx.x; e < rows * HD; e += blockDim.x) out[e] = __float2bfloat16_rn(0.f);
+  int k_lo, k_hi, n_t;
+  if (CL) {
+    // the sequence's 64-key tiles dealt out evenly over the cluster; a CTA
+    // may get none and still takes part in the merge
+    const int tiles = (kv_len + KT - 1) / KT;
+    const int t_lo = split * tiles / p.n_split, t_hi = (split + 1) * tiles / p.n_split;
+    k_lo = t_lo * KT;
+    k_hi = min(kv_len, t_hi * KT);
+    n_t = t_hi - t_lo;
+  } else {
+    k_lo = split * p.split;
+    if (k_lo >= kv_len) {  // no key of this sequence in this split (whole block)
+      if (split == 0) {    // no key at all: the output rows are zero
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + ((size_t)b * p.nh + h0) * HD;
+        for (int e = threadIdx.x; e < rows * HD; e += blockDim.x) out[e] = __float2bfloat16_rn(0.f);
+      }
+      return;
     }
-    return;
+    k_hi = min(kv_len, k_lo + p.split);
+    n_t = (k_hi - k_lo + KT - 1) / KT;
   }
-  const int k_hi = min(kv_len, k_lo + p.split);
-  const int n_t = (k_hi - k_lo + KT - 1) / KT;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -120,14 +144,6 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
       mbar_init(&bars->empty[s], 4);
     }
     fence_mbar_init();
-  }
-  // Q rows of this head group -> swizzled shared copy (zero rows past `rows`)
-  for (int e = threadIdx.x; e < ROWS * (HD / 8); e += THREADS) {
-    const int r = e / (HD / 8), c8 = (e % (HD / 8)) * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < rows) v = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
-                                                      ((size_t)b * p.nh + h0 + r) * HD + c8);
-    *reinterpret_cast<uint4*>(sq + swz<ROWS>(r, c8)) = v;
   }
   __syncthreads();
 
@@ -151,10 +167,36 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
       for (int t = max(0, n_t - C::STAGES); t < n_t; ++t)
         mbar_wait(&bars->full[t % C::STAGES], (t / C::STAGES) & 1, err);
     }
+    __syncwarp();
+    if (CL && p.n_split > 1) {  // the producer warp joins the two cluster barriers of the merge
+      tc::cluster_sync();
+      tc::cluster_sync();
+    }
     return;
   }
 
   // ------------------------------------------------------------------ consumers
+  // Q rows of this head group -> swizzled shared copy (zero rows past
+  // `rows`), while the first K/V tiles are in flight.  All loads are issued
+  // before the first store.
+  {
+    constexpr int QV = ROWS * (HD / 8) / 128;  // 16-byte vectors per consumer thread
+    uint4 v[QV];
+#pragma unroll
+    for (int i = 0; i < QV; ++i) {
+      const int e = threadIdx.x + i * 128, r = e / (HD / 8), c8 = (e % (HD / 8)) * 8;
+      v[i] = make_uint4(0, 0, 0, 0);
+      if (r < rows)
+        v[i] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
+                                               ((size_t)b * p.nh + h0 + r) * HD + c8);
+    }
+#pragma unroll
+    for (int i = 0; i < QV; ++i) {
+      const int e = threadIdx.x + i * 128, r = e / (HD / 8), c8 = (e % (HD / 8)) * 8;
+      *reinterpret_cast<uint4*>(sq + swz<ROWS>(r, c8)) = v[i];
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+  }
   const int gr = lane >> 2, tq = lane & 3;  // fragment row group / thread in quad
   const int mrow = lane & 7, mat = lane >> 3;  // ldmatrix: row within matrix, matrix index
   const uint32_t q_base = smem_u32(sq);
@@ -324,7 +366,53 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
            red[(2 * ROWS + r) * C::RED_STRIDE + c] + red[(3 * ROWS + r) * C::RED_STRIDE + c];
   };
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-  const int n_active = (kv_len + p.split - 1) / p.split;   // splits that hold keys of this sequence
+  if (CL && p.n_split > 1) {
+    // ---------------------------------------------------------- cluster merge
+    // this CTA's o (summed over its 4 warps, relative to its max) in place of
+    // warp 0's rows; (max, sum) per row are in bars->cm
+    for (int e = tid; e < rows * HD; e += 128) {
+      const int r = e / HD, c = e % HD;
+      red[r * C::RED_STRIDE + c] = red_sum(r, c);
+    }
+    tc::cluster_sync();
+    // float4 output pieces dealt out over the cluster's consumer threads; each
+    // reads the n_split partial rows from the CTAs' shared memory
+    const int nsp = p.n_split;
+    const uint32_t red_u = smem_u32(red), cm_u = smem_u32(&bars->cm[0][0]);
+    for (int e = split * 128 + tid; e < rows * (HD / 4); e += nsp * 128) {
+      const int r = e / (HD / 4), c = (e % (HD / 4)) * 4;
+      float2 ml[8];
+      float M = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q < nsp) {
+          ml[q] = tc::ld_dsmem_f32x2(tc::mapa_shared(cm_u + r * 8, q));
+          M = fmaxf(M, ml[q].x);
+        }
+      }
+      float L = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q < nsp && ml[q].x != -INFINITY) {
+          const float w = tc::ex2(ml[q].x - M);
+          const float4 v = tc::ld_dsmem_f32x4(tc::mapa_shared(red_u + (r * C::RED_STRIDE + c) * 4, q));
+          L += ml[q].y * w;
+          acc.x = fmaf(v.x, w, acc.x);
+          acc.y = fmaf(v.y, w, acc.y);
+          acc.z = fmaf(v.z, w, acc.z);
+          acc.w = fmaf(v.w, w, acc.w);
+        }
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * p.nh + h0 + r) * HD + c);
+      dst[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      dst[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    }
+    tc::cluster_sync();  // no CTA leaves while another may still read its shared memory
+    return;
+  }
+  const int n_active = CL ? 1 : (kv_len + p.split - 1) / p.split;   // splits that hold keys of this sequence
   if (n_active == 1) {
     // the only split: normalise and write the output directly
     for (int e = tid; e < rows * HD; e += 128) {
@@ -352,40 +440,46 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
   asm volatile("bar.sync 1, 128;" ::: "memory");
   if (!bars->last) return;
   __threadfence();
-  // merge: per head row, lanes take the splits -> max, sum and one weight
-  // 2^(m_s - M) / L per split (kept in shared memory); then every thread
-  // takes float4 output columns and sums the splits with independent loads.
+  // merge: (1) every (head row, split) pair's (m, l) is fetched at once into
+  // shared memory (one round trip); (2) per head row, lanes over the splits
+  // -> max, sum and one weight 2^(m_s - M) / L per split, from shared memory
+  // only; (3) every thread takes float4 output columns and sums the splits
+  // with independent loads.
   const size_t stride = HD + kWsPad;
-  float* wgt = red;  // [ROWS][n_active]
+  float2* mls = reinterpret_cast<float2*>(red);  // [rows][n_active]: (m, l), then (weight, -)
+  for (int e = tid; e < rows * n_active; e += 128) {
+    const int r = e / n_active, s = e - r * n_active;
+    mls[e] = __ldcg(reinterpret_cast<const float2*>(p.ws + (((size_t)b * p.nh + h0 + r) * p.n_split + s) * stride + HD));
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
   for (int r = warp; r < rows; r += 4) {
-    const float* part = p.ws + ((size_t)b * p.nh + h0 + r) * p.n_split * stride;
+    float2* ml = mls + r * n_active;
     float M = -INFINITY;
-    for (int s = lane; s < n_active; s += 32) M = fmaxf(M, __ldcg(part + s * stride + HD));
+    for (int s = lane; s < n_active; s += 32) M = fmaxf(M, ml[s].x);
 #pragma unroll
     for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
     float L = 0.f;
     for (int s = lane; s < n_active; s += 32) {
-      const float ms = __ldcg(part + s * stride + HD);
-      const float e = ms == -INFINITY ? 0.f : tc::ex2(ms - M);
-      wgt[r * n_active + s] = e;
-      L += __ldcg(part + s * stride + HD + 1) * e;
+      const float2 v = ml[s];
+      const float e = v.x == -INFINITY ? 0.f : tc::ex2(v.x - M);
+      ml[s].x = e;
+      L += v.y * e;
     }
 #pragma unroll
     for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o2);
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    __syncwarp();
-    for (int s = lane; s < n_active; s += 32) wgt[r * n_active + s] *= inv;
+    for (int s = lane; s < n_active; s += 32) ml[s].x *= inv;
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
   for (int e = tid; e < rows * (HD / 4); e += 128) {
     const int r = e / (HD / 4), c = (e % (HD / 4)) * 4;
     const float* part = p.ws + ((size_t)b * p.nh + h0 + r) * p.n_split * stride + c;
-    const float* w = wgt + r * n_active;
+    const float2* w = mls + r * n_active;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
     for (int s = 0; s < n_active; ++s) {
       const float4 v = __ldcg(reinterpret_cast<const float4*>(part + s * stride));
-      const float ws_ = w[s];
+      const float ws_ = w[s].x;
       acc.x = fmaf(v.x, ws_, acc.x);
       acc.y = fmaf(v.y, ws_, acc.y);
       acc.z = fmaf(v.z, ws_, acc.z);
@@ -398,7 +492,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
   if (tid == 0) atomicExch(counter, 0u);  // leave the counter at zero for the next call
 }
 
-template <int HD, int MT>
+template <int HD, int MT, bool CL>
 cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
   using C = DCfg<HD, MT>;
   static bool attr_set[64] = {};
@@ -406,7 +500,7 @@ cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(decode_mma_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaFuncSetAttribute(decode_mma_kernel<HD, MT, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -414,9 +508,39 @@ cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
   const uint64_t rows = (uint64_t)p.B * p.nkv * p.cap;
   if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
-  dim3 grid((unsigned)(p.n_split * p.n_hgrp), p.nkv, p.B);
-  decode_mma_kernel<HD, MT><<<grid, THREADS, C::SMEM, st>>>(tk, tv, p, p.n_hgrp);
-  return cudaGetLastError();
+  const dim3 grid((unsigned)(p.n_split * p.n_hgrp), p.nkv, p.B);
+  if (!CL) {
+    decode_mma_kernel<HD, MT, false><<<grid, THREADS, C::SMEM, st>>>(tk, tv, p, p.n_hgrp);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.n_split;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_mma_kernel<HD, MT, true>, tk, tv, p, p.n_hgrp);
+}
+
+// Splits per (sequence, KV head, head group) for the cluster-merged decode,
+// or 0 to use the workspace splits: about two CTAs per SM over the whole
+// problem and at most 2048 keys a CTA, within one portable cluster (<= 8).
+int cluster_splits(const DecodeParams& p) {
+  const long long groups = (long long)p.B * p.nkv * p.n_hgrp;
+  const int by_len = (p.cap + 2047) / 2048;
+  if (by_len > kMaxClusterSplits) return 0;
+  long long n = (2 * 148 + groups - 1) / groups;
+  if (n < by_len) n = by_len;
+  if (n > kMaxClusterSplits) n = kMaxClusterSplits;
+  const int tiles = (p.cap + KT - 1) / KT;
+  if (n > tiles) n = tiles;
+  return (int)(n < 1 ? 1 : n);
 }
 
 }  // namespace
@@ -424,19 +548,25 @@ cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
   static_assert(true, "one m16 tile per head group (see decode_mtiles)");
   switch (p.hd) {
-    case 64: return launch_hd<64, 1>(p, st);
-    case 128: return launch_hd<128, 1>(p, st);
+    case 64: return p.cluster ? launch_hd<64, 1, true>(p, st) : launch_hd<64, 1, false>(p, st);
+    case 128: return p.cluster ? launch_hd<128, 1, true>(p, st) : launch_hd<128, 1, false>(p, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-int launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st, cudaError_t* err) {
-  if (bf16 && (p.hd == 64 || p.hd == 128)) {  // merges its splits itself
+int launch_decode(const DecodeParams& p0, bool bf16, cudaStream_t st, cudaError_t* err) {
+  if (bf16 && (p0.hd == 64 || p0.hd == 128)) {  // merges its splits itself
+    DecodeParams p = p0;
+    const int nc = p.auto_split ? cluster_splits(p) : 0;
+    if (nc > 0) {
+      p.cluster = 1;
+      p.n_split = nc;
+    }
     *err = launch_decode_mma(p, st);
     return 1;
   }
-  cudaError_t e = launch_decode_simt(p, bf16, st);
-  if (e == cudaSuccess) e = launch_decode_combine(p, bf16, st);
+  cudaError_t e = launch_decode_simt(p0, bf16, st);
+  if (e == cudaSuccess) e = launch_decode_combine(p0, bf16, st);
   *err = e;
   return 2;
 }

@@ -43,7 +43,13 @@ struct DecodeParams {
   int* err;
   unsigned* counters;     // [B, nkv, n_hgrp]: finished splits (zero between calls)
   int n_hgrp;             // groups of <= 16 query heads per KV head
+  int auto_split;         // the caller left the split to the library
+  int cluster;            // set by launch_decode: splits merged inside a thread-block cluster
 };
+
+// Most key splits per sequence: the tensor-core decode's final merge keeps
+// (m, l) of every (head row, split) pair in shared memory.
+constexpr int kMaxSplits = 512;
 
 constexpr int kWsPad = 4;  // per-partial row: hd floats of o, then m, l and two pad words
 
@@ -69,7 +75,7 @@ cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t
 
 // Tensor-core (tcgen05 + TMA) kernels, bf16 only.
 cudaError_t launch_qkv_tc(const QkvParams& p, int num_sms, cudaStream_t st);
-cudaError_t launch_qkv_smallm(const QkvParams& p, cudaStream_t st);  // B*S <= 64
+cudaError_t launch_qkv_smallm(const QkvParams& p, int num_sms, cudaStream_t st);  // B*S <= 64
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
 cudaError_t launch_prefill_fa(const PrefillParams& p, cudaStream_t st);    // head_dim 64/128, 2 Q tiles/CTA
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128
@@ -84,6 +90,10 @@ int launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st, cudaError_t
 // Zero fill outside [0, inner) x [0, outer).  False if encoding fails.
 bool make_tmap_bf16_2d(void* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                        uint32_t box_inner, uint32_t box_outer);
+// 3-D bf16 TMA descriptor with 128-byte swizzle: dims innermost first,
+// strides (bytes) of dims 1 and 2, box extents.  Zero fill outside the dims.
+bool make_tmap_bf16_3d(void* map, const void* base, const uint64_t dims[3], const uint64_t stride_bytes[2],
+                       const uint32_t box[3]);
 
 // Shared by the C-ABI translation units (defined in api.cu).
 int device_check(int** err);  // GQA_OK, or the status for the current device

@@ -6,8 +6,12 @@
 // (N x D) to do 2*T*N*D flops: it is bound by the W stream (the "batch-1 is
 // matrix-vector, memory-bound" case of the MHA -> GQA blog, section 3.1), so
 // the design goal is to spread W over every SM with many bytes in flight.
+// Both kernels below work in units of 16 rows of W (8 RoPE pairs, see the
+// register kernel); the TMA-ring kernel (further down) serves hidden % 64 == 0
+// when the tokens' hidden states fit in shared memory, the register kernel
+// everything else.
 //
-// CTA = 16 rows of W: 8 consecutive features at offset i0 of the first half
+// Register kernel.  CTA = 16 rows of W: 8 consecutive features at offset i0 of the first half
 // of one head and the 8 features i0 + hd/2 of its second half, i.e. 8 RoPE
 // pairs, so the rotation happens inside the CTA.  8 warps split D; each
 // thread streams 16-byte vectors of its W rows (no L1 allocation) and of the
@@ -46,6 +50,39 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Epilogue of one RoPE pair: features i0 + r (lo) and hd/2 + i0 + r (hi) of
+// head block hb for token tok.  Q and K heads are rotated by the token's
+// position (rotate-half form), then Q goes to [B, nh, S, hd] and K/V to
+// cache row `pos` of [B, nkv, cap, hd]; a position outside the cache is
+// flagged and skipped.
+template <int HD>
+__device__ __forceinline__ void rope_store_pair(const QkvParams& p, int hb, int i0, int r, int tok, float lo,
+                                                float hi, double inv_freq) {
+  const bool is_q = hb < p.nh, is_k = !is_q && hb < p.nh + p.nkv;
+  const int b = tok / p.S, s = tok - b * p.S;
+  const int pos = p.pos[tok];
+  if (is_q || is_k) {
+    float c, sn;
+    rope_cos_sin(pos, inv_freq, &c, &sn);
+    const float nl = lo * c - hi * sn, nh_ = hi * c + lo * sn;
+    lo = nl;
+    hi = nh_;
+  }
+  __nv_bfloat16* dst;
+  if (is_q) {
+    dst = static_cast<__nv_bfloat16*>(p.q_out) + (((size_t)b * p.nh + hb) * p.S + s) * HD;
+  } else {
+    if (pos < 0 || pos >= p.cap) {
+      raise_error(p.err, GQA_DEVERR_POSITION_RANGE);
+      return;
+    }
+    const int jh = is_k ? hb - p.nh : hb - p.nh - p.nkv;
+    dst = static_cast<__nv_bfloat16*>(is_k ? p.k_cache : p.v_cache) + (((size_t)b * p.nkv + jh) * p.cap + pos) * HD;
+  }
+  dst[i0 + r] = __float2bfloat16_rn(lo);
+  dst[HD / 2 + i0 + r] = __float2bfloat16_rn(hi);
 }
 
 template <int NT, int HD>
@@ -110,7 +147,6 @@ __global__ void __launch_bounds__(WARPS * 32, 2) qkv_smallm_kernel(QkvParams p) 
   }
   __syncthreads();
 
-  const bool is_q = hb < p.nh, is_k = !is_q && hb < p.nh + p.nkv;
   for (int e = threadIdx.x; e < 8 * T; e += WARPS * 32) {
     if (e >= 8 * TP) break;
     const int r = e & 7, tok = e >> 3;
@@ -120,28 +156,226 @@ __global__ void __launch_bounds__(WARPS * 32, 2) qkv_smallm_kernel(QkvParams p) 
       lo += red[w][r][tok];
       hi += red[w][r + 8][tok];
     }
-    const int b = tok / p.S, s = tok - b * p.S;
-    const int pos = p.pos[tok];
-    if (is_q || is_k) {
-      float c, sn;
-      rope_cos_sin(pos, inv_freq[r], &c, &sn);
-      const float nl = lo * c - hi * sn, nh_ = hi * c + lo * sn;
-      lo = nl;
-      hi = nh_;
+    rope_store_pair<HD>(p, hb, i0, r, tok, lo, hi, inv_freq[r]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Streaming variant, used when hidden % 64 == 0 and the tokens' hidden states
+// fit in shared memory next to the W ring (the usual one-token step).  The
+// register kernel above loads, waits and multiplies in rounds, and its 16-row
+// CTAs come in more than one wave; here persistent CTAs (one per SM) walk the
+// same 16-row work units u = blockIdx.x, +gridDim.x, ...  and a TMA producer
+// warp keeps a ring of W slabs in flight across unit boundaries, so the W
+// stream does not drain between units or waves.
+//
+//   X   [T, hidden] -> shared memory once per CTA by the consumer threads, in
+//       the layout of 64-column, 128-byte-swizzled boxes of TP rows (rows past
+//       T zero), while the producer starts the W ring
+//   W   per stage: the 8 lo rows and the 8 hi rows of the unit over 512
+//       columns (two 3-D boxes of 8 column blocks x 8 rows x 64 columns)
+//   consumer warp w takes column block w of every stage: ldmatrix fragments
+//       of W (rows as M) and X (tokens as N), mma.sync m16n8k16
+//   after a unit's last stage the 8 warps' sums meet in shared memory and the
+//   RoPE + scatter epilogue of the register kernel runs.
+constexpr int SW_WARPS = 8;                       // consumer warps (+1 producer)
+constexpr int SW_STAGES = 6;
+constexpr int SW_KB = 8;                          // 64-column blocks per stage
+constexpr int SW_HALF = SW_KB * 8 * 128;          // 8 rows x 512 columns
+constexpr int SW_STAGE = 2 * SW_HALF;             // lo + hi rows
+constexpr int SW_SMEM_MAX = 227 * 1024;
+static_assert(SW_KB == SW_WARPS, "one column block per consumer warp and stage");
+
+inline size_t stream_smem(int NT, int nblk) {
+  const size_t TP = (size_t)NT * 8;
+  return 1024 /*align*/ + (size_t)SW_STAGES * SW_STAGE + (size_t)nblk * TP * 128 +
+         (size_t)SW_WARPS * 16 * (TP + 1) * 4 + 2 * SW_STAGES * 8;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+template <int NT, int HD>
+__global__ void __launch_bounds__((SW_WARPS + 1) * 32, 1)
+qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
+                  int n_units) {
+  constexpr int TP = NT * 8;
+  constexpr int GROUPS = HD / 16;
+  constexpr int XBOX = TP * 128;                   // one 64-column block of X
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nblk = p.hidden / 64;
+  const int nst = (nblk + SW_KB - 1) / SW_KB;
+  uint8_t* ring = smem;
+  uint8_t* xs = smem + SW_STAGES * SW_STAGE;
+  float* red = reinterpret_cast<float*>(xs + (size_t)nblk * XBOX);      // [warp][16 rows][TP + 1]
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + SW_WARPS * 16 * (TP + 1));
+  uint64_t* empty = full + SW_STAGES;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int T = p.B * p.S;
+  int* err = p.err;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SW_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], SW_WARPS);
     }
-    __nv_bfloat16* dst;
-    if (is_q) {
-      dst = static_cast<__nv_bfloat16*>(p.q_out) + (((size_t)b * p.nh + hb) * p.S + s) * HD;
-    } else {
-      if (pos < 0 || pos >= p.cap) {
-        raise_error(p.err, GQA_DEVERR_POSITION_RANGE);
-        continue;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == SW_WARPS) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmw);
+      int it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int rlo = (u / GROUPS) * HD + (u % GROUPS) * 8;
+        for (int st = 0; st < nst; ++st) {
+          const int s = it % SW_STAGES;
+          if (!mbar_wait(&empty[s], ((it / SW_STAGES) & 1) ^ 1, err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], SW_STAGE);
+          tc::tma_load_3d(ring + s * SW_STAGE, &tmw, 0, rlo, st * SW_KB, &full[s]);
+          tc::tma_load_3d(ring + s * SW_STAGE + SW_HALF, &tmw, 0, rlo + HD / 2, st * SW_KB, &full[s]);
+          ++it;
+        }
       }
-      const int jh = is_k ? hb - p.nh : hb - p.nh - p.nkv;
-      dst = static_cast<__nv_bfloat16*>(is_k ? p.k_cache : p.v_cache) + (((size_t)b * p.nkv + jh) * p.cap + pos) * HD;
+      // every issued copy has landed before the block may exit
+      for (int t = max(0, it - SW_STAGES); t < it; ++t) mbar_wait(&full[t % SW_STAGES], (t / SW_STAGES) & 1, err);
     }
-    dst[i0 + r] = __float2bfloat16_rn(lo);
-    dst[HD / 2 + i0 + r] = __float2bfloat16_rn(hi);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int g = lane >> 2, tq = lane & 3;
+  const int mrow = lane & 7, mat = lane >> 3;     // ldmatrix: row in matrix, matrix index
+  const uint32_t ring_u = smem_u32(ring), xs_u = smem_u32(xs);
+  {
+    // X -> shared memory (the swizzled layout of a 64-column TMA box of TP
+    // rows; rows past T zero) by the consumer threads, 8 vectors in flight
+    // each, while the producer fills the W ring.  (Fetched by TMA next to
+    // the W slabs, the same X measured markedly slower on B200.)
+    const __nv_bfloat16* X = static_cast<const __nv_bfloat16*>(p.x);
+    const int nchunk = nblk * TP * 8;
+    for (int e0 = threadIdx.x; e0 < nchunk; e0 += SW_WARPS * 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i * SW_WARPS * 32;
+        const int kb = e / (TP * 8), rem = e % (TP * 8), row = rem / 8, ch = rem % 8;
+        v[i] = make_uint4(0, 0, 0, 0);
+        if (e < nchunk && row < T)
+          v[i] = *reinterpret_cast<const uint4*>(X + (size_t)row * p.hidden + kb * 64 + ch * 8);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i * SW_WARPS * 32;
+        const int kb = e / (TP * 8), rem = e % (TP * 8), row = rem / 8, ch = rem % 8;
+        if (e < nchunk) *reinterpret_cast<uint4*>(xs + kb * XBOX + row * 128 + ((ch ^ (row & 7)) << 4)) = v[i];
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(SW_WARPS * 32) : "memory");
+  }
+  bool dead = false;
+  int it = 0;
+  for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    for (int st = 0; st < nst; ++st, ++it) {
+      const int s = it % SW_STAGES;
+      if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&full[s], (it / SW_STAGES) & 1, err));
+      const int kb = st * SW_KB + warp;
+      if (!dead && kb < nblk) {
+        const uint32_t wb = ring_u + s * SW_STAGE + warp * 1024;
+        const uint32_t xb = xs_u + kb * XBOX;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          // W matrices: (lo rows, k 0-7), (hi rows, k 0-7), (lo, k 8-15), (hi, k 8-15)
+          uint32_t a0, a1, a2, a3;
+          const int wch = 2 * ks + (mat >> 1);
+          ldsm_x4(wb + (mat & 1) * SW_HALF + mrow * 128 + ((wch ^ mrow) << 4), a0, a1, a2, a3);
+#pragma unroll
+          for (int np = 0; np < NT; np += 2) {
+            // X matrices: (tokens np*8.., k 0-7), (same, k 8-15), (tokens (np+1)*8.., k 0-7), (same, k 8-15);
+            // with a single token tile the last two repeat the first two
+            const int tok = (np + ((mat >> 1) & (NT > 1 ? 1 : 0))) * 8 + mrow;
+            const int xch = 2 * ks + (mat & 1);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(xb + tok * 128 + ((xch ^ mrow) << 4), b0, b1, b2, b3);
+            mma16816(acc[np], a0, a1, a2, a3, b0, b1);
+            if (NT > 1) mma16816(acc[np + 1 < NT ? np + 1 : np], a0, a1, a2, a3, b2, b3);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0 && !dead) mbar_arrive(&empty[s]);
+    }
+
+    // the 8 warps' partial sums: c0,c1 = (lo row g, tokens 8n+2tq, +1); c2,c3 = (hi row g, same)
+    float* rw = red + warp * 16 * (TP + 1);
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      rw[g * (TP + 1) + n * 8 + 2 * tq] = acc[n][0];
+      rw[g * (TP + 1) + n * 8 + 2 * tq + 1] = acc[n][1];
+      rw[(g + 8) * (TP + 1) + n * 8 + 2 * tq] = acc[n][2];
+      rw[(g + 8) * (TP + 1) + n * 8 + 2 * tq + 1] = acc[n][3];
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(SW_WARPS * 32) : "memory");
+    const int hb = u / GROUPS, i0 = (u % GROUPS) * 8;
+    for (int e = threadIdx.x; e < 8 * T; e += SW_WARPS * 32) {
+      const int r = e & 7, tok = e >> 3;
+      float lo = 0.f, hi = 0.f;
+#pragma unroll
+      for (int w = 0; w < SW_WARPS; ++w) {
+        lo += red[(w * 16 + r) * (TP + 1) + tok];
+        hi += red[(w * 16 + r + 8) * (TP + 1) + tok];
+      }
+      if (!dead) rope_store_pair<HD>(p, hb, i0, r, tok, lo, hi, rope_inv_freq(i0 + r, HD, p.theta));
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(SW_WARPS * 32) : "memory");
+  }
+}
+
+template <int NT, int HD>
+cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
+  const int nblk = p.hidden / 64;
+  const size_t smem = stream_smem(NT, nblk);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(qkv_stream_kernel<NT, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SW_SMEM_MAX);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int N = (p.nh + 2 * p.nkv) * HD;
+  CUtensorMap tw;
+  // W viewed as [column block][row][64 columns]: a box is 8 blocks x 8 rows
+  const uint64_t wd[3] = {64, (uint64_t)N, (uint64_t)nblk};
+  const uint64_t ws[2] = {(uint64_t)p.hidden * 2, 128};
+  const uint32_t wbox[3] = {64, 8, SW_KB};
+  if (!make_tmap_bf16_3d(&tw, p.w, wd, ws, wbox)) return cudaErrorInvalidValue;
+  const int n_units = N / 16;
+  const int grid = n_units < num_sms ? n_units : num_sms;
+  qkv_stream_kernel<NT, HD><<<grid, (SW_WARPS + 1) * 32, smem, st>>>(tw, p, n_units);
+  return cudaGetLastError();
+}
+
+template <int NT>
+cudaError_t launch_stream(const QkvParams& p, int num_sms, cudaStream_t st) {
+  switch (p.hd) {
+    case 32: return launch_stream_hd<NT, 32>(p, num_sms, st);
+    case 64: return launch_stream_hd<NT, 64>(p, num_sms, st);
+    case 128: return launch_stream_hd<NT, 128>(p, num_sms, st);
+    default: return cudaErrorInvalidValue;
   }
 }
 
@@ -160,13 +394,24 @@ cudaError_t launch_nt(const QkvParams& p, cudaStream_t st) {
 
 }  // namespace
 
-cudaError_t launch_qkv_smallm(const QkvParams& p, cudaStream_t st) {
+cudaError_t launch_qkv_smallm(const QkvParams& p, int num_sms, cudaStream_t st) {
   const int T = p.B * p.S;
-  if (T <= 8) return launch_nt<1>(p, st);
-  if (T <= 16) return launch_nt<2>(p, st);
-  if (T <= 32) return launch_nt<4>(p, st);
-  if (T <= 64) return launch_nt<8>(p, st);
-  return cudaErrorInvalidValue;
+  const int nt = T <= 8 ? 1 : T <= 16 ? 2 : T <= 32 ? 4 : T <= 64 ? 8 : 0;
+  if (nt == 0) return cudaErrorInvalidValue;
+  if (p.hidden % 64 == 0 && stream_smem(nt, p.hidden / 64) <= (size_t)SW_SMEM_MAX) {
+    switch (nt) {
+      case 1: return launch_stream<1>(p, num_sms, st);
+      case 2: return launch_stream<2>(p, num_sms, st);
+      case 4: return launch_stream<4>(p, num_sms, st);
+      default: return launch_stream<8>(p, num_sms, st);
+    }
+  }
+  switch (nt) {
+    case 1: return launch_nt<1>(p, st);
+    case 2: return launch_nt<2>(p, st);
+    case 4: return launch_nt<4>(p, st);
+    default: return launch_nt<8>(p, st);
+  }
 }
 
 }  // namespace gqa

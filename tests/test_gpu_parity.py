@@ -52,11 +52,20 @@ QKV_CASES = [
     ("bf16", 3, 150, 136, 3, 1, 64, 160, True),     # N = 320 (partial 256-tile), K tail, T = 450
     ("bf16", 2, 300, 256, 12, 2, 32, 320, False),   # hd 32: 8 heads per tile
     ("bf16", 2, 70, 100, 4, 2, 64, 80, True),       # hidden % 8 != 0: the SIMT path
-    # few tokens (the W-streaming kernel), every token-count variant
+    # few tokens, hidden % 64 == 0 and the hidden states fit in shared memory:
+    # the TMA-ring kernel, every token-count variant
     ("bf16", 3, 1, 2048, 32, 4, 64, 16, True),
+    ("bf16", 8, 1, 6144, 48, 1, 128, 40, True),     # 400 units: several per CTA, 12 stages each
+    ("bf16", 5, 1, 4096, 16, 4, 64, 8, True),
+    ("bf16", 8, 1, 7168, 8, 1, 128, 8, True),       # 112 column blocks, 14 stages
+    ("bf16", 4, 4, 1088, 8, 2, 64, 32, True),       # T = 16: 17 column blocks
+    ("bf16", 3, 4, 3584, 4, 2, 128, 16, True),      # T = 12
+    ("bf16", 3, 9, 768, 6, 3, 128, 64, False),
+    ("bf16", 8, 5, 256, 12, 2, 32, 9, True),
+    # few tokens, hidden % 64 != 0: the register-streaming kernel, every token-count variant
+    ("bf16", 5, 1, 520, 8, 2, 64, 8, True),
     ("bf16", 4, 3, 520, 8, 2, 128, 8, True),
     ("bf16", 2, 10, 1000, 6, 1, 128, 16, True),
-    ("bf16", 8, 5, 256, 12, 2, 32, 9, True),
     ("bf16", 1, 64, 136, 4, 4, 64, 64, False),
 ]
 
@@ -235,16 +244,48 @@ def test_decode_workspace_reuse_leaves_counters_zero():
 
 
 def test_decode_split_count_invariance():
-    """n_split in {1, 2, 7, max} agree to float32 rounding of the merge."""
+    """Workspace splits of 448, 256 and 64 keys (1, 2 and 7 splits) and the
+    automatic cluster-merged split (7 CTAs of one tile each) agree to the
+    float32 rounding of the merge."""
     dtype, hd, nh, nkv = "bf16", 128, 8, 1
     lens = np.array([448, 448], dtype=np.int32)
     B, cap = 2, 448
     q = W.normal_tensor((B, nh, hd), 8, 0, dtype)
     kc = nan_padded(B, nkv, cap, hd, lens, 8, 1, dtype)
     vc = nan_padded(B, nkv, cap, hd, lens, 8, 2, dtype)
-    outs = [host(run_decode(q, kc, vc, lens, nh, dtype, kv_split=s)) for s in (448, 256, 64)]
+    outs = [host(run_decode(q, kc, vc, lens, nh, dtype, kv_split=s)) for s in (448, 256, 64, 0)]
     for o in outs[1:]:
         assert np.max(np.abs(o - outs[0])) <= 2 ** -7 * np.max(np.abs(outs[0]))
+
+
+@pytest.mark.parametrize("hd", (64, 128))
+def test_decode_cluster_merge_ragged(hd):
+    """Automatic split of a small ragged batch: each sequence's tiles are dealt
+    out over a cluster of up to 8 CTAs, some of which get none (lengths 0, 1,
+    64, 65), and the partials meet in distributed shared memory."""
+    dtype, nh, nkv, cap = "bf16", 48, 1, 1040
+    lens = np.array([0, 1, 64, 65, 528, 1040, 17, 900], dtype=np.int32)
+    B = len(lens)
+    q = W.normal_tensor((B, nh, hd), 12, 0, dtype)
+    kc = nan_padded(B, nkv, cap, hd, lens, 12, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, lens, 12, 2, dtype)
+    got = host(run_decode(q, kc, vc, lens, nh, dtype))
+    assert np.all(got[0] == 0)
+    want = ref.decode_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens)
+    gate(got[1:], want[1:], dtype, "cluster-merged decode")
+
+
+def test_decode_long_cache_uses_workspace_splits():
+    """A cache longer than 8 x 2048 keys takes the workspace splits even when
+    the split is left to the library."""
+    dtype, hd, nh, nkv, cap = "bf16", 128, 8, 1, 20000
+    lens = np.array([20000, 12345], dtype=np.int32)
+    B = len(lens)
+    q = W.normal_tensor((B, nh, hd), 13, 0, dtype)
+    kc = nan_padded(B, nkv, cap, hd, lens, 13, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, lens, 13, 2, dtype)
+    want = ref.decode_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens)
+    gate(host(run_decode(q, kc, vc, lens, nh, dtype)), want, dtype, "long-cache decode")
 
 
 def test_decode_zero_and_clamped_lengths():
