@@ -164,10 +164,12 @@ __global__ void __launch_bounds__(WARPS * 32, 2) qkv_smallm_kernel(QkvParams p) 
 // Streaming variant, used when hidden % 64 == 0 and the tokens' hidden states
 // fit in shared memory next to the W ring (the usual one-token step).  The
 // register kernel above loads, waits and multiplies in rounds, and its 16-row
-// CTAs come in more than one wave; here persistent CTAs (one per SM) walk the
-// same 16-row work units u = blockIdx.x, +gridDim.x, ...  and a TMA producer
-// warp keeps a ring of W slabs in flight across unit boundaries, so the W
-// stream does not drain between units or waves.
+// CTAs come in more than one wave; here persistent CTAs (one per SM, or two
+// with a shorter ring when the hidden states are small and there are more
+// units than SMs) walk the same 16-row work units u = blockIdx.x,
+// +gridDim.x, ...  and a TMA producer warp keeps a ring of W slabs in flight
+// across unit boundaries, so the W stream does not drain between units or
+// waves.
 //
 //   X   [T, hidden] -> shared memory once per CTA by the consumer threads, in
 //       the layout of 64-column, 128-byte-swizzled boxes of TP rows (rows past
@@ -177,19 +179,23 @@ __global__ void __launch_bounds__(WARPS * 32, 2) qkv_smallm_kernel(QkvParams p) 
 //   consumer warp w takes column block w of every stage: ldmatrix fragments
 //       of W (rows as M) and X (tokens as N), mma.sync m16n8k16
 //   after a unit's last stage the 8 warps' sums meet in shared memory and the
-//   RoPE + scatter epilogue of the register kernel runs.
+//   RoPE + scatter epilogue of the register kernel runs (frequencies from a
+//   per-CTA table).  Measured on B200, handing the epilogue to a warp of its
+//   own was slower: one warp's serial double-precision angle reductions then
+//   form the kernel's tail.
 constexpr int SW_WARPS = 8;                       // consumer warps (+1 producer)
-constexpr int SW_STAGES = 6;
+constexpr int SW_STAGES = 6;                      // ring depth with one CTA per SM (at most)
 constexpr int SW_KB = 8;                          // 64-column blocks per stage
 constexpr int SW_HALF = SW_KB * 8 * 128;          // 8 rows x 512 columns
 constexpr int SW_STAGE = 2 * SW_HALF;             // lo + hi rows
 constexpr int SW_SMEM_MAX = 227 * 1024;
+constexpr int HD_MAX = 128;
 static_assert(SW_KB == SW_WARPS, "one column block per consumer warp and stage");
 
-inline size_t stream_smem(int NT, int nblk) {
+inline size_t stream_smem(int NT, int nblk, int stages = SW_STAGES) {
   const size_t TP = (size_t)NT * 8;
-  return 1024 /*align*/ + (size_t)SW_STAGES * SW_STAGE + (size_t)nblk * TP * 128 +
-         (size_t)SW_WARPS * 16 * (TP + 1) * 4 + 2 * SW_STAGES * 8;
+  return 1024 /*align*/ + (size_t)stages * SW_STAGE + (size_t)nblk * TP * 128 +
+         (size_t)SW_WARPS * 16 * (TP + 1) * 4 + 2 * SW_STAGES * 8 + (size_t)(HD_MAX / 2) * 8;
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -200,7 +206,7 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
 template <int NT, int HD>
 __global__ void __launch_bounds__((SW_WARPS + 1) * 32, 1)
 qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
-                  int n_units) {
+                  int n_units, int nstages) {
   constexpr int TP = NT * 8;
   constexpr int GROUPS = HD / 16;
   constexpr int XBOX = TP * 128;                   // one 64-column block of X
@@ -209,16 +215,17 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
   const int nblk = p.hidden / 64;
   const int nst = (nblk + SW_KB - 1) / SW_KB;
   uint8_t* ring = smem;
-  uint8_t* xs = smem + SW_STAGES * SW_STAGE;
+  uint8_t* xs = smem + nstages * SW_STAGE;
   float* red = reinterpret_cast<float*>(xs + (size_t)nblk * XBOX);      // [warp][16 rows][TP + 1]
   uint64_t* full = reinterpret_cast<uint64_t*>(red + SW_WARPS * 16 * (TP + 1));
   uint64_t* empty = full + SW_STAGES;
+  double* inv_freq = reinterpret_cast<double*>(empty + SW_STAGES);   // [HD / 2]
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int T = p.B * p.S;
   int* err = p.err;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SW_STAGES; ++s) {
+    for (int s = 0; s < nstages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], SW_WARPS);
     }
@@ -230,13 +237,16 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tc::prefetch_tmap(&tmw);
-      int it = 0;
+      // ring slot s and its phase parity, advanced without a division (the
+      // ring depth is a launch parameter; a runtime divide per stage
+      // measured as a several-microsecond loss)
+      int it = 0, s = 0;
+      uint32_t ph = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         const int rlo = (u / GROUPS) * HD + (u % GROUPS) * 8;
         for (int st = 0; st < nst; ++st) {
-          const int s = it % SW_STAGES;
-          if (!mbar_wait(&empty[s], ((it / SW_STAGES) & 1) ^ 1, err)) {
+          if (!mbar_wait(&empty[s], ph ^ 1, err)) {
             ok = false;
             break;
           }
@@ -244,10 +254,21 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
           tc::tma_load_3d(ring + s * SW_STAGE, &tmw, 0, rlo, st * SW_KB, &full[s]);
           tc::tma_load_3d(ring + s * SW_STAGE + SW_HALF, &tmw, 0, rlo + HD / 2, st * SW_KB, &full[s]);
           ++it;
+          if (++s == nstages) {
+            s = 0;
+            ph ^= 1;
+          }
         }
       }
-      // every issued copy has landed before the block may exit
-      for (int t = max(0, it - SW_STAGES); t < it; ++t) mbar_wait(&full[t % SW_STAGES], (t / SW_STAGES) & 1, err);
+      // every issued copy has landed before the block may exit: walk back
+      // over the last min(it, nstages) copies
+      for (int k = 0; k < min(it, nstages); ++k) {
+        if (--s < 0) {
+          s = nstages - 1;
+          ph ^= 1;
+        }
+        mbar_wait(&full[s], ph, err);
+      }
     }
     return;
   }
@@ -280,42 +301,64 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
         if (e < nchunk) *reinterpret_cast<uint4*>(xs + kb * XBOX + row * 128 + ((ch ^ (row & 7)) << 4)) = v[i];
       }
     }
+    // the RoPE frequencies of the head dimension, once per CTA
+    for (int f = threadIdx.x; f < HD / 2; f += SW_WARPS * 32) inv_freq[f] = rope_inv_freq(f, HD, p.theta);
     asm volatile("bar.sync 1, %0;" ::"n"(SW_WARPS * 32) : "memory");
   }
   bool dead = false;
-  int it = 0;
+  int s = 0;            // ring slot and phase parity, advanced as in the producer
+  uint32_t ph = 0;
   for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
     float acc[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    for (int st = 0; st < nst; ++st, ++it) {
-      const int s = it % SW_STAGES;
-      if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&full[s], (it / SW_STAGES) & 1, err));
+    for (int st = 0; st < nst; ++st) {
+      if (!dead) dead = !__all_sync(0xffffffffu, mbar_wait(&full[s], ph, err));
       const int kb = st * SW_KB + warp;
       if (!dead && kb < nblk) {
         const uint32_t wb = ring_u + s * SW_STAGE + warp * 1024;
         const uint32_t xb = xs_u + kb * XBOX;
+        if (NT == 1) {
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          // W matrices: (lo rows, k 0-7), (hi rows, k 0-7), (lo, k 8-15), (hi, k 8-15)
-          uint32_t a0, a1, a2, a3;
-          const int wch = 2 * ks + (mat >> 1);
-          ldsm_x4(wb + (mat & 1) * SW_HALF + mrow * 128 + ((wch ^ mrow) << 4), a0, a1, a2, a3);
-#pragma unroll
-          for (int np = 0; np < NT; np += 2) {
-            // X matrices: (tokens np*8.., k 0-7), (same, k 8-15), (tokens (np+1)*8.., k 0-7), (same, k 8-15);
-            // with a single token tile the last two repeat the first two
-            const int tok = (np + ((mat >> 1) & (NT > 1 ? 1 : 0))) * 8 + mrow;
-            const int xch = 2 * ks + (mat & 1);
+          for (int ks = 0; ks < 4; ks += 2) {
+            // X matrices: (tokens 0-7, 16-byte chunks 2ks .. 2ks+3): k16 steps ks and ks + 1
             uint32_t b0, b1, b2, b3;
-            ldsm_x4(xb + tok * 128 + ((xch ^ mrow) << 4), b0, b1, b2, b3);
-            mma16816(acc[np], a0, a1, a2, a3, b0, b1);
-            if (NT > 1) mma16816(acc[np + 1 < NT ? np + 1 : np], a0, a1, a2, a3, b2, b3);
+            ldsm_x4(xb + mrow * 128 + (((2 * ks + mat) ^ mrow) << 4), b0, b1, b2, b3);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              // W matrices: (lo rows, k 0-7), (hi rows, k 0-7), (lo, k 8-15), (hi, k 8-15)
+              uint32_t a0, a1, a2, a3;
+              const int wch = 2 * (ks + h) + (mat >> 1);
+              ldsm_x4(wb + (mat & 1) * SW_HALF + mrow * 128 + ((wch ^ mrow) << 4), a0, a1, a2, a3);
+              mma16816(acc[0], a0, a1, a2, a3, h ? b2 : b0, h ? b3 : b1);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            // W matrices: (lo rows, k 0-7), (hi rows, k 0-7), (lo, k 8-15), (hi, k 8-15)
+            uint32_t a0, a1, a2, a3;
+            const int wch = 2 * ks + (mat >> 1);
+            ldsm_x4(wb + (mat & 1) * SW_HALF + mrow * 128 + ((wch ^ mrow) << 4), a0, a1, a2, a3);
+#pragma unroll
+            for (int np = 0; np < NT; np += 2) {
+              // X matrices: (tokens np*8.., k 0-7), (same, k 8-15), (tokens (np+1)*8.., k 0-7), (same, k 8-15)
+              const int tok = (np + (mat >> 1)) * 8 + mrow;
+              const int xch = 2 * ks + (mat & 1);
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4(xb + tok * 128 + ((xch ^ mrow) << 4), b0, b1, b2, b3);
+              mma16816(acc[np], a0, a1, a2, a3, b0, b1);
+              mma16816(acc[np + 1 < NT ? np + 1 : np], a0, a1, a2, a3, b2, b3);
+            }
           }
         }
       }
       __syncwarp();
       if (lane == 0 && !dead) mbar_arrive(&empty[s]);
+      if (++s == nstages) {
+        s = 0;
+        ph ^= 1;
+      }
     }
 
     // the 8 warps' partial sums: c0,c1 = (lo row g, tokens 8n+2tq, +1); c2,c3 = (hi row g, same)
@@ -337,7 +380,7 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
         lo += red[(w * 16 + r) * (TP + 1) + tok];
         hi += red[(w * 16 + r + 8) * (TP + 1) + tok];
       }
-      if (!dead) rope_store_pair<HD>(p, hb, i0, r, tok, lo, hi, rope_inv_freq(i0 + r, HD, p.theta));
+      if (!dead) rope_store_pair<HD>(p, hb, i0, r, tok, lo, hi, inv_freq[i0 + r]);
     }
     asm volatile("bar.sync 1, %0;" ::"n"(SW_WARPS * 32) : "memory");
   }
@@ -346,7 +389,6 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
 template <int NT, int HD>
 cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
   const int nblk = p.hidden / 64;
-  const size_t smem = stream_smem(NT, nblk);
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -357,15 +399,35 @@ cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
     attr_set[dev] = true;
   }
   const int N = (p.nh + 2 * p.nkv) * HD;
+  const int n_units = N / 16;
+  // More units than SMs and small hidden states: two CTAs per SM with a
+  // shorter ring each, so that a few hundred units run in one wave instead
+  // of a few SMs taking a second unit after everyone else is done.
+  int stages = SW_STAGES, per_sm = 1;
+  if (n_units > num_sms) {
+    for (int s2 = SW_STAGES; s2 >= 3; --s2) {
+      int fit = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, qkv_stream_kernel<NT, HD>, (SW_WARPS + 1) * 32,
+                                                        stream_smem(NT, nblk, s2)) != cudaSuccess) {
+        cudaGetLastError();
+        break;
+      }
+      if (fit >= 2) {
+        stages = s2;
+        per_sm = 2;
+        break;
+      }
+    }
+  }
+  const size_t smem = stream_smem(NT, nblk, stages);
   CUtensorMap tw;
   // W viewed as [column block][row][64 columns]: a box is 8 blocks x 8 rows
   const uint64_t wd[3] = {64, (uint64_t)N, (uint64_t)nblk};
   const uint64_t ws[2] = {(uint64_t)p.hidden * 2, 128};
   const uint32_t wbox[3] = {64, 8, SW_KB};
   if (!make_tmap_bf16_3d(&tw, p.w, wd, ws, wbox)) return cudaErrorInvalidValue;
-  const int n_units = N / 16;
-  const int grid = n_units < num_sms ? n_units : num_sms;
-  qkv_stream_kernel<NT, HD><<<grid, (SW_WARPS + 1) * 32, smem, st>>>(tw, p, n_units);
+  const int grid = n_units < per_sm * num_sms ? n_units : per_sm * num_sms;
+  qkv_stream_kernel<NT, HD><<<grid, (SW_WARPS + 1) * 32, smem, st>>>(tw, p, n_units, stages);
   return cudaGetLastError();
 }
 
