@@ -555,6 +555,18 @@ cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
 }
 
 int launch_decode(const DecodeParams& p0, bool bf16, cudaStream_t st, cudaError_t* err) {
+  if (bf16 && p0.auto_split) {
+    // large batches with large head groups: tcgen05 tiles (mma.sync would be
+    // tensor-bound there)
+    const int nc = decode_tc_splits(p0);
+    if (nc > 0) {
+      DecodeParams p = p0;
+      p.cluster = 1;
+      p.n_split = nc;
+      *err = launch_decode_tc(p, st);
+      return 1;
+    }
+  }
   if (bf16 && (p0.hd == 64 || p0.hd == 128)) {  // merges its splits itself
     DecodeParams p = p0;
     const int nc = p.auto_split ? cluster_splits(p) : 0;

@@ -79,6 +79,12 @@ cudaError_t launch_qkv_smallm(const QkvParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
 cudaError_t launch_prefill_fa(const PrefillParams& p, cudaStream_t st);    // head_dim 64/128, 2 Q tiles/CTA
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128
+// tcgen05 decode for large batches with g > 16 (heads as the 128 MMA rows),
+// splits merged inside a thread-block cluster (p.n_split <= 8 CTAs);
+// decode_tc_splits gives that split count for a problem, or 0 when the
+// problem is for the mma.sync kernel.
+cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
+int decode_tc_splits(const DecodeParams& p);
 
 // Decode: the tensor-core kernel for bf16 head_dim 64/128 (the last split of
 // each (sequence, KV head, head group) merges the partials itself, using the

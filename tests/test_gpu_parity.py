@@ -275,6 +275,27 @@ def test_decode_cluster_merge_ragged(hd):
     gate(got[1:], want[1:], dtype, "cluster-merged decode")
 
 
+@pytest.mark.parametrize("hd,nh,nkv,B", [(64, 48, 1, 32), (128, 160, 1, 32), (128, 64, 2, 16)],
+                         ids=["hd64-g48", "hd128-g160-two-head-groups", "hd128-g32-nkv2"])
+def test_decode_tcgen05_large_batch(hd, nh, nkv, B):
+    """Large batches with g > 16 (at least 2^18 cached key rows) take the
+    tcgen05 decode: heads as the 128 MMA rows, each sequence's 64-key tiles
+    dealt out over a cluster whose CTAs merge through distributed shared
+    memory.  Ragged lengths with 0, 1 and tile edges; g = 160 has a second,
+    partial head group."""
+    dtype, cap = "bf16", 8192
+    edge = [0, 1, 63, 64, 65, 1023, 1024, 1025, 2100, 4096, 8191, 8192]
+    rng = np.random.default_rng(21)
+    lens = np.array(edge + list(rng.integers(1, cap + 1, size=B - len(edge))), dtype=np.int32)[:B]
+    q = W.normal_tensor((B, nh, hd), 14, 0, dtype)
+    kc = nan_padded(B, nkv, cap, hd, lens, 14, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, lens, 14, 2, dtype)
+    got = host(run_decode(q, kc, vc, lens, nh, dtype))
+    assert np.all(got[0] == 0)
+    want = ref.decode_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens)
+    gate(got[1:], want[1:], dtype, "tcgen05 decode")
+
+
 def test_decode_long_cache_uses_workspace_splits():
     """A cache longer than 8 x 2048 keys takes the workspace splits even when
     the split is left to the library."""
