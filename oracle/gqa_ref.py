@@ -21,6 +21,9 @@ Sources (page title, then section):
 * custom-op overhead gist (``overhead.py``): ``forward(positions,
   hidden_states)`` applies a position-dependent step to q and k only, after
   the fused projection.
+* "MHA -> GQA: 提升 LLM 推理效率", section 4.3 (剪枝训练): the new KV projection
+  of each group of heads is initialised by mean pooling the group's
+  projections (the offline MHA -> GQA weight transform).
 
 Readings where the pages are silent (each restated in the design notes):
 
@@ -240,3 +243,29 @@ def decode_attention(q, k_cache, v_cache, kv_lens, pairs=None):
     if pairs is None:
         return out.reshape(B, nh, hd)
     return out
+
+
+def meanpool_kv_projection(w_qkv_mha: np.ndarray, n_heads: int, n_kv_heads: int,
+                           head_dim: int) -> np.ndarray:
+    """MHA -> GQA weight transform ("MHA -> GQA" blog, section 4.3): the
+    initial projection of each new KV head is the mean of the projections of
+    the g = n_heads / n_kv_heads heads of its group; the query projection is
+    kept.  The groups are consecutive heads, h -> h // g, the same head map
+    as attention uses.
+
+    ``w_qkv_mha`` is the fused MHA weight ``[3 * n_heads * hd, D]`` (query,
+    key, value blocks of ``n_heads * hd`` rows each); the result is the fused
+    GQA weight ``[(n_heads + 2 * n_kv_heads) * hd, D]``.
+    """
+    nh, nkv, hd = n_heads, n_kv_heads, head_dim
+    assert nh % nkv == 0 and w_qkv_mha.shape[0] == 3 * nh * hd
+    g = nh // nkv
+    w = np.asarray(w_qkv_mha, dtype=np.float64)
+    D = w.shape[1]
+    q = w[: nh * hd]
+    out = [q]
+    for block in (1, 2):                                   # key, then value projection
+        heads = w[block * nh * hd:(block + 1) * nh * hd].reshape(nh, hd, D)
+        out.append(heads.reshape(nkv, g, hd, D).mean(axis=1).reshape(nkv * hd, D))
+    return np.concatenate(out, axis=0)
+

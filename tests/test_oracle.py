@@ -547,3 +547,96 @@ def test_round_bf16_exact_and_ties_to_even():
     assert ref.round_bf16(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
     a = rng(31).standard_normal(10000) * 37
     assert np.max(np.abs(ref.round_bf16(a) - a) / np.abs(a)) <= 2 ** -8
+
+
+# --------------------------------------------------------------------------
+# MHA -> GQA weight transform (MHA -> GQA blog, section 4.3: mean pooling of
+# each group's projections)
+# --------------------------------------------------------------------------
+def brute_meanpool(w, nh, nkv, hd):
+    g = nh // nkv
+    D = w.shape[1]
+    out = np.zeros(((nh + 2 * nkv) * hd, D))
+    for r in range(nh * hd):
+        out[r] = w[r]
+    for block in (1, 2):
+        for j in range(nkv):
+            for d in range(hd):
+                for c in range(D):
+                    acc = 0.0
+                    for i in range(g):
+                        acc += float(w[block * nh * hd + (j * g + i) * hd + d, c])
+                    out[nh * hd + (block - 1) * nkv * hd + j * hd + d, c] = acc / g
+    return out
+
+
+def check_meanpool_of_equal_heads_turns_mha_into_gqa():
+    """A GQA weight whose KV heads are replicated g times (consecutive heads,
+    as repeat_kv does) is an MHA weight with equal heads in each group.
+    Pooling it gives the GQA weight back, and the layer computes the same
+    attention as MHA before the transform and as GQA after it."""
+    nh, nkv, hd, D, B, S = 4, 2, 4, 8, 1, 5
+    g = nh // nkv
+    r = rng(41)
+    w_gqa = r.normal(size=((nh + 2 * nkv) * hd, D))
+    kv = [w_gqa[nh * hd + k * nkv * hd: nh * hd + (k + 1) * nkv * hd].reshape(nkv, hd, D) for k in (0, 1)]
+    w_mha = np.concatenate([w_gqa[: nh * hd]] + [np.repeat(t, g, axis=0).reshape(nh * hd, D) for t in kv])
+    pooled = ref.meanpool_kv_projection(w_mha, nh, nkv, hd)
+    np.testing.assert_allclose(pooled, w_gqa, rtol=0, atol=1e-12)
+    x = r.normal(size=(B, S, D))
+    pos = np.arange(S)[None, :]
+    lens = np.array([S])
+    outs = []
+    for w, kvh in ((w_mha, nh), (pooled, nkv)):
+        q, kc, vc = ref.qkv_rope_project(x, w, pos, nh, kvh, hd, 10000.0,
+                                         np.zeros((B, kvh, S, hd)), np.zeros((B, kvh, S, hd)))
+        outs.append(ref.prefill_attention(q, kc, vc, lens, True))
+    np.testing.assert_allclose(outs[0], outs[1], rtol=0, atol=1e-12)
+
+
+def test_meanpool_of_equal_heads_turns_mha_into_gqa():
+    check_meanpool_of_equal_heads_turns_mha_into_gqa()
+
+
+def test_meanpool_brute_force():
+    nh, nkv, hd, D = 6, 2, 2, 3
+    w = rng(42).normal(size=(3 * nh * hd, D))
+    np.testing.assert_allclose(ref.meanpool_kv_projection(w, nh, nkv, hd), brute_meanpool(w, nh, nkv, hd),
+                               rtol=0, atol=1e-12)
+
+
+def test_meanpool_mha_is_identity_and_mqa_averages_every_head():
+    nh, hd, D = 4, 2, 5
+    w = rng(43).normal(size=(3 * nh * hd, D))
+    np.testing.assert_array_equal(ref.meanpool_kv_projection(w, nh, nh, hd), w)     # n_kv_heads = n_heads
+    mqa = ref.meanpool_kv_projection(w, nh, 1, hd)                                   # n_kv_heads = 1
+    assert mqa.shape == ((nh + 2) * hd, D)
+    for block in (1, 2):
+        heads = [w[block * nh * hd + h * hd: block * nh * hd + (h + 1) * hd] for h in range(nh)]
+        want = sum(heads) / nh
+        np.testing.assert_allclose(mqa[nh * hd + (block - 1) * hd: nh * hd + block * hd], want, rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(mqa[: nh * hd], w[: nh * hd])                       # query rows kept
+
+
+def test_meanpool_is_linear():
+    nh, nkv, hd, D = 8, 2, 4, 3
+    r = rng(44)
+    a, b = r.normal(size=(3 * nh * hd, D)), r.normal(size=(3 * nh * hd, D))
+    lhs = ref.meanpool_kv_projection(2.0 * a - 0.5 * b, nh, nkv, hd)
+    rhs = 2.0 * ref.meanpool_kv_projection(a, nh, nkv, hd) - 0.5 * ref.meanpool_kv_projection(b, nh, nkv, hd)
+    np.testing.assert_allclose(lhs, rhs, rtol=0, atol=1e-12)
+
+
+def test_planted_strided_pooling_groups_are_caught(monkeypatch):
+    """Pooling heads h with the same h mod nkv (instead of the consecutive
+    groups h // g that attention reads) breaks the MHA -> GQA identity."""
+    def strided(w, nh, nkv, hd):
+        D = w.shape[1]
+        out = [w[: nh * hd]]
+        for block in (1, 2):
+            heads = w[block * nh * hd:(block + 1) * nh * hd].reshape(nh // nkv, nkv, hd, D)
+            out.append(heads.mean(axis=0).reshape(nkv * hd, D))
+        return np.concatenate(out)
+    monkeypatch.setattr(ref, "meanpool_kv_projection", strided)
+    assert _fails(check_meanpool_of_equal_heads_turns_mha_into_gqa)
+
