@@ -337,8 +337,11 @@ def measure_workloads(dev, peaks, iters=10):
     KV 512..8192, MHA/GQA/MQA caches): KV GB/s; 8K-token prefill (B 2, 16
     heads, hd 128, KV heads 16/4, causal and not): TFLOP/s; the MQA generation
     loop (B 8, hidden 6144, 48 heads, 1 KV head, prompt 16 + 1024 steps):
-    tokens/s.  Each kernel is timed alone with CUDA events, L2 flushed before
-    every timed call (a 512 MB write), median of `iters`."""
+    tokens/s; the TinyLlama layer's smaller prefill shapes (1 x 128, 8 x 512):
+    projection + attention tokens/s; the MHA -> GQA mean-pool weight
+    transform on the Llama-2-7B projection (32 -> 8 KV heads): GB/s.  Each
+    kernel is timed alone with CUDA events, L2 flushed before every timed call
+    (a 512 MB write), median of `iters`."""
     import numpy as np
     import torch
 
@@ -451,6 +454,41 @@ def measure_workloads(dev, peaks, iters=10):
         "weight_stream_GB/s_graph": round(per_step_bytes * T / (ms_graph / 1e3) / 1e9, 1),
         "note": "W_qkv (78.6 MB) is re-read every step and may stay partly L2-resident across steps"}
     del graph
+
+    # ---- TinyLlama layer, the smaller prefill shapes of the same config
+    wl = W.TINYLLAMA_PREFILL
+    sh = wl.shape
+    w = (torch.randn(sh.n_qkv, sh.hidden, generator=gen, device=dev) * 0.02).to(bf)
+    small = {}
+    for (B, S) in wl.batch_seq:
+        if B * S >= 8192:
+            continue            # the 4 x 2048 shape is the bench step itself
+        x = torch.randn(B, S, sh.hidden, generator=gen, device=dev).to(bf)
+        pos = torch.arange(S, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+        q = torch.empty(B, sh.n_heads, S, sh.head_dim, dtype=bf, device=dev)
+        kc = torch.empty(B, sh.n_kv_heads, S, sh.head_dim, dtype=bf, device=dev)
+        vc = torch.empty_like(kc)
+        o = torch.empty(B, S, sh.n_heads, sh.head_dim, dtype=bf, device=dev)
+        ln = torch.full((B,), S, dtype=torch.int32, device=dev)
+        ms_p = timed(lambda: gqa.qkv_rope_project(x, w, pos, sh.n_heads, sh.n_kv_heads, sh.head_dim,
+                                                  sh.rope_theta, q, kc, vc, stream))
+        ms_a = timed(lambda: gqa.gqa_attn_prefill(q, kc, vc, ln, True, o, stream=stream))
+        fl_p = 2.0 * B * S * sh.hidden * sh.n_qkv
+        fl_a = 4.0 * B * sh.n_heads * S * S * sh.head_dim * 0.5
+        small[f"{B}x{S}"] = {"qkv_ms": round(ms_p, 4), "qkv_TFLOP/s": round(fl_p / (ms_p / 1e3) / 1e12, 1),
+                             "attn_ms": round(ms_a, 4), "attn_TFLOP/s": round(fl_a / (ms_a / 1e3) / 1e12, 1),
+                             "tokens_per_s": round(B * S / ((ms_p + ms_a) / 1e3), 1)}
+    out["tinyllama_prefill_small"] = small
+
+    # ---- MHA -> GQA weight transform on the Llama-2-7B projection (32 heads -> 8 KV heads)
+    nh, hd, D, nkv = 32, 128, 4096, 8
+    w_mha = (torch.randn(3 * nh * hd, D, generator=gen, device=dev) * 0.02).to(bf)
+    w_gqa = torch.empty((nh + 2 * nkv) * hd, D, dtype=bf, device=dev)
+    ms = timed(lambda: gqa.gqa_meanpool_kv_heads(w_mha, nh, nkv, hd, w_gqa, stream=stream))
+    nbytes = 2.0 * D * hd * (3 * nh + nh + 2 * nkv)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["mha_to_gqa_meanpool_llama2_7b"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                                            "frac_hbm": round(gbs / hbm, 4), "bytes": int(nbytes)}
     return out
 
 

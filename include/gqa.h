@@ -201,6 +201,33 @@ int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
                             const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,
                             int cache_cap, int kv_split, void* out, int dtype, void* stream);
 
+/*
+ * gqa_meanpool_kv_heads - MHA -> GQA weight transform ("MHA -> GQA: 提升 LLM
+ * 推理效率", section 4.3: the new KV projection of each group of heads is
+ * initialised by mean pooling the group's projections).
+ *
+ * From a fused MHA weight it writes the fused GQA weight with n_kv_heads KV
+ * heads: query rows copied; key (value) row j*head_dim + d of the result is
+ * the mean of rows (j*g + i)*head_dim + d, i < g = n_heads / n_kv_heads, of
+ * the MHA key (value) block.  The groups are the consecutive heads that the
+ * attention calls map onto one KV head (h -> h / g).  Sums in fp32, one
+ * rounding to the dtype.
+ *
+ *   w_qkv_mha  [3 * n_heads * head_dim, hidden] dtype: query, key and value
+ *              blocks of n_heads * head_dim rows each (nn.Linear [out, in])
+ *   w_qkv_gqa  [(n_heads + 2 * n_kv_heads) * head_dim, hidden] dtype, written;
+ *              must not overlap w_qkv_mha
+ *   hidden     a multiple of 8 (bf16) or 4 (fp32): rows are read as 16-byte
+ *              vectors; both pointers 16-byte aligned
+ * n_kv_heads = n_heads copies the weight; n_kv_heads = 1 gives MQA.
+ * Errors: GQA_ERR_INVALID_ARG (null or overlapping buffers, non-positive
+ * sizes, n_heads % n_kv_heads != 0), GQA_ERR_UNSUPPORTED_SHAPE (hidden not a
+ * vector multiple), GQA_ERR_MISALIGNED, GQA_ERR_UNSUPPORTED_DTYPE, and the
+ * device/launch statuses.  Asynchronous on `stream`; allocates nothing.
+ */
+int gqa_meanpool_kv_heads(const void* w_qkv_mha, int hidden, int n_heads, int n_kv_heads, int head_dim,
+                          void* w_qkv_gqa, int dtype, void* stream);
+
 /* Human-readable text of a gqa_status value (static storage). */
 const char* gqa_status_string(int status);
 

@@ -16,7 +16,7 @@ __all__ = [
     "GQA_F32", "GQA_BF16", "GQAError", "library_path", "lib",
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
-    "gqa_launch_count", "gqa_attn_decode_noalloc", "EXPORTED_SYMBOLS",
+    "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -25,7 +25,7 @@ GQA_BF16 = 1
 EXPORTED_SYMBOLS = (
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
-    "gqa_launch_count", "gqa_attn_decode_noalloc",
+    "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
     L.gqa_launch_count.restype = ctypes.c_uint64
     L.gqa_attn_decode_noalloc.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     L.gqa_attn_decode_noalloc.restype = i32
+    L.gqa_meanpool_kv_heads.argtypes = [vp, i32, i32, i32, i32, vp, i32, vp]
+    L.gqa_meanpool_kv_heads.restype = i32
     _LIB = L
     return L
 
@@ -210,3 +212,19 @@ def gqa_attn_decode_noalloc(q, k_cache, v_cache, kv_lens, out, kv_split: int = 0
         _ptr(out, dt, (B, nh, hd), "out"), _dtype_code(q), _stream(stream),
     )
     _check("gqa_attn_decode_noalloc", lib().gqa_attn_decode_noalloc(*args))
+
+
+def gqa_meanpool_kv_heads(w_qkv_mha, n_heads: int, n_kv_heads: int, head_dim: int, w_qkv_gqa,
+                          stream=None) -> None:
+    """MHA -> GQA weight transform: w_qkv_mha [3*nh*hd, hidden] -> w_qkv_gqa
+    [(nh + 2*nkv)*hd, hidden], each group's key/value projections mean-pooled
+    (include/gqa.h)."""
+    dt = w_qkv_mha.dtype
+    hidden = w_qkv_mha.shape[1]
+    args = (
+        _ptr(w_qkv_mha, dt, (3 * n_heads * head_dim, hidden), "w_qkv_mha"), hidden, n_heads, n_kv_heads, head_dim,
+        _ptr(w_qkv_gqa, dt, ((n_heads + 2 * n_kv_heads) * head_dim, hidden), "w_qkv_gqa"),
+        _dtype_code(w_qkv_mha), _stream(stream),
+    )
+    _check("gqa_meanpool_kv_heads", lib().gqa_meanpool_kv_heads(*args))
+

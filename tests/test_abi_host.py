@@ -99,6 +99,23 @@ def test_decode_rejects(kw, code):
     assert _decode(**kw) == code
 
 
+def _meanpool(**kw):
+    a = dict(w=P, hidden=64, nh=8, nkv=2, hd=64, out=P + (1 << 24), dtype=1, stream=None)
+    a.update(kw)
+    return gqa.lib().gqa_meanpool_kv_heads(a["w"], a["hidden"], a["nh"], a["nkv"], a["hd"], a["out"], a["dtype"],
+                                           a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(w=None), INVALID), (dict(out=None), INVALID), (dict(nh=6, nkv=4), INVALID), (dict(nkv=0), INVALID),
+    (dict(hidden=0), INVALID), (dict(hd=-64), INVALID), (dict(hidden=60), SHAPE), (dict(hidden=6, dtype=0), SHAPE),
+    (dict(dtype=5), DTYPE), (dict(w=MIS), MISALIGNED), (dict(out=P + (1 << 24) + 4), MISALIGNED),
+    (dict(out=P + 4096), INVALID),   # output overlaps the input
+])
+def test_meanpool_rejects(kw, code):
+    assert _meanpool(**kw) == code
+
+
 def test_empty_inputs_are_noops():
     # B == 0 or S == 0 returns OK without launching (pointers may then be NULL)
     assert _qkv(B=0, x=None, w=None, pos=None, q=None, k=None, v=None) == 0
@@ -129,3 +146,4 @@ def test_valid_call_without_gpu_reports_no_device():
     assert _qkv() in (NODEV, ARCH)
     assert _prefill() in (NODEV, ARCH)
     assert _decode() in (NODEV, ARCH)
+    assert _meanpool() in (NODEV, ARCH)

@@ -339,3 +339,36 @@ def test_prefill_last_row_equals_decode_on_gpu():
     want = ref.decode_attention(qd.f64, kc.f64, vc.f64, lens)
     gate(host(d), want, dtype, "decode")
     gate(host(out)[:, -1], want, dtype, "prefill last row")
+
+
+# --------------------------------------------------------------------------
+# MHA -> GQA weight transform (mean pooling of each group's KV projections)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype,nh,nkv,hd,D", [
+    ("bf16", 32, 8, 128, 512), ("bf16", 32, 1, 64, 264), ("bf16", 12, 4, 32, 8), ("bf16", 6, 6, 64, 136),
+    ("f32", 12, 4, 64, 100), ("f32", 6, 2, 128, 36),
+])
+def test_meanpool_kv_heads_parity(dtype, nh, nkv, hd, D):
+    w = W.normal_tensor((3 * nh * hd, D), 15, nh + nkv, dtype, std=0.02)
+    out = torch.empty(((nh + 2 * nkv) * hd, D), dtype=TORCH_DT[dtype], device="cuda")
+    gqa.gqa_meanpool_kv_heads(dev(w), nh, nkv, hd, out)
+    want = ref.meanpool_kv_projection(w.f64, nh, nkv, hd)
+    raw = w.store.view(np.uint16 if dtype == "bf16" else np.uint32)
+    assert np.array_equal(bits(out)[: nh * hd], raw[: nh * hd])               # query rows copied bit for bit
+    if nkv == nh:
+        assert np.array_equal(bits(out), raw)                                 # n_kv_heads = n_heads: a copy
+    gate(host(out), want, dtype, "mean-pooled W_qkv")
+
+
+def test_meanpool_of_replicated_kv_heads_is_exact():
+    """An MHA weight whose KV heads repeat each GQA head g times (g a power of
+    two) pools back to the GQA weight bit for bit."""
+    nh, nkv, hd, D = 16, 4, 64, 128
+    g = nh // nkv
+    w_gqa = W.normal_tensor(((nh + 2 * nkv) * hd, D), 16, 0, "bf16", std=0.02)
+    s = w_gqa.store
+    kv = [s[nh * hd + k * nkv * hd: nh * hd + (k + 1) * nkv * hd].reshape(nkv, hd, D) for k in (0, 1)]
+    mha = np.concatenate([s[: nh * hd]] + [np.repeat(t, g, axis=0).reshape(nh * hd, D) for t in kv])
+    out = torch.empty(((nh + 2 * nkv) * hd, D), dtype=torch.bfloat16, device="cuda")
+    gqa.gqa_meanpool_kv_heads(dev(W.Tensor(np.ascontiguousarray(mha), "bf16")), nh, nkv, hd, out)
+    assert np.array_equal(bits(out), s)
