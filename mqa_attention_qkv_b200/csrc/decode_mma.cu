@@ -546,7 +546,6 @@ int cluster_splits(const DecodeParams& p) {
 }  // namespace
 
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
-  static_assert(true, "one m16 tile per head group (see decode_mtiles)");
   switch (p.hd) {
     case 64: return p.cluster ? launch_hd<64, 1, true>(p, st) : launch_hd<64, 1, false>(p, st);
     case 128: return p.cluster ? launch_hd<128, 1, true>(p, st) : launch_hd<128, 1, false>(p, st);

@@ -22,6 +22,8 @@
 // operands, so W and X agree on which K element each slot holds.  The 8
 // warps' accumulators are summed through shared memory, then 64 threads
 // rotate and store the 8 pairs for every token.
+#include <atomic>
+
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -189,6 +191,7 @@ constexpr int SW_KB = 8;                          // 64-column blocks per stage
 constexpr int SW_HALF = SW_KB * 8 * 128;          // 8 rows x 512 columns
 constexpr int SW_STAGE = 2 * SW_HALF;             // lo + hi rows
 constexpr int SW_SMEM_MAX = 227 * 1024;
+constexpr int SW_MAX_NBLK = 256;                  // column-block counts whose launch shape is cached
 constexpr int HD_MAX = 128;
 static_assert(SW_KB == SW_WARPS, "one column block per consumer warp and stage");
 
@@ -405,18 +408,30 @@ cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
   // of a few SMs taking a second unit after everyone else is done.
   int stages = SW_STAGES, per_sm = 1;
   if (n_units > num_sms) {
-    for (int s2 = SW_STAGES; s2 >= 3; --s2) {
-      int fit = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, qkv_stream_kernel<NT, HD>, (SW_WARPS + 1) * 32,
-                                                        stream_smem(NT, nblk, s2)) != cudaSuccess) {
-        cudaGetLastError();
-        break;
+    // the deepest ring with which two CTAs fit on an SM (0: none), found once
+    // per column-block count (a host-side occupancy query per call would sit
+    // in the launch path of every generation step)
+    static std::atomic<int> two_per_sm[SW_MAX_NBLK + 1];   // 0 unknown, -1 none, else stages
+    int known = nblk <= SW_MAX_NBLK ? two_per_sm[nblk].load(std::memory_order_relaxed) : 0;
+    if (known == 0) {
+      known = -1;
+      for (int s2 = SW_STAGES; s2 >= 3; --s2) {
+        int fit = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, qkv_stream_kernel<NT, HD>, (SW_WARPS + 1) * 32,
+                                                          stream_smem(NT, nblk, s2)) != cudaSuccess) {
+          cudaGetLastError();
+          break;
+        }
+        if (fit >= 2) {
+          known = s2;
+          break;
+        }
       }
-      if (fit >= 2) {
-        stages = s2;
-        per_sm = 2;
-        break;
-      }
+      if (nblk <= SW_MAX_NBLK) two_per_sm[nblk].store(known, std::memory_order_relaxed);
+    }
+    if (known > 0) {
+      stages = known;
+      per_sm = 2;
     }
   }
   const size_t smem = stream_smem(NT, nblk, stages);
