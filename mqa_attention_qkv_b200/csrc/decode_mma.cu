@@ -495,15 +495,10 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
 template <int HD, int MT, bool CL>
 cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
   using C = DCfg<HD, MT>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e =
-        cudaFuncSetAttribute(decode_mma_kernel<HD, MT, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(decode_mma_kernel<HD, MT, CL>), C::SMEM);
+      e != cudaSuccess)
+    return e;
   CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)p.B * p.nkv * p.cap;
   if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;

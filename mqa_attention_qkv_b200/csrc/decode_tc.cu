@@ -418,14 +418,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
 template <int HD>
 cudaError_t launch_hd(const DecodeParams& p, int n_hg, cudaStream_t st) {
   using C = DtCfg<HD>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(decode_tc_kernel<HD>), C::SMEM);
+      e != cudaSuccess)
+    return e;
   CUtensorMap tq, tk, tv;
   const uint64_t q_rows = (uint64_t)p.B * p.nh, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
   if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, BM)) return cudaErrorInvalidValue;

@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace gqa {
 
 struct QkvParams {
@@ -91,6 +93,23 @@ int decode_tc_splits(const DecodeParams& p);
 // counters), else SIMT partials + the log-sum-exp combine kernel.  Partial m
 // is in log2 units.  Returns the number of kernels launched; *err the status.
 int launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st, cudaError_t* err);
+
+// Raise a kernel's dynamic shared-memory limit on the current device, once per
+// device (`done` is the caller's per-kernel flag array).  The attribute is
+// idempotent, so two threads racing on a first call both set it; devices past
+// the array are set on every call.
+inline cudaError_t smem_attr_once(std::atomic<bool> (&done)[64], const void* func, int bytes) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = -1;
+  }
+  const bool cached = dev >= 0 && dev < 64;
+  if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cached) done[dev].store(true, std::memory_order_release);
+  return e;
+}
 
 // 2-D bf16 TMA descriptor with 128-byte swizzle; `map` points at a CUtensorMap.
 // Zero fill outside [0, inner) x [0, outer).  False if encoding fails.

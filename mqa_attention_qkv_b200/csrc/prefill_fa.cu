@@ -412,14 +412,10 @@ prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 template <int HD, int POLY>
 cudaError_t launch_hd(const PrefillParams& p, cudaStream_t st) {
   using C = FaCfg<HD>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_fa_kernel<HD, POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(prefill_fa_kernel<HD, POLY>), C::SMEM);
+      e != cudaSuccess)
+    return e;
   CUtensorMap tq, tk, tv;
   const uint64_t q_rows = (uint64_t)p.B * p.nh * p.S, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
   if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;

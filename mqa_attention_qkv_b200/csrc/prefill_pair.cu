@@ -308,14 +308,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st) {
   if (p.hd != HD) return cudaErrorInvalidValue;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(prefill_pair_kernel), SMEM);
+      e != cudaSuccess)
+    return e;
   CUtensorMap tq, tk, tv;
   const uint64_t q_rows = (uint64_t)p.B * p.nh * p.S, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
   if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;

@@ -392,15 +392,10 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
 template <int NT, int HD>
 cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
   const int nblk = p.hidden / 64;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(qkv_stream_kernel<NT, HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SW_SMEM_MAX);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(qkv_stream_kernel<NT, HD>), SW_SMEM_MAX);
+      e != cudaSuccess)
+    return e;
   const int N = (p.nh + 2 * p.nkv) * HD;
   const int n_units = N / 16;
   // More units than SMs and small hidden states: two CTAs per SM with a

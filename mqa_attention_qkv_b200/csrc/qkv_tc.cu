@@ -230,14 +230,10 @@ qkv_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ C
 
 template <int HD>
 cudaError_t launch_hd(const CUtensorMap& tx, const CUtensorMap& tw, const TcArgs& a, int grid, cudaStream_t st) {
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(qkv_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(qkv_tc_kernel<HD>), SMEM_BYTES);
+      e != cudaSuccess)
+    return e;
   qkv_tc_kernel<HD><<<grid, THREADS, SMEM_BYTES, st>>>(tx, tw, a);
   return cudaGetLastError();
 }
