@@ -21,6 +21,10 @@ Sources (page title, then section):
 * custom-op overhead gist (``overhead.py``): ``forward(positions,
   hidden_states)`` applies a position-dependent step to q and k only, after
   the fused projection.
+* "MHA -> GQA: 提升 LLM 推理效率", section 3.2: a PagedAttention KV cache is
+  stored non-contiguously, in fixed-size pages that a block table maps to each
+  sequence (the paged decode here keeps the tensor cores by making pages whole
+  key tiles).
 * "MHA -> GQA: 提升 LLM 推理效率", section 4.3 (剪枝训练): the new KV projection
   of each group of heads is initialised by mean pooling the group's
   projections (the offline MHA -> GQA weight transform).
@@ -268,4 +272,31 @@ def meanpool_kv_projection(w_qkv_mha: np.ndarray, n_heads: int, n_kv_heads: int,
         heads = w[block * nh * hd:(block + 1) * nh * hd].reshape(nh, hd, D)
         out.append(heads.reshape(nkv, g, hd, D).mean(axis=1).reshape(nkv * hd, D))
     return np.concatenate(out, axis=0)
+
+
+def gather_pages(pages: np.ndarray, block_table: np.ndarray, kv_lens: np.ndarray, page_size: int) -> np.ndarray:
+    """The logical cache ``[B, nkv, cap, hd]`` (cap = pages per sequence x
+    page size) of a paged cache: key t of sequence b lives in physical page
+    ``block_table[b, t // page_size]`` at row ``t % page_size``; ``pages`` is
+    ``[num_pages, nkv, page_size, hd]``.  Rows at or past a sequence's length
+    are NaN (never read by attention)."""
+    pages = np.asarray(pages, dtype=np.float64)
+    B, max_pages = block_table.shape
+    _, nkv, ps, hd = pages.shape
+    assert ps == page_size
+    out = np.full((B, nkv, max_pages * ps, hd), np.nan)
+    for b in range(B):
+        L = int(kv_lens[b])
+        for t in range(0, max(L, 0), ps):
+            n = min(ps, L - t)
+            out[b, :, t:t + n] = pages[int(block_table[b, t // ps]), :, :n]
+    return out
+
+
+def paged_decode_attention(q, k_pages, v_pages, block_table, kv_lens, page_size, pairs=None):
+    """Decode attention over a paged KV cache: the plain decode over the
+    logical rows that the block table names."""
+    kc = gather_pages(k_pages, block_table, kv_lens, page_size)
+    vc = gather_pages(v_pages, block_table, kv_lens, page_size)
+    return decode_attention(q, kc, vc, kv_lens, pairs=pairs)
 

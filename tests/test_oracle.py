@@ -640,3 +640,78 @@ def test_planted_strided_pooling_groups_are_caught(monkeypatch):
     monkeypatch.setattr(ref, "meanpool_kv_projection", strided)
     assert _fails(check_meanpool_of_equal_heads_turns_mha_into_gqa)
 
+
+# --------------------------------------------------------------------------
+# paged KV cache (MHA -> GQA blog, section 3.2: PagedAttention's
+# non-contiguous cache)
+# --------------------------------------------------------------------------
+def paged_setup(seed=51, B=3, nkv=2, nh=4, hd=4, ps=4, max_pages=3):
+    r = rng(seed)
+    cap = ps * max_pages
+    kc, vc = r.normal(size=(B, nkv, cap, hd)), r.normal(size=(B, nkv, cap, hd))
+    q = r.normal(size=(B, nh, hd))
+    lens = np.array([cap, 5, 1])[:B]
+    # the contiguous cache cut into pages: page (b, p) = rows [p*ps, (p+1)*ps) of sequence b
+    kp = kc.reshape(B, nkv, max_pages, ps, hd).transpose(0, 2, 1, 3, 4).reshape(B * max_pages, nkv, ps, hd)
+    vp = vc.reshape(B, nkv, max_pages, ps, hd).transpose(0, 2, 1, 3, 4).reshape(B * max_pages, nkv, ps, hd)
+    table = np.arange(B * max_pages).reshape(B, max_pages)
+    return q, kc, vc, kp, vp, table, lens, ps
+
+
+def check_paged_page_order_does_not_matter():
+    q, kc, vc, kp, vp, table, lens, ps = paged_setup()
+    base = ref.paged_decode_attention(q, kp, vp, table, lens, ps)
+    perm = rng(52).permutation(kp.shape[0])            # physical page i moves to slot perm[i]
+    kp2, vp2 = np.empty_like(kp), np.empty_like(vp)
+    kp2[perm], vp2[perm] = kp, vp
+    np.testing.assert_array_equal(ref.paged_decode_attention(q, kp2, vp2, perm[table], lens, ps), base)
+
+
+def test_paged_cache_with_identity_table_is_the_contiguous_cache():
+    q, kc, vc, kp, vp, table, lens, ps = paged_setup()
+    g = ref.gather_pages(kp, table, lens, ps)
+    for b, L in enumerate(lens):
+        np.testing.assert_array_equal(g[b, :, :L], kc[b, :, :L])
+        assert np.all(np.isnan(g[b, :, L:]))
+    np.testing.assert_array_equal(ref.paged_decode_attention(q, kp, vp, table, lens, ps),
+                                  ref.decode_attention(q, kc, vc, lens))
+
+
+def test_paged_page_order_does_not_matter():
+    check_paged_page_order_does_not_matter()
+
+
+def test_paged_brute_force():
+    q, kc, vc, kp, vp, table, lens, ps = paged_setup(seed=53)
+    perm = rng(54).permutation(kp.shape[0])
+    kp2, vp2 = np.empty_like(kp), np.empty_like(vp)
+    kp2[perm], vp2[perm] = kp, vp
+    t2 = perm[table]
+    B, nh, hd = q.shape
+    nkv = kp.shape[1]
+    want = np.zeros((B, nh, hd))
+    for b in range(B):
+        for h in range(nh):
+            j = h // (nh // nkv)
+            scores, vals = [], []
+            for t in range(int(lens[b])):
+                page, row = int(t2[b, t // ps]), t % ps
+                scores.append(sum(float(q[b, h, d]) * float(kp2[page, j, row, d]) for d in range(hd)) / math.sqrt(hd))
+                vals.append(vp2[page, j, row])
+            m = max(scores)
+            w = [math.exp(s_ - m) for s_ in scores]
+            want[b, h] = sum(wi * vi for wi, vi in zip(w, vals)) / sum(w)
+    np.testing.assert_allclose(ref.paged_decode_attention(q, kp2, vp2, t2, lens, ps), want, rtol=0, atol=1e-12)
+
+
+def test_planted_ignored_block_table_is_caught(monkeypatch):
+    """Reading page p of sequence b from physical page b*max_pages + p (the
+    table ignored) breaks the page-order invariance."""
+    orig = ref.gather_pages
+
+    def ignore_table(pages, block_table, kv_lens, page_size):
+        B, max_pages = block_table.shape
+        return orig(pages, np.arange(B * max_pages).reshape(B, max_pages), kv_lens, page_size)
+    monkeypatch.setattr(ref, "gather_pages", ignore_table)
+    assert _fails(check_paged_page_order_does_not_matter)
+
