@@ -332,16 +332,18 @@ def _set_mb(st):
 # ---------------------------------------------------------------------------
 # the other workloads of the metric, measured kernel by kernel
 # ---------------------------------------------------------------------------
-def measure_workloads(dev, peaks, iters=10):
+def measure_workloads(dev, peaks, iters=10, only=None):
     """Llama-2-7B-shaped batched decode (B 64, 32 query heads, hd 128, ragged
-    KV 512..8192, MHA/GQA/MQA caches): KV GB/s; 8K-token prefill (B 2, 16
+    KV 512..8192, MHA/GQA/MQA caches, contiguous and in shuffled 64-key
+    pages): KV GB/s; 8K-token prefill (B 2, 16
     heads, hd 128, KV heads 16/4, causal and not): TFLOP/s; the MQA generation
     loop (B 8, hidden 6144, 48 heads, 1 KV head, prompt 16 + 1024 steps):
     tokens/s; the TinyLlama layer's smaller prefill shapes (1 x 128, 8 x 512):
     projection + attention tokens/s; the MHA -> GQA mean-pool weight
     transform on the Llama-2-7B projection (32 -> 8 KV heads): GB/s.  Each
     kernel is timed alone with CUDA events, L2 flushed before every timed call
-    (a 512 MB write), median of `iters`."""
+    (a 512 MB write), median of `iters`.  ``only``: a set of section names
+    (decode, prefill8k, generate, small, meanpool) to measure; None = all."""
     import numpy as np
     import torch
 
@@ -370,125 +372,148 @@ def measure_workloads(dev, peaks, iters=10):
     out = {}
     hbm, bf16_peak = peaks["hbm_gbs"], peaks["bf16_tflops"]
 
+    want = (lambda name: only is None or name in only)
+
     # ---- batched decode
-    wl = W.LLAMA2_DECODE
-    e = wl.extra
-    B, nh, hd, cap = e["batch"], wl.shape.n_heads, wl.shape.head_dim, e["cap"]
-    lens_np = W.ragged_lengths(B, e["kv_lo"], e["kv_hi"], wl.seed)
-    lens = torch.from_numpy(lens_np).to(dev)
-    q = torch.randn(B, nh, hd, generator=gen, device=dev).to(bf)
-    dec = {}
-    for nkv in e["n_kv_heads_cases"]:
-        kc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
-        vc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
-        o = torch.empty(B, nh, hd, dtype=bf, device=dev)
-        ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
-        ms = timed(lambda: gqa.gqa_attn_decode(q, kc, vc, lens, o, ws, stream=stream))
-        nbytes = 2.0 * (2 * nkv * hd * float(lens_np.sum()) + 2 * B * nh * hd)
-        gbs = nbytes / (ms / 1e3) / 1e9
-        dec[f"nkv{nkv}"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
-                            "bytes": int(nbytes)}
-        del kc, vc
-    out["llama2_decode_b64"] = dec
+    if want("decode"):
+        wl = W.LLAMA2_DECODE
+        e = wl.extra
+        B, nh, hd, cap = e["batch"], wl.shape.n_heads, wl.shape.head_dim, e["cap"]
+        lens_np = W.ragged_lengths(B, e["kv_lo"], e["kv_hi"], wl.seed)
+        lens = torch.from_numpy(lens_np).to(dev)
+        q = torch.randn(B, nh, hd, generator=gen, device=dev).to(bf)
+        dec = {}
+        for nkv in e["n_kv_heads_cases"]:
+            kc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
+            vc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
+            o = torch.empty(B, nh, hd, dtype=bf, device=dev)
+            ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
+            ms = timed(lambda: gqa.gqa_attn_decode(q, kc, vc, lens, o, ws, stream=stream))
+            nbytes = 2.0 * (2 * nkv * hd * float(lens_np.sum()) + 2 * B * nh * hd)
+            gbs = nbytes / (ms / 1e3) / 1e9
+            dec[f"nkv{nkv}"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                                "bytes": int(nbytes)}
+            # the same cache cut into 64-key pages, shuffled over the page pool
+            ps, maxp = 64, cap // 64
+            perm = torch.randperm(B * maxp, generator=torch.Generator().manual_seed(nkv)).to(dev)
+            table = perm.view(B, maxp).to(torch.int32).contiguous()
+
+            def paged(c):
+                pool = torch.empty(B * maxp, nkv, ps, hd, dtype=bf, device=dev)
+                pool[perm] = c.view(B, nkv, maxp, ps, hd).transpose(1, 2).reshape(B * maxp, nkv, ps, hd)
+                return pool
+
+            kp, vp = paged(kc), paged(vc)
+            del kc, vc
+            ms = timed(lambda: gqa.gqa_attn_decode_paged(q, kp, vp, table, lens, o, ws, stream=stream))
+            gbs = nbytes / (ms / 1e3) / 1e9
+            dec[f"nkv{nkv}_paged64"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                                        "bytes": int(nbytes)}
+            del kp, vp
+        out["llama2_decode_b64"] = dec
 
     # ---- long-context prefill
-    wl = W.LONG_PREFILL
-    B, S = wl.batch_seq[0]
-    nh, hd = wl.shape.n_heads, wl.shape.head_dim
-    lp = {}
-    for nkv in wl.extra["n_kv_heads_cases"]:
-        q = torch.randn(B, nh, S, hd, generator=gen, device=dev).to(bf)
-        k = torch.randn(B, nkv, S, hd, generator=gen, device=dev).to(bf)
-        v = torch.randn(B, nkv, S, hd, generator=gen, device=dev).to(bf)
-        o = torch.empty(B, S, nh, hd, dtype=bf, device=dev)
-        ln = torch.full((B,), S, dtype=torch.int32, device=dev)
-        for causal in (True, False):
-            ms = timed(lambda: gqa.gqa_attn_prefill(q, k, v, ln, causal, o, stream=stream))
-            fl = 4.0 * B * nh * S * S * hd * (0.5 if causal else 1.0)
-            tf = fl / (ms / 1e3) / 1e12
-            lp[f"nkv{nkv}_{'causal' if causal else 'full'}"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
-                                                                 "frac_bf16": round(tf / bf16_peak, 4)}
-    out["long_prefill_2x8192"] = lp
+    if want("prefill8k"):
+        wl = W.LONG_PREFILL
+        B, S = wl.batch_seq[0]
+        nh, hd = wl.shape.n_heads, wl.shape.head_dim
+        lp = {}
+        for nkv in wl.extra["n_kv_heads_cases"]:
+            q = torch.randn(B, nh, S, hd, generator=gen, device=dev).to(bf)
+            k = torch.randn(B, nkv, S, hd, generator=gen, device=dev).to(bf)
+            v = torch.randn(B, nkv, S, hd, generator=gen, device=dev).to(bf)
+            o = torch.empty(B, S, nh, hd, dtype=bf, device=dev)
+            ln = torch.full((B,), S, dtype=torch.int32, device=dev)
+            for causal in (True, False):
+                ms = timed(lambda: gqa.gqa_attn_prefill(q, k, v, ln, causal, o, stream=stream))
+                fl = 4.0 * B * nh * S * S * hd * (0.5 if causal else 1.0)
+                tf = fl / (ms / 1e3) / 1e12
+                lp[f"nkv{nkv}_{'causal' if causal else 'full'}"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                                                     "frac_bf16": round(tf / bf16_peak, 4)}
+        out["long_prefill_2x8192"] = lp
 
     # ---- MQA generation loop (prompt 16, 1024 steps), one timed region
-    wl = W.MQA_GENERATE
-    sh, e = wl.shape, wl.extra
-    B, P, T, cap = e["batch"], e["prompt"], e["steps"], e["cap"]
-    nh, nkv, hd = sh.n_heads, sh.n_kv_heads, sh.head_dim
-    w = (torch.randn(sh.n_qkv, sh.hidden, generator=gen, device=dev) * 0.02).to(bf)
-    xp = torch.randn(B, P, sh.hidden, generator=gen, device=dev).to(bf)
-    xs = torch.randn(T, B, 1, sh.hidden, generator=gen, device=dev).to(bf)
-    kc = torch.zeros(B, nkv, cap, hd, dtype=bf, device=dev)
-    vc = torch.zeros_like(kc)
-    qp = torch.empty(B, nh, P, hd, dtype=bf, device=dev)
-    op = torch.empty(B, P, nh, hd, dtype=bf, device=dev)
-    qt = torch.empty(B, nh, 1, hd, dtype=bf, device=dev)
-    ot = torch.empty(T, B, nh, hd, dtype=bf, device=dev)
-    posp = torch.arange(P, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
-    pos_steps = (P + torch.arange(T, dtype=torch.int32, device=dev)).view(T, 1, 1).expand(T, B, 1).contiguous()
-    len_steps = (P + 1 + torch.arange(T, dtype=torch.int32, device=dev)).view(T, 1).expand(T, B).contiguous()
-    lp_ = torch.full((B,), P, dtype=torch.int32, device=dev)
-    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
+    if want("generate"):
+        wl = W.MQA_GENERATE
+        sh, e = wl.shape, wl.extra
+        B, P, T, cap = e["batch"], e["prompt"], e["steps"], e["cap"]
+        nh, nkv, hd = sh.n_heads, sh.n_kv_heads, sh.head_dim
+        w = (torch.randn(sh.n_qkv, sh.hidden, generator=gen, device=dev) * 0.02).to(bf)
+        xp = torch.randn(B, P, sh.hidden, generator=gen, device=dev).to(bf)
+        xs = torch.randn(T, B, 1, sh.hidden, generator=gen, device=dev).to(bf)
+        kc = torch.zeros(B, nkv, cap, hd, dtype=bf, device=dev)
+        vc = torch.zeros_like(kc)
+        qp = torch.empty(B, nh, P, hd, dtype=bf, device=dev)
+        op = torch.empty(B, P, nh, hd, dtype=bf, device=dev)
+        qt = torch.empty(B, nh, 1, hd, dtype=bf, device=dev)
+        ot = torch.empty(T, B, nh, hd, dtype=bf, device=dev)
+        posp = torch.arange(P, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+        pos_steps = (P + torch.arange(T, dtype=torch.int32, device=dev)).view(T, 1, 1).expand(T, B, 1).contiguous()
+        len_steps = (P + 1 + torch.arange(T, dtype=torch.int32, device=dev)).view(T, 1).expand(T, B).contiguous()
+        lp_ = torch.full((B,), P, dtype=torch.int32, device=dev)
+        ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
 
-    def gen_loop():
-        st = torch.cuda.current_stream(dev)   # the capture stream while a graph is being recorded
-        gqa.qkv_rope_project(xp, w, posp, nh, nkv, hd, sh.rope_theta, qp, kc, vc, st)
-        gqa.gqa_attn_prefill(qp, kc, vc, lp_, True, op, stream=st)
-        for t in range(T):
-            gqa.qkv_rope_project(xs[t], w, pos_steps[t], nh, nkv, hd, sh.rope_theta, qt, kc, vc, st)
-            gqa.gqa_attn_decode(qt.view(B, nh, hd), kc, vc, len_steps[t], ot[t], ws, stream=st)
+        def gen_loop():
+            st = torch.cuda.current_stream(dev)   # the capture stream while a graph is being recorded
+            gqa.qkv_rope_project(xp, w, posp, nh, nkv, hd, sh.rope_theta, qp, kc, vc, st)
+            gqa.gqa_attn_prefill(qp, kc, vc, lp_, True, op, stream=st)
+            for t in range(T):
+                gqa.qkv_rope_project(xs[t], w, pos_steps[t], nh, nkv, hd, sh.rope_theta, qt, kc, vc, st)
+                gqa.gqa_attn_decode(qt.view(B, nh, hd), kc, vc, len_steps[t], ot[t], ws, stream=st)
 
-    gen_loop()
-    ms_direct = timed_once(gen_loop, stream)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
         gen_loop()
-    graph.replay()
-    ms_graph = timed_once(graph.replay, stream)
-    toks = B * (P + T)
-    per_step_bytes = 2.0 * sh.n_qkv * sh.hidden
-    out["mqa_generate_b8_p16_g1024"] = {
-        "ms_direct": round(ms_direct, 3), "ms_graph": round(ms_graph, 3),
-        "tokens_per_s_direct": round(toks / (ms_direct / 1e3), 1),
-        "tokens_per_s_graph": round(toks / (ms_graph / 1e3), 1),
-        "weight_stream_GB/s_graph": round(per_step_bytes * T / (ms_graph / 1e3) / 1e9, 1),
-        "note": "W_qkv (78.6 MB) is re-read every step and may stay partly L2-resident across steps"}
-    del graph
+        ms_direct = timed_once(gen_loop, stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            gen_loop()
+        graph.replay()
+        ms_graph = timed_once(graph.replay, stream)
+        toks = B * (P + T)
+        per_step_bytes = 2.0 * sh.n_qkv * sh.hidden
+        out["mqa_generate_b8_p16_g1024"] = {
+            "ms_direct": round(ms_direct, 3), "ms_graph": round(ms_graph, 3),
+            "tokens_per_s_direct": round(toks / (ms_direct / 1e3), 1),
+            "tokens_per_s_graph": round(toks / (ms_graph / 1e3), 1),
+            "weight_stream_GB/s_graph": round(per_step_bytes * T / (ms_graph / 1e3) / 1e9, 1),
+            "note": "W_qkv (78.6 MB) is re-read every step and may stay partly L2-resident across steps"}
+        del graph
 
     # ---- TinyLlama layer, the smaller prefill shapes of the same config
-    wl = W.TINYLLAMA_PREFILL
-    sh = wl.shape
-    w = (torch.randn(sh.n_qkv, sh.hidden, generator=gen, device=dev) * 0.02).to(bf)
-    small = {}
-    for (B, S) in wl.batch_seq:
-        if B * S >= 8192:
-            continue            # the 4 x 2048 shape is the bench step itself
-        x = torch.randn(B, S, sh.hidden, generator=gen, device=dev).to(bf)
-        pos = torch.arange(S, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
-        q = torch.empty(B, sh.n_heads, S, sh.head_dim, dtype=bf, device=dev)
-        kc = torch.empty(B, sh.n_kv_heads, S, sh.head_dim, dtype=bf, device=dev)
-        vc = torch.empty_like(kc)
-        o = torch.empty(B, S, sh.n_heads, sh.head_dim, dtype=bf, device=dev)
-        ln = torch.full((B,), S, dtype=torch.int32, device=dev)
-        ms_p = timed(lambda: gqa.qkv_rope_project(x, w, pos, sh.n_heads, sh.n_kv_heads, sh.head_dim,
-                                                  sh.rope_theta, q, kc, vc, stream))
-        ms_a = timed(lambda: gqa.gqa_attn_prefill(q, kc, vc, ln, True, o, stream=stream))
-        fl_p = 2.0 * B * S * sh.hidden * sh.n_qkv
-        fl_a = 4.0 * B * sh.n_heads * S * S * sh.head_dim * 0.5
-        small[f"{B}x{S}"] = {"qkv_ms": round(ms_p, 4), "qkv_TFLOP/s": round(fl_p / (ms_p / 1e3) / 1e12, 1),
-                             "attn_ms": round(ms_a, 4), "attn_TFLOP/s": round(fl_a / (ms_a / 1e3) / 1e12, 1),
-                             "tokens_per_s": round(B * S / ((ms_p + ms_a) / 1e3), 1)}
-    out["tinyllama_prefill_small"] = small
+    if want("small"):
+        wl = W.TINYLLAMA_PREFILL
+        sh = wl.shape
+        w = (torch.randn(sh.n_qkv, sh.hidden, generator=gen, device=dev) * 0.02).to(bf)
+        small = {}
+        for (B, S) in wl.batch_seq:
+            if B * S >= 8192:
+                continue            # the 4 x 2048 shape is the bench step itself
+            x = torch.randn(B, S, sh.hidden, generator=gen, device=dev).to(bf)
+            pos = torch.arange(S, dtype=torch.int32, device=dev).repeat(B, 1).contiguous()
+            q = torch.empty(B, sh.n_heads, S, sh.head_dim, dtype=bf, device=dev)
+            kc = torch.empty(B, sh.n_kv_heads, S, sh.head_dim, dtype=bf, device=dev)
+            vc = torch.empty_like(kc)
+            o = torch.empty(B, S, sh.n_heads, sh.head_dim, dtype=bf, device=dev)
+            ln = torch.full((B,), S, dtype=torch.int32, device=dev)
+            ms_p = timed(lambda: gqa.qkv_rope_project(x, w, pos, sh.n_heads, sh.n_kv_heads, sh.head_dim,
+                                                      sh.rope_theta, q, kc, vc, stream))
+            ms_a = timed(lambda: gqa.gqa_attn_prefill(q, kc, vc, ln, True, o, stream=stream))
+            fl_p = 2.0 * B * S * sh.hidden * sh.n_qkv
+            fl_a = 4.0 * B * sh.n_heads * S * S * sh.head_dim * 0.5
+            small[f"{B}x{S}"] = {"qkv_ms": round(ms_p, 4), "qkv_TFLOP/s": round(fl_p / (ms_p / 1e3) / 1e12, 1),
+                                 "attn_ms": round(ms_a, 4), "attn_TFLOP/s": round(fl_a / (ms_a / 1e3) / 1e12, 1),
+                                 "tokens_per_s": round(B * S / ((ms_p + ms_a) / 1e3), 1)}
+        out["tinyllama_prefill_small"] = small
 
     # ---- MHA -> GQA weight transform on the Llama-2-7B projection (32 heads -> 8 KV heads)
-    nh, hd, D, nkv = 32, 128, 4096, 8
-    w_mha = (torch.randn(3 * nh * hd, D, generator=gen, device=dev) * 0.02).to(bf)
-    w_gqa = torch.empty((nh + 2 * nkv) * hd, D, dtype=bf, device=dev)
-    ms = timed(lambda: gqa.gqa_meanpool_kv_heads(w_mha, nh, nkv, hd, w_gqa, stream=stream))
-    nbytes = 2.0 * D * hd * (3 * nh + nh + 2 * nkv)
-    gbs = nbytes / (ms / 1e3) / 1e9
-    out["mha_to_gqa_meanpool_llama2_7b"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
-                                            "frac_hbm": round(gbs / hbm, 4), "bytes": int(nbytes)}
+    if want("meanpool"):
+        nh, hd, D, nkv = 32, 128, 4096, 8
+        w_mha = (torch.randn(3 * nh * hd, D, generator=gen, device=dev) * 0.02).to(bf)
+        w_gqa = torch.empty((nh + 2 * nkv) * hd, D, dtype=bf, device=dev)
+        ms = timed(lambda: gqa.gqa_meanpool_kv_heads(w_mha, nh, nkv, hd, w_gqa, stream=stream))
+        nbytes = 2.0 * D * hd * (3 * nh + nh + 2 * nkv)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out["mha_to_gqa_meanpool_llama2_7b"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                                                "frac_hbm": round(gbs / hbm, 4), "bytes": int(nbytes)}
     return out
 
 

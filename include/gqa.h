@@ -64,7 +64,8 @@ enum gqa_status {
 enum gqa_device_error_bits {
   GQA_DEVERR_POSITION_RANGE = 1,   /* a position outside [0, cache_cap): K/V row not written */
   GQA_DEVERR_KVLEN_RANGE = 2,      /* a kv_len above cache_cap (clamped) or below 0 (taken as 0) */
-  GQA_DEVERR_WAIT_TIMEOUT = 4      /* a pipeline wait gave up after its time limit */
+  GQA_DEVERR_WAIT_TIMEOUT = 4,     /* a pipeline wait gave up after its time limit */
+  GQA_DEVERR_PAGE_RANGE = 8        /* a block-table entry outside [0, num_pages): read as zeros */
 };
 
 /*
@@ -227,6 +228,46 @@ int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
  */
 int gqa_meanpool_kv_heads(const void* w_qkv_mha, int hidden, int n_heads, int n_kv_heads, int head_dim,
                           void* w_qkv_gqa, int dtype, void* stream);
+
+/*
+ * gqa_attn_decode_paged - gqa_attn_decode over a paged KV cache.
+ *
+ * Source: "MHA -> GQA: 提升 LLM 推理效率", section 3.2: a PagedAttention cache
+ * keeps each sequence's keys and values in fixed-size pages that need not be
+ * contiguous, and a block table lists a sequence's pages in order.  The
+ * attention is exactly gqa_attn_decode over the cache that the table
+ * describes; only the address of each key row changes.  Pages hold a whole
+ * number of 64-key tiles, so every tile the kernel copies lies inside one
+ * page and is fetched with one tensor copy per 64 columns, as in the
+ * contiguous case.
+ *
+ *   q            [B, n_heads, head_dim] bf16
+ *   k_pages,
+ *   v_pages      [num_pages, n_kv_heads, page_size, head_dim] bf16: key t of
+ *                sequence b is row t % page_size of page
+ *                block_table[b][t / page_size], for every KV head
+ *   block_table  [B, max_pages] int32, row-major; entries past a sequence's
+ *                last page are not read.  An entry outside [0, num_pages)
+ *                raises GQA_DEVERR_PAGE_RANGE and its keys read as zeros
+ *   kv_lens      [B] int32: clamped to [0, max_pages * page_size]
+ *                (GQA_DEVERR_KVLEN_RANGE)
+ *   page_size    keys per page: a positive multiple of 64
+ *   kv_split     as for gqa_attn_decode, with cache_cap = max_pages * page_size
+ *   out          [B, n_heads, head_dim] bf16
+ *   workspace    as for gqa_attn_decode: at least
+ *                gqa_attn_decode_workspace_size(B, n_heads, n_kv_heads,
+ *                head_dim, max_pages * page_size, kv_split) bytes, zero-filled
+ *                before its first use
+ *
+ * bf16 with head_dim 64 or 128 only (GQA_ERR_UNSUPPORTED_DTYPE /
+ * GQA_ERR_UNSUPPORTED_SHAPE otherwise).  Same statuses as gqa_attn_decode;
+ * asynchronous on `stream`.
+ */
+int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                          const int32_t* block_table, const int32_t* kv_lens, int B, int n_heads,
+                          int n_kv_heads, int head_dim, int page_size, int max_pages, int num_pages,
+                          int kv_split, void* out, void* workspace, size_t workspace_bytes, int dtype,
+                          void* stream);
 
 /* Human-readable text of a gqa_status value (static storage). */
 const char* gqa_status_string(int status);

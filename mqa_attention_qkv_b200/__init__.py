@@ -16,7 +16,8 @@ __all__ = [
     "GQA_F32", "GQA_BF16", "GQAError", "library_path", "lib",
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
-    "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "EXPORTED_SYMBOLS",
+    "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
+    "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -25,7 +26,7 @@ GQA_BF16 = 1
 EXPORTED_SYMBOLS = (
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
-    "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads",
+    "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +72,9 @@ def lib() -> ctypes.CDLL:
     L.gqa_attn_decode_noalloc.restype = i32
     L.gqa_meanpool_kv_heads.argtypes = [vp, i32, i32, i32, i32, vp, i32, vp]
     L.gqa_meanpool_kv_heads.restype = i32
+    L.gqa_attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, sz,
+                                        i32, vp]
+    L.gqa_attn_decode_paged.restype = i32
     _LIB = L
     return L
 
@@ -182,6 +186,29 @@ def gqa_attn_decode(q, k_cache, v_cache, kv_lens, out, workspace, kv_split: int 
         _dtype_code(q), _stream(stream),
     )
     _check("gqa_attn_decode", lib().gqa_attn_decode(*args))
+
+
+def gqa_attn_decode_paged(q, k_pages, v_pages, block_table, kv_lens, out, workspace, kv_split: int = 0,
+                          stream=None) -> None:
+    """q [B,nh,hd] bf16, pages [num_pages,nkv,page_size,hd] bf16, block_table
+    [B,max_pages] int32, kv_lens [B] int32 -> out [B,nh,hd].  ``workspace`` as
+    for gqa_attn_decode with cache_cap = max_pages * page_size."""
+    import torch
+    B, nh, hd = q.shape
+    num_pages, nkv, page_size = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    max_pages = block_table.shape[1]
+    dt = q.dtype
+    ws_bytes = workspace.numel() * workspace.element_size()
+    args = (
+        _ptr(q, dt, name="q"), _ptr(k_pages, dt, (num_pages, nkv, page_size, hd), "k_pages"),
+        _ptr(v_pages, dt, (num_pages, nkv, page_size, hd), "v_pages"),
+        _ptr(block_table, torch.int32, (B, max_pages), "block_table"),
+        _ptr(kv_lens, torch.int32, (B,), "kv_lens"),
+        B, nh, nkv, hd, page_size, max_pages, num_pages, int(kv_split),
+        _ptr(out, dt, (B, nh, hd), "out"), _ptr(workspace, name="workspace"), ws_bytes,
+        _dtype_code(q), _stream(stream),
+    )
+    _check("gqa_attn_decode_paged", lib().gqa_attn_decode_paged(*args))
 
 
 def gqa_device_error() -> int:

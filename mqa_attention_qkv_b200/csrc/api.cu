@@ -110,7 +110,7 @@ DecodeParams decode_params(const void* q, const void* k_cache, const void* v_cac
   unsigned* counters = static_cast<unsigned*>(workspace);
   float* partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + decode_counter_bytes(B, nkv, n_hgrp));
   return DecodeParams{q, k_cache, v_cache, kv_lens, B, nh, nkv, hd, cap, split, (cap + split - 1) / split,
-                      partials, out, err, counters, n_hgrp, kv_split == 0, 0};
+                      partials, out, err, counters, n_hgrp, kv_split == 0, 0, nullptr, 0, 0, 0};
 }
 
 }  // namespace gqa
@@ -252,6 +252,47 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   const int n = gqa::launch_decode(p, dtype == GQA_BF16, s, &e);
+  return launch_status(e, n);
+}
+
+int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                          const int32_t* block_table, const int32_t* kv_lens, int B, int n_heads,
+                          int n_kv_heads, int head_dim, int page_size, int max_pages, int num_pages,
+                          int kv_split, void* out, void* workspace, size_t workspace_bytes, int dtype,
+                          void* stream) {
+  if (dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || n_heads <= 0 || n_kv_heads <= 0 || page_size <= 0 || max_pages <= 0 || num_pages <= 0)
+    return GQA_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads != 0 || page_size % 64) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED_SHAPE;
+  const long long cap = (long long)max_pages * page_size;
+  // every cache row index (page, KV head, row) stays a 32-bit int
+  if (cap >= (1ll << 31) || (long long)num_pages * n_kv_heads * page_size >= (1ll << 31) ||
+      (long long)B * max_pages >= (1ll << 31) || B > 65535 || n_kv_heads > 65535)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;
+  if (kv_split > 0 && (cap + kv_split - 1) / kv_split > kMaxSplits) return GQA_ERR_INVALID_ARG;
+  if (B == 0) return GQA_OK;
+  if (!q || !k_pages || !v_pages || !block_table || !kv_lens || !out || !workspace) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out) ||
+      !aligned16(workspace) || !aligned4(kv_lens) || !aligned4(block_table))
+    return GQA_ERR_MISALIGNED;
+  const size_t need = gqa_attn_decode_workspace_size(B, n_heads, n_kv_heads, head_dim, (int)cap, kv_split);
+  if (need == 0) return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (workspace_bytes < need) return GQA_ERR_WORKSPACE_TOO_SMALL;
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (!d) return st;
+
+  gqa::DecodeParams p = gqa::decode_params(q, k_pages, v_pages, kv_lens, B, n_heads, n_kv_heads, head_dim,
+                                           (int)cap, kv_split, out, workspace, d->err);
+  p.block_table = block_table;
+  p.page_size = page_size;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  const int n = gqa::launch_decode(p, true, s, &e);
   return launch_status(e, n);
 }
 

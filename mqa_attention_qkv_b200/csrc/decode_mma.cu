@@ -152,15 +152,35 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
     if (lane == 0) {
       tc::prefetch_tmap(&tmk);
       tc::prefetch_tmap(&tmv);
-      const int row0 = (b * p.nkv + j) * p.cap + k_lo;
+      // cache row of a tile's first key: contiguous [B, nkv, cap, hd], or through
+      // the block table (a 64-key tile never crosses a page: pages are
+      // multiples of 64 keys and tiles start at multiples of 64); the table
+      // entry is re-read only when the page changes
+      int cur_page = -1, page_base = 0;
+      auto tile_row = [&](int key) {
+        if (!p.block_table) return (b * p.nkv + j) * p.cap + key;
+        const int lp = key / p.page_size;
+        if (lp != cur_page) {
+          cur_page = lp;
+          const int pg = __ldg(p.block_table + (size_t)b * p.max_pages + lp);
+          if (pg < 0 || pg >= p.num_pages) {
+            raise_error(err, GQA_DEVERR_PAGE_RANGE);
+            page_base = p.num_pages * p.nkv * p.page_size;   // past the end: the copy reads zeros
+          } else {
+            page_base = (pg * p.nkv + j) * p.page_size;
+          }
+        }
+        return page_base + (key - cur_page * p.page_size);
+      };
       for (int t = 0; t < n_t; ++t) {
         const int s = t % C::STAGES;
+        const int row = tile_row(k_lo + t * KT);
         if (!mbar_wait(&bars->empty[s], ((t / C::STAGES) & 1) ^ 1, err)) break;
         mbar_arrive_expect_tx(&bars->full[s], C::STAGE_BYTES);
         uint8_t* kt = smem + s * C::STAGE_BYTES;
         for (int bx = 0; bx < C::NBOX; ++bx) {
-          tc::tma_load_2d(kt + bx * C::BOX_BYTES, &tmk, bx * 64, row0 + t * KT, &bars->full[s]);
-          tc::tma_load_2d(kt + C::TILE_BYTES + bx * C::BOX_BYTES, &tmv, bx * 64, row0 + t * KT, &bars->full[s]);
+          tc::tma_load_2d(kt + bx * C::BOX_BYTES, &tmk, bx * 64, row, &bars->full[s]);
+          tc::tma_load_2d(kt + C::TILE_BYTES + bx * C::BOX_BYTES, &tmv, bx * 64, row, &bars->full[s]);
         }
       }
       // every issued load has landed before the block may exit
@@ -500,7 +520,7 @@ cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
       e != cudaSuccess)
     return e;
   CUtensorMap tk, tv;
-  const uint64_t rows = (uint64_t)p.B * p.nkv * p.cap;
+  const uint64_t rows = p.block_table ? (uint64_t)p.num_pages * p.nkv * p.page_size : (uint64_t)p.B * p.nkv * p.cap;
   if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
   const dim3 grid((unsigned)(p.n_split * p.n_hgrp), p.nkv, p.B);
@@ -549,7 +569,7 @@ cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
 }
 
 int launch_decode(const DecodeParams& p0, bool bf16, cudaStream_t st, cudaError_t* err) {
-  if (bf16 && p0.auto_split) {
+  if (bf16 && p0.auto_split && !p0.block_table) {
     // large batches with large head groups: tcgen05 tiles (mma.sync would be
     // tensor-bound there)
     const int nc = decode_tc_splits(p0);

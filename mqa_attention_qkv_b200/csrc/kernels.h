@@ -47,6 +47,11 @@ struct DecodeParams {
   int n_hgrp;             // groups of <= 16 query heads per KV head
   int auto_split;         // the caller left the split to the library
   int cluster;            // set by launch_decode: splits merged inside a thread-block cluster
+  // paged cache (block_table != nullptr): k_cache/v_cache are pages
+  // [num_pages, nkv, page_size, hd]; key t of sequence b is row t % page_size
+  // of page block_table[b * max_pages + t / page_size]; cap = max_pages * page_size
+  const int32_t* block_table;
+  int page_size, max_pages, num_pages;
 };
 
 // Most key splits per sequence: the tensor-core decode's final merge keeps

@@ -116,6 +116,28 @@ def test_meanpool_rejects(kw, code):
     assert _meanpool(**kw) == code
 
 
+def _paged(**kw):
+    a = dict(q=P, k=P, v=P, table=P, lens=P, B=2, nh=8, nkv=2, hd=128, ps=64, maxp=4, nump=8, split=0, out=P,
+             ws=P, ws_bytes=1 << 30, dtype=1, stream=None)
+    a.update(kw)
+    return gqa.lib().gqa_attn_decode_paged(a["q"], a["k"], a["v"], a["table"], a["lens"], a["B"], a["nh"],
+                                           a["nkv"], a["hd"], a["ps"], a["maxp"], a["nump"], a["split"], a["out"],
+                                           a["ws"], a["ws_bytes"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(table=None), INVALID), (dict(lens=None), INVALID), (dict(k=None), INVALID), (dict(ws=None), INVALID),
+    (dict(ps=0), INVALID), (dict(ps=96), INVALID), (dict(maxp=0), INVALID), (dict(nump=0), INVALID),
+    (dict(nh=6, nkv=4), INVALID), (dict(split=100), INVALID), (dict(split=-64), INVALID),
+    (dict(hd=32), SHAPE), (dict(hd=96), SHAPE), (dict(dtype=0), DTYPE),
+    (dict(ps=1 << 20, maxp=1 << 12), SHAPE),          # 2^32 keys a sequence
+    (dict(ps=1 << 16, nump=1 << 15), SHAPE),          # 2^32 cache rows
+    (dict(ws_bytes=16), WS), (dict(table=P + 2), MISALIGNED), (dict(v=MIS), MISALIGNED),
+])
+def test_paged_decode_rejects(kw, code):
+    assert _paged(**kw) == code
+
+
 def test_empty_inputs_are_noops():
     # B == 0 or S == 0 returns OK without launching (pointers may then be NULL)
     assert _qkv(B=0, x=None, w=None, pos=None, q=None, k=None, v=None) == 0
@@ -123,6 +145,7 @@ def test_empty_inputs_are_noops():
     assert _prefill(B=0, q=None) == 0
     assert _prefill(S=0) == 0
     assert _decode(B=0, q=None, ws=None) == 0
+    assert _paged(B=0, q=None, table=None, ws=None) == 0
 
 
 def test_workspace_size_query():
@@ -147,3 +170,4 @@ def test_valid_call_without_gpu_reports_no_device():
     assert _prefill() in (NODEV, ARCH)
     assert _decode() in (NODEV, ARCH)
     assert _meanpool() in (NODEV, ARCH)
+    assert _paged() in (NODEV, ARCH)

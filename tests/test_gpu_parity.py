@@ -310,6 +310,101 @@ def test_decode_long_cache_uses_workspace_splits():
     gate(host(run_decode(q, kc, vc, lens, nh, dtype)), want, dtype, "long-cache decode")
 
 
+def paged_inputs(B, nh, nkv, hd, ps, lens, seed, extra_pages=5):
+    """The seeded contiguous decode cache cut into pages of ``ps`` keys, the
+    pages shuffled into a pool with ``extra_pages`` NaN-filled pages that no
+    table names; table entries past a sequence's last page are -1."""
+    cap = -(-max(int(lens.max()), 1) // ps) * ps
+    max_pages = cap // ps
+    q = W.normal_tensor((B, nh, hd), seed, 0, "bf16")
+    kc = nan_padded(B, nkv, cap, hd, lens, seed, 1, "bf16")
+    vc = nan_padded(B, nkv, cap, hd, lens, seed, 2, "bf16")
+    n_pool = B * max_pages + extra_pages
+    perm = np.random.default_rng(seed + 1000).permutation(n_pool)      # logical page i -> physical perm[i]
+
+    def cut(c):
+        logical = c.store.reshape(B, nkv, max_pages, ps, hd).transpose(0, 2, 1, 3, 4).reshape(-1, nkv, ps, hd)
+        pool = np.full((n_pool, nkv, ps, hd), SENTINEL["bf16"], dtype=np.uint16)
+        pool[perm[:B * max_pages]] = logical
+        return W.Tensor(pool, "bf16")
+
+    table = perm[:B * max_pages].reshape(B, max_pages).astype(np.int32)
+    for b in range(B):
+        table[b, -(-int(lens[b]) // ps):] = -1
+    return q, kc, vc, cut(kc), cut(vc), table, cap
+
+
+def run_decode_paged(q, kp, vp, table, lens, nh, kv_split=0):
+    B, _, hd = q.shape
+    nkv, ps = kp.shape[1], kp.shape[2]
+    cap = table.shape[1] * ps
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap, kv_split) // 4 + 1,
+                     dtype=torch.float32, device="cuda")
+    out = torch.empty((B, nh, hd), dtype=torch.bfloat16, device="cuda")
+    gqa.gqa_attn_decode_paged(dev(q), dev(kp), dev(vp), dev_i32(table), dev_i32(lens), out, ws, kv_split=kv_split)
+    return out
+
+
+@pytest.mark.parametrize("hd,g,nkv,ps", [(128, 8, 1, 64), (128, 4, 2, 128), (64, 48, 1, 64), (64, 2, 4, 256),
+                                         (128, 32, 1, 192)])
+def test_paged_decode_parity(hd, g, nkv, ps):
+    """Decode over shuffled pages against the oracle's paged decode, for the
+    automatic split and two fixed ones, and bit for bit against the same
+    cache laid out contiguously (only the address of each tile differs)."""
+    nh = g * nkv
+    lens = np.array([1, 63, 64, 65, 300, 1000, 0, 513, 2000], dtype=np.int32)
+    B = len(lens)
+    q, kc, vc, kp, vp, table, cap = paged_inputs(B, nh, nkv, hd, ps, lens, 60 + hd + ps)
+    want = ref.paged_decode_attention(q.f64, kp.f64, vp.f64, table, lens, ps)
+    gqa.gqa_device_error()
+    for split in (0, 64, 192):
+        got_t = run_decode_paged(q, kp, vp, table, lens, nh, kv_split=split)
+        got = host(got_t)
+        assert np.all(got[6] == 0)
+        keep = lens > 0
+        gate(got[keep], want[keep], "bf16", f"paged decode split={split}")
+        flat = run_decode(q, kc, vc, lens, nh, "bf16", kv_split=split)
+        np.testing.assert_array_equal(bits(got_t), bits(flat))
+    assert gqa.gqa_device_error() == 0
+
+
+def test_paged_decode_shared_pages():
+    """Two sequences whose tables name the same physical pages (a shared
+    prompt prefix) attend over the same keys: identical queries give
+    identical outputs."""
+    hd, nh, nkv, ps = 128, 16, 2, 64
+    lens = np.array([700, 700], dtype=np.int32)
+    q, kc, vc, kp, vp, table, cap = paged_inputs(2, nh, nkv, hd, ps, lens, 71)
+    table[1] = table[0]
+    qs = W.Tensor(np.ascontiguousarray(np.broadcast_to(q.store[:1], q.store.shape)), "bf16")
+    out = run_decode_paged(qs, kp, vp, table, lens, nh)
+    got = bits(out)
+    np.testing.assert_array_equal(got[0], got[1])
+    want = ref.paged_decode_attention(qs.f64, kp.f64, vp.f64, table, lens, ps)
+    gate(host(out), want, "bf16", "shared pages")
+
+
+def test_paged_decode_bad_table_entry_flags_and_reads_zeros():
+    """A table entry outside the page pool raises the page-range bit; its
+    keys read as zeros (score 0, value 0), which the oracle reproduces with a
+    zero page in that slot."""
+    hd, nh, nkv, ps = 64, 8, 1, 64
+    lens = np.array([256, 130], dtype=np.int32)
+    q, kc, vc, kp, vp, table, cap = paged_inputs(2, nh, nkv, hd, ps, lens, 72)
+    n_pool = kp.shape[0]
+    bad = table.copy()
+    bad[0, 1] = n_pool + 3
+    bad[1, 0] = -7
+    gqa.gqa_device_error()
+    got = host(run_decode_paged(q, kp, vp, bad, lens, nh))
+    assert gqa.gqa_device_error() & 8
+    zk = np.concatenate([kp.f64, np.zeros((1,) + kp.shape[1:])])
+    zv = np.concatenate([vp.f64, np.zeros((1,) + vp.shape[1:])])
+    zt = np.where((bad < 0) | (bad >= n_pool), n_pool, bad)      # bad entries -> the zero page
+    want = ref.paged_decode_attention(q.f64, zk, zv, zt, lens, ps)
+    gate(got, want, "bf16", "zero-read pages")
+
+
 def test_decode_zero_and_clamped_lengths():
     dtype, hd, nh, nkv, cap = "bf16", 64, 4, 2, 128
     lens = np.array([0, 128, 5], dtype=np.int32)

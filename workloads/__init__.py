@@ -66,7 +66,8 @@ class Tensor:
     @property
     def f64(self) -> np.ndarray:
         if self.dtype == "bf16":
-            return bf16_to_f32(self.store).astype(np.float64)
+            with np.errstate(invalid="ignore"):          # NaN sentinels in padded caches
+                return bf16_to_f32(self.store).astype(np.float64)
         return self.store.astype(np.float64)
 
     @property
