@@ -126,6 +126,24 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The largest of the replicas' values (each measured on its own device
+    clock): the slowest replica sets the job's time."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: float, world: int, steps: int, ms_total: float) -> float:
+    """Units that all replicas processed, per second of the (max-over-ranks)
+    timed region."""
+    return units_per_step_per_rank * world * steps / (ms_total / 1e3)
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -194,13 +212,6 @@ def run_ours(args):
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     # warm-up
     for i in range(args.warmup):
         step(sets[i % N_ROT])
@@ -220,13 +231,13 @@ def run_ours(args):
     barrier()
     launches = gqa.gqa_launch_count() - n0
     clk = clocks.stop()
-    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     per_kernel = {n: [evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)]
                   for k, n in enumerate(names)}
 
     tokens_per_step = B * S + B
     ms_step = ms_total / args.steps
-    value = tokens_per_step * world * args.steps / (ms_total / 1e3)
+    value = whole_job_rate(tokens_per_step, world, args.steps, ms_total)
 
     # algorithmic work per launch
     peaks, peak_src = load_peaks()
@@ -286,10 +297,10 @@ def run_ours(args):
             e2e_step(i)
         b_.record(stream)
         barrier()
-        ms_e2e = max_over_ranks(a.elapsed_time(b_))
+        ms_e2e = max_over_ranks(a.elapsed_time(b_), world, dev)
         h2d = hx[0].numel() * 2 + hxd[0].numel() * 2 + hpos.numel() * 4
         d2h = ho.numel() * 2 + hod.numel() * 2
-        e2e = {"value": round(tokens_per_step * world * args.steps / (ms_e2e / 1e3), 1), "unit": "tokens/s",
+        e2e = {"value": round(whole_job_rate(tokens_per_step, world, args.steps, ms_e2e), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(ms_e2e / args.steps, 4)}
 
