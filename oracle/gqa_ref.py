@@ -25,6 +25,11 @@ Sources (page title, then section):
   stored non-contiguously, in fixed-size pages that a block table maps to each
   sequence (the paged decode here keeps the tensor cores by making pages whole
   key tiles).
+* "FlashAttention-3" (together.ai summary), section "残る最適化と今後の統合":
+  the paper adds variable-length sequences.  Read as the packed layout of
+  the FlashAttention library: the sequences of a batch are concatenated
+  along the token axis and delimited by cumulative offsets (cu_seqlens), so
+  that no padding is stored or computed.
 * "MHA -> GQA: 提升 LLM 推理效率", section 4.3 (剪枝训练): the new KV projection
   of each group of heads is initialised by mean pooling the group's
   projections (the offline MHA -> GQA weight transform).
@@ -49,6 +54,7 @@ __all__ = [
     "fused_projection", "split_qkv", "rope_inv_freq", "apply_rope",
     "qkv_rope_project", "kv_head_of", "softmax", "attend_row",
     "prefill_attention", "decode_attention", "default_q_positions", "round_bf16",
+    "varlen_prefill_attention", "meanpool_kv_projection", "gather_pages", "paged_decode_attention",
 ]
 
 
@@ -246,6 +252,39 @@ def decode_attention(q, k_cache, v_cache, kv_lens, pairs=None):
         out[i], _ = attend_row(q[b, h], K, V)
     if pairs is None:
         return out.reshape(B, nh, hd)
+    return out
+
+
+def varlen_prefill_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, causal):
+    """Prefill attention over packed variable-length sequences.
+
+    q ``[Tq, nh, hd]``, k and v ``[Tk, nkv, hd]``; sequence i owns query rows
+    ``[cu_seqlens_q[i], cu_seqlens_q[i+1])`` and key rows
+    ``[cu_seqlens_k[i], cu_seqlens_k[i+1])`` and attends to its own keys only.
+    With Sq queries over Sk keys, query s of a sequence sits at position
+    Sk - Sq + s (bottom-right alignment, as in the padded prefill) and, when
+    causal, sees the keys at positions <= its own.  Returns O ``[Tq, nh, hd]``;
+    a query that sees no key gets a zero row."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64)
+    assert cq.shape == ck.shape and cq[0] == 0 and ck[0] == 0
+    assert np.all(np.diff(cq) >= 0) and np.all(np.diff(ck) >= 0)
+    Tq, nh, hd = q.shape
+    nkv = k.shape[1]
+    assert cq[-1] == Tq and ck[-1] == k.shape[0] == v.shape[0]
+    out = np.zeros((Tq, nh, hd))
+    for i in range(len(cq) - 1):
+        Sq, Sk = int(cq[i + 1] - cq[i]), int(ck[i + 1] - ck[i])
+        for s in range(Sq):
+            n_vis = min(Sk, Sk - Sq + s + 1) if causal else Sk
+            for h in range(nh):
+                j = kv_head_of(h, nh, nkv)
+                keys = k[ck[i]:ck[i + 1], j]
+                vals = v[ck[i]:ck[i + 1], j]
+                out[cq[i] + s, h], _ = attend_row(q[cq[i] + s, h], keys, vals, max(n_vis, 0))
     return out
 
 

@@ -715,3 +715,128 @@ def test_planted_ignored_block_table_is_caught(monkeypatch):
     monkeypatch.setattr(ref, "gather_pages", ignore_table)
     assert _fails(check_paged_page_order_does_not_matter)
 
+
+
+# --------------------------------------------------------------------------
+# packed variable-length prefill (FlashAttention-3 summary, section
+# "残る最適化と今後の統合": variable-length sequences; cu_seqlens offsets)
+# --------------------------------------------------------------------------
+def varlen_setup(seed=61, nh=4, nkv=2, hd=4, q_lens=(3, 0, 5, 1, 4), k_lens=(5, 2, 5, 1, 9)):
+    r = rng(seed)
+    cq = np.concatenate([[0], np.cumsum(q_lens)])
+    ck = np.concatenate([[0], np.cumsum(k_lens)])
+    q = r.normal(size=(cq[-1], nh, hd))
+    k = r.normal(size=(ck[-1], nkv, hd))
+    v = r.normal(size=(ck[-1], nkv, hd))
+    return q, k, v, cq, ck
+
+
+def brute_varlen(q, k, v, cq, ck, causal):
+    """Literal loops: for each packed query row, find its sequence by
+    scanning the offsets, then softmax over that sequence's visible keys."""
+    Tq, nh, hd = q.shape
+    nkv = k.shape[1]
+    out = np.zeros((Tq, nh, hd))
+    for r_ in range(Tq):
+        i = max(n for n in range(len(cq) - 1) if cq[n] <= r_ < cq[n + 1])
+        Sq, Sk = cq[i + 1] - cq[i], ck[i + 1] - ck[i]
+        pos = Sk - Sq + (r_ - cq[i])
+        for h in range(nh):
+            j = h // (nh // nkv)
+            keys = [t for t in range(Sk) if not causal or t <= pos]
+            if not keys:
+                continue
+            sc = [sum(float(q[r_, h, d]) * float(k[ck[i] + t, j, d]) for d in range(hd)) / math.sqrt(hd) for t in keys]
+            m = max(sc)
+            w = [math.exp(x - m) for x in sc]
+            out[r_, h] = sum(wi * v[ck[i] + t, j] for wi, t in zip(w, keys)) / sum(w)
+    return out
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_varlen_prefill_brute_force(causal):
+    q, k, v, cq, ck = varlen_setup()
+    np.testing.assert_allclose(ref.varlen_prefill_attention(q, k, v, cq, ck, causal),
+                               brute_varlen(q, k, v, cq, ck, causal), rtol=0, atol=1e-12)
+
+
+def check_varlen_block_diagonal_mask(causal=True):
+    """The whole packed batch as ONE attention whose mask is block-diagonal
+    (a query sees only its own sequence's keys) and, when causal, lower
+    triangular within a block from the bottom-right corner."""
+    q, k, v, cq, ck = varlen_setup(seed=62)
+    Tq, nh, hd = q.shape
+    nkv = k.shape[1]
+    seg_q = np.searchsorted(cq, np.arange(Tq), side="right") - 1
+    seg_k = np.searchsorted(ck, np.arange(k.shape[0]), side="right") - 1
+    rel_q = np.arange(Tq) - cq[seg_q] + (ck[seg_q + 1] - ck[seg_q]) - (cq[seg_q + 1] - cq[seg_q])
+    rel_k = np.arange(k.shape[0]) - ck[seg_k]
+    mask = seg_q[:, None] == seg_k[None, :]
+    if causal:
+        mask &= rel_k[None, :] <= rel_q[:, None]
+    want = np.zeros((Tq, nh, hd))
+    for h in range(nh):
+        j = h // (nh // nkv)
+        s = np.where(mask, q[:, h] @ k[:, j].T / np.sqrt(hd), -np.inf)
+        has = mask.any(axis=1)
+        e = np.exp(s - np.where(has, s.max(axis=1), 0.0)[:, None])
+        want[has, h] = (e[has] / e[has].sum(axis=1, keepdims=True)) @ v[:, j]
+    np.testing.assert_allclose(ref.varlen_prefill_attention(q, k, v, cq, ck, causal), want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_varlen_prefill_is_block_diagonal_attention(causal):
+    check_varlen_block_diagonal_mask(causal)
+
+
+def test_varlen_prefill_equals_padded_prefill():
+    """Packing and padding give the same rows: the padded prefill over
+    [B, nh, S_max, hd] queries with kv_lens and bottom-right positions."""
+    q, k, v, cq, ck = varlen_setup(seed=63, q_lens=(3, 5, 1, 4), k_lens=(5, 5, 1, 9))
+    B = len(cq) - 1
+    nh, hd = q.shape[1], q.shape[2]
+    nkv = k.shape[1]
+    S, cap = int(np.diff(cq).max()), int(np.diff(ck).max())
+    qp = np.zeros((B, nh, S, hd))
+    kp, vp = np.zeros((B, nkv, cap, hd)), np.zeros((B, nkv, cap, hd))
+    pos = np.zeros((B, S), dtype=np.int64)
+    for b in range(B):
+        Sq, Sk = cq[b + 1] - cq[b], ck[b + 1] - ck[b]
+        qp[b, :, :Sq] = q[cq[b]:cq[b + 1]].transpose(1, 0, 2)
+        kp[b, :, :Sk] = k[ck[b]:ck[b + 1]].transpose(1, 0, 2)
+        vp[b, :, :Sk] = v[ck[b]:ck[b + 1]].transpose(1, 0, 2)
+        pos[b] = Sk - Sq + np.arange(S)
+    padded = ref.prefill_attention(qp, kp, vp, np.diff(ck), True, q_positions=pos)
+    got = ref.varlen_prefill_attention(q, k, v, cq, ck, True)
+    for b in range(B):
+        np.testing.assert_allclose(got[cq[b]:cq[b + 1]], padded[b, :cq[b + 1] - cq[b]], rtol=0, atol=1e-12)
+
+
+def test_varlen_prefill_special_cases():
+    q, k, v, cq, ck = varlen_setup(seed=64)
+    out = ref.varlen_prefill_attention(q, k, v, cq, ck, True)
+    # a query of the 1-key sequence (index 3) sees exactly its one value
+    nh, nkv = q.shape[1], k.shape[1]
+    for h in range(nh):
+        np.testing.assert_allclose(out[cq[3], h], v[ck[3], h // (nh // nkv)], rtol=0, atol=1e-15)
+    # a sequence with no keys gives zero rows
+    q2, k2, v2, cq2, ck2 = varlen_setup(seed=65, q_lens=(2, 3), k_lens=(0, 4))
+    o2 = ref.varlen_prefill_attention(q2, k2, v2, cq2, ck2, False)
+    assert np.all(o2[:2] == 0) and np.all(np.abs(o2[2:]) > 0)
+    # one sequence is the plain causal prefill
+    q3, k3, v3, cq3, ck3 = varlen_setup(seed=66, q_lens=(6,), k_lens=(6,))
+    plain = ref.prefill_attention(q3.transpose(1, 0, 2)[None], k3.transpose(1, 0, 2)[None],
+                                  v3.transpose(1, 0, 2)[None], np.array([6]), True)[0]
+    np.testing.assert_allclose(ref.varlen_prefill_attention(q3, k3, v3, cq3, ck3, True), plain, rtol=0, atol=1e-12)
+
+
+def test_planted_varlen_key_offset_is_caught(monkeypatch):
+    """Reading a sequence's keys one row late (an off-by-one in the key
+    offsets) fails the block-diagonal pin."""
+    orig = ref.varlen_prefill_attention
+
+    def shifted(q, k, v, cq, ck, causal):
+        ck2 = np.minimum(np.asarray(ck) + np.r_[0, np.ones(len(ck) - 2, dtype=int), 0], ck[-1])
+        return orig(q, k, v, cq, ck2, causal)
+    monkeypatch.setattr(ref, "varlen_prefill_attention", shifted)
+    assert _fails(check_varlen_block_diagonal_mask)
