@@ -20,7 +20,9 @@ Sources (page title, then section):
   softmax(QK^T)V computed here.
 * custom-op overhead gist (``overhead.py``): ``forward(positions,
   hidden_states)`` applies a position-dependent step to q and k only, after
-  the fused projection.
+  the fused projection; the attention output (heads concatenated per token)
+  then goes through the output projection, and the decoder layer adds the
+  residual stream to it.
 * "MHA -> GQA: 提升 LLM 推理效率", section 3.2: a PagedAttention KV cache is
   stored non-contiguously, in fixed-size pages that a block table maps to each
   sequence (the paged decode here keeps the tensor cores by making pages whole
@@ -54,7 +56,7 @@ __all__ = [
     "fused_projection", "split_qkv", "rope_inv_freq", "apply_rope",
     "qkv_rope_project", "kv_head_of", "softmax", "attend_row",
     "prefill_attention", "decode_attention", "default_q_positions", "round_bf16",
-    "varlen_prefill_attention", "meanpool_kv_projection", "gather_pages", "paged_decode_attention",
+    "varlen_prefill_attention", "output_projection", "meanpool_kv_projection", "gather_pages", "paged_decode_attention",
 ]
 
 
@@ -286,6 +288,19 @@ def varlen_prefill_attention(q, k, v, cu_seqlens_q, cu_seqlens_k, causal):
                 vals = v[ck[i]:ck[i + 1], j]
                 out[cq[i] + s, h], _ = attend_row(q[cq[i] + s, h], keys, vals, max(n_vis, 0))
     return out
+
+
+def output_projection(attn_out, w_o, residual=None):
+    """The attention layer's last step: each token's head outputs
+    concatenated in head order (``[..., nh, hd]`` -> ``[..., nh*hd]``) times
+    W_o^T (``[hidden, nh*hd]``, nn.Linear layout, no bias), plus the residual
+    stream ``[..., hidden]`` when one is given."""
+    o = np.asarray(attn_out, dtype=np.float64)
+    w = np.asarray(w_o, dtype=np.float64)
+    y = o.reshape(o.shape[:-2] + (o.shape[-2] * o.shape[-1],)) @ w.T
+    if residual is not None:
+        y = y + np.asarray(residual, dtype=np.float64)
+    return y
 
 
 def meanpool_kv_projection(w_qkv_mha: np.ndarray, n_heads: int, n_kv_heads: int,

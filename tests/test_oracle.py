@@ -840,3 +840,79 @@ def test_planted_varlen_key_offset_is_caught(monkeypatch):
         return orig(q, k, v, cq, ck2, causal)
     monkeypatch.setattr(ref, "varlen_prefill_attention", shifted)
     assert _fails(check_varlen_block_diagonal_mask)
+
+
+# --------------------------------------------------------------------------
+# output projection (custom-op overhead gist: LlamaAttention ends with the
+# output projection; the decoder layer adds the residual)
+# --------------------------------------------------------------------------
+def test_output_projection_brute_force():
+    r = rng(71)
+    T, nh, hd, D = 3, 4, 2, 5
+    o, w, res = r.normal(size=(T, nh, hd)), r.normal(size=(D, nh * hd)), r.normal(size=(T, D))
+    want = np.zeros((T, D))
+    for t in range(T):
+        for n in range(D):
+            acc = float(res[t, n])
+            for h in range(nh):
+                for d in range(hd):
+                    acc += float(o[t, h, d]) * float(w[n, h * hd + d])
+            want[t, n] = acc
+    np.testing.assert_allclose(ref.output_projection(o, w, res), want, rtol=0, atol=1e-12)
+
+
+def check_output_projection_is_a_sum_over_heads():
+    """The head-split form a fused epilogue computes: each head's output
+    times its own hd-column slice of W_o, summed over heads."""
+    r = rng(72)
+    B, S, nh, hd, D = 2, 3, 4, 8, 16
+    o, w = r.normal(size=(B, S, nh, hd)), r.normal(size=(D, nh * hd))
+    want = sum(o[:, :, h] @ w[:, h * hd:(h + 1) * hd].T for h in range(nh))
+    np.testing.assert_allclose(ref.output_projection(o, w), want, rtol=0, atol=1e-12)
+
+
+def test_output_projection_is_a_sum_over_heads():
+    check_output_projection_is_a_sum_over_heads()
+
+
+def test_output_projection_zero_weight_passes_the_residual():
+    """The gist initialises its projections to zero: the layer then returns
+    the residual stream unchanged."""
+    r = rng(73)
+    res = r.normal(size=(2, 3, 12))
+    np.testing.assert_array_equal(ref.output_projection(r.normal(size=(2, 3, 3, 4)), np.zeros((12, 12)), res), res)
+
+
+def test_layer_prefill_then_decode_equals_one_prefill():
+    """The whole attention layer (projection, RoPE, attention, output
+    projection): a prompt's prefill followed by decode steps gives, token by
+    token, the rows of one causal prefill over all the tokens."""
+    r = rng(74)
+    D, nh, nkv, hd, P, T = 16, 4, 2, 4, 5, 3
+    x = r.normal(size=(1, P + T, D))
+    w = r.normal(size=((nh + 2 * nkv) * hd, D)) * 0.3
+    wo = r.normal(size=(D, nh * hd)) * 0.3
+    cap = P + T
+    z = np.zeros((1, nkv, cap, hd))
+    pos_all = np.arange(P + T)[None]
+    q, kc, vc = ref.qkv_rope_project(x, w, pos_all, nh, nkv, hd, 1e4, z, z)
+    full = ref.output_projection(ref.prefill_attention(q, kc, vc, np.array([P + T]), True), wo, x)
+    q, kc, vc = ref.qkv_rope_project(x[:, :P], w, pos_all[:, :P], nh, nkv, hd, 1e4, z, z)
+    rows = [ref.output_projection(ref.prefill_attention(q, kc, vc, np.array([P]), True), wo, x[:, :P])]
+    for t in range(P, P + T):
+        q, kc, vc = ref.qkv_rope_project(x[:, t:t + 1], w, np.array([[t]]), nh, nkv, hd, 1e4, kc, vc)
+        o = ref.decode_attention(q[:, :, 0], kc, vc, np.array([t + 1]))
+        rows.append(ref.output_projection(o[:, None], wo, x[:, t:t + 1]))
+    np.testing.assert_allclose(np.concatenate(rows, axis=1), full, rtol=0, atol=1e-12)
+
+
+def test_planted_head_major_concat_is_caught(monkeypatch):
+    """Concatenating as [hd, nh] (channel-major) instead of head order fails
+    the head-split pin."""
+    orig = ref.output_projection
+
+    def channel_major(attn_out, w_o, residual=None):
+        o = np.asarray(attn_out)
+        return orig(np.swapaxes(o, -1, -2).reshape(o.shape), w_o, residual)
+    monkeypatch.setattr(ref, "output_projection", channel_major)
+    assert _fails(check_output_projection_is_a_sum_over_heads)
