@@ -34,6 +34,11 @@
  *   documented per call and recorded in a device error word that
  *   gqa_device_error() reads.
  * - head_dim must be 32, 64 or 128; B == 0 or S == 0 is a valid no-op.
+ * - Size limits (GQA_ERR_UNSUPPORTED_SHAPE beyond them): every tensor below
+ *   2^40 elements; B and n_heads (prefill) or n_kv_heads (decode) at most
+ *   65535; fewer than 2^31 cache rows (B * n_kv_heads * cache_cap, or
+ *   num_pages * n_kv_heads * page_size for a paged cache), query rows
+ *   (B * n_heads * S) and tokens (B * S).
  * - Runs only on compute capability 10.0 devices (B200, sm_100a).
  */
 #ifndef GQA_B200_H

@@ -84,6 +84,9 @@ int auto_split(int B, int nkv, int n_hgrp, int cap) {
 }
 
 constexpr long long kMaxElems = 1ll << 40;
+// Rows of the tensor-map views ([B*nkv*cap, hd] caches, [B*nh*S, hd] queries)
+// are addressed with 32-bit coordinates and int row arithmetic.
+constexpr long long kMaxRows = 1ll << 31;
 
 }  // namespace
 
@@ -192,7 +195,8 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
   if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
   if (!hd_ok(head_dim)) return GQA_ERR_UNSUPPORTED_SHAPE;
   if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems ||
-      (long long)B * n_heads * S * head_dim > kMaxElems || B > 65535 || n_heads > 65535)
+      (long long)B * n_heads * S * head_dim > kMaxElems || B > 65535 || n_heads > 65535 ||
+      (long long)B * n_kv_heads * cache_cap >= kMaxRows || (long long)B * n_heads * S >= kMaxRows)
     return GQA_ERR_UNSUPPORTED_SHAPE;
   if (B == 0 || S == 0) return GQA_OK;
   if (!q || !k_cache || !v_cache || !kv_lens || !out) return GQA_ERR_INVALID_ARG;
@@ -234,7 +238,8 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
   if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;
   if (kv_split > 0 && (cache_cap + kv_split - 1) / kv_split > kMaxSplits) return GQA_ERR_INVALID_ARG;
   if (!hd_ok(head_dim)) return GQA_ERR_UNSUPPORTED_SHAPE;
-  if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems || B > 65535 || n_kv_heads > 65535)
+  if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems || B > 65535 || n_kv_heads > 65535 ||
+      (long long)B * n_kv_heads * cache_cap >= kMaxRows)
     return GQA_ERR_UNSUPPORTED_SHAPE;
   if (B == 0) return GQA_OK;
   if (!q || !k_cache || !v_cache || !kv_lens || !out || !workspace) return GQA_ERR_INVALID_ARG;
@@ -267,7 +272,7 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
   if (head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED_SHAPE;
   const long long cap = (long long)max_pages * page_size;
   // every cache row index (page, KV head, row) stays a 32-bit int
-  if (cap >= (1ll << 31) || (long long)num_pages * n_kv_heads * page_size >= (1ll << 31) ||
+  if (cap >= kMaxRows || (long long)num_pages * n_kv_heads * page_size >= kMaxRows ||
       (long long)B * max_pages >= (1ll << 31) || B > 65535 || n_kv_heads > 65535)
     return GQA_ERR_UNSUPPORTED_SHAPE;
   if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;

@@ -70,7 +70,8 @@ int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
   if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
   if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;
   if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED_SHAPE;
-  if ((long long)B * n_kv_heads * cache_cap * head_dim > (1ll << 40) || B > 65535 || n_kv_heads > 65535)
+  if ((long long)B * n_kv_heads * cache_cap * head_dim > (1ll << 40) || B > 65535 || n_kv_heads > 65535 ||
+      (long long)B * n_kv_heads * cache_cap >= (1ll << 31))   // 32-bit cache row coordinates
     return GQA_ERR_UNSUPPORTED_SHAPE;
   if (B == 0) return GQA_OK;
   if (!q || !k_cache || !v_cache || !kv_lens || !out) return GQA_ERR_INVALID_ARG;

@@ -85,6 +85,8 @@ def test_qkv_rejects(kw, code):
     (dict(q=None), INVALID), (dict(lens=None), INVALID), (dict(out=None), INVALID),
     (dict(nh=3, nkv=2), INVALID), (dict(cap=0), INVALID), (dict(hd=16), SHAPE),
     (dict(dtype=-1), DTYPE), (dict(out=MIS), MISALIGNED), (dict(qpos=P + 1), MISALIGNED),
+    (dict(B=2, nkv=2, cap=1 << 29), SHAPE),             # 2^31 cache rows
+    (dict(B=1, nh=4, nkv=2, S=1 << 29), SHAPE),         # 2^31 query rows
 ])
 def test_prefill_rejects(kw, code):
     assert _prefill(**kw) == code
@@ -94,6 +96,7 @@ def test_prefill_rejects(kw, code):
     (dict(ws=None), INVALID), (dict(lens=None), INVALID), (dict(split=100), INVALID),
     (dict(split=-64), INVALID), (dict(nh=4, nkv=3), INVALID), (dict(hd=48), SHAPE),
     (dict(ws_bytes=16), WS), (dict(ws=MIS), MISALIGNED), (dict(dtype=7), DTYPE),
+    (dict(B=2, nkv=2, nh=4, cap=1 << 29, split=1 << 21), SHAPE),   # 2^31 cache rows
 ])
 def test_decode_rejects(kw, code):
     assert _decode(**kw) == code
