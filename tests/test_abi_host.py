@@ -174,3 +174,29 @@ def test_valid_call_without_gpu_reports_no_device():
     assert _decode() in (NODEV, ARCH)
     assert _meanpool() in (NODEV, ARCH)
     assert _paged() in (NODEV, ARCH)
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    """No fallback: with the shared library absent every call raises."""
+    monkeypatch.setattr(gqa, "_LIB", None)
+    monkeypatch.setattr(gqa, "library_path", lambda: str(tmp_path / "libgqa_b200.so"))
+    with pytest.raises(ImportError):
+        gqa.lib()
+    with pytest.raises(ImportError):
+        gqa.gqa_attn_decode_workspace_size(1, 8, 1, 128, 64)
+    with pytest.raises(ImportError):
+        gqa.gqa_launch_count()
+
+
+def test_binding_rejects_host_tensors():
+    """Tensors must live on the GPU: host tensors are refused before any
+    library call."""
+    import torch
+    q = torch.zeros(2, 8, 64, dtype=torch.bfloat16)
+    kc = torch.zeros(2, 2, 64, 64, dtype=torch.bfloat16)
+    lens = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        gqa.gqa_attn_decode(q, kc, kc, lens, q.clone(), torch.zeros(1024, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        gqa.gqa_attn_decode_paged(q, kc, kc, torch.zeros(2, 1, dtype=torch.int32), lens, q.clone(),
+                                  torch.zeros(1024, dtype=torch.uint8))
