@@ -70,7 +70,9 @@ enum gqa_device_error_bits {
   GQA_DEVERR_POSITION_RANGE = 1,   /* a position outside [0, cache_cap): K/V row not written */
   GQA_DEVERR_KVLEN_RANGE = 2,      /* a kv_len above cache_cap (clamped) or below 0 (taken as 0) */
   GQA_DEVERR_WAIT_TIMEOUT = 4,     /* a pipeline wait gave up after its time limit */
-  GQA_DEVERR_PAGE_RANGE = 8        /* a block-table entry outside [0, num_pages): read as zeros */
+  GQA_DEVERR_PAGE_RANGE = 8,       /* a block-table entry outside [0, num_pages): read as zeros */
+  GQA_DEVERR_SEQLEN_RANGE = 16     /* packed offsets decreasing or past the tensors (clamped), or a
+                                      query run longer than max_seqlen_q (rows past it not written) */
 };
 
 /*
@@ -133,6 +135,41 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
                      const int32_t* q_positions, const int32_t* kv_lens,
                      int B, int S, int n_heads, int n_kv_heads, int head_dim,
                      int cache_cap, int causal, void* out, int dtype, void* stream);
+
+/*
+ * gqa_attn_prefill_varlen - gqa_attn_prefill over packed variable-length
+ * sequences.
+ *
+ * Source: "FlashAttention-3" (together.ai summary), section "残る最適化と今後の
+ * 統合": the paper adds variable-length sequences.  Read as the packed
+ * layout of the FlashAttention library: the sequences of a batch are
+ * concatenated along the token axis and delimited by cumulative offsets, so
+ * no padding is stored, read or computed.  Sequence b owns query rows
+ * [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key/value rows
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]) and attends to its own keys only.
+ * With Sq queries over Sk keys, query s sits at position Sk - Sq + s
+ * (bottom-right, as the padded call's default), and when causal sees the
+ * keys at positions <= its own; a query that sees no key gets a zero row.
+ *
+ *   q             [total_q, n_heads, head_dim] bf16 (token-major, packed)
+ *   k, v          [total_k, n_kv_heads, head_dim] bf16
+ *   cu_seqlens_q,
+ *   cu_seqlens_k  [B + 1] int32, non-decreasing, from 0 to total_q / total_k.
+ *                 Offsets outside the tensors, or decreasing, are clamped
+ *                 and raise GQA_DEVERR_SEQLEN_RANGE
+ *   max_seqlen_q  the longest query run (sizes the grid); a longer run raises
+ *                 GQA_DEVERR_SEQLEN_RANGE and its rows past the grid are not
+ *                 written
+ *   out           [total_q, n_heads, head_dim] bf16
+ *
+ * bf16 with head_dim 64 or 128 only.  total_q == 0, B == 0 or
+ * max_seqlen_q == 0 is a no-op; total_k may be 0 (zero rows).  Statuses as
+ * gqa_attn_prefill; asynchronous on `stream`.
+ */
+int gqa_attn_prefill_varlen(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, int B, int total_q, int total_k, int max_seqlen_q,
+                            int n_heads, int n_kv_heads, int head_dim, int causal, void* out, int dtype,
+                            void* stream);
 
 /*
  * gqa_attn_decode_workspace_size - bytes of device workspace gqa_attn_decode

@@ -17,7 +17,7 @@ __all__ = [
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
-    "EXPORTED_SYMBOLS",
+    "gqa_attn_prefill_varlen", "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -27,6 +27,7 @@ EXPORTED_SYMBOLS = (
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
+    "gqa_attn_prefill_varlen",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -75,6 +76,8 @@ def lib() -> ctypes.CDLL:
     L.gqa_attn_decode_paged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, vp, sz,
                                         i32, vp]
     L.gqa_attn_decode_paged.restype = i32
+    L.gqa_attn_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+    L.gqa_attn_prefill_varlen.restype = i32
     _LIB = L
     return L
 
@@ -186,6 +189,25 @@ def gqa_attn_decode(q, k_cache, v_cache, kv_lens, out, workspace, kv_split: int 
         _dtype_code(q), _stream(stream),
     )
     _check("gqa_attn_decode", lib().gqa_attn_decode(*args))
+
+
+def gqa_attn_prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool, out,
+                            stream=None) -> None:
+    """Packed variable-length prefill: q [total_q,nh,hd], k/v [total_k,nkv,hd]
+    bf16, cu_seqlens_q/k [B+1] int32 -> out [total_q,nh,hd] (include/gqa.h)."""
+    import torch
+    total_q, nh, hd = q.shape
+    total_k, nkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.shape[0] - 1
+    dt = q.dtype
+    args = (
+        _ptr(q, dt, name="q"), _ptr(k, dt, (total_k, nkv, hd), "k"), _ptr(v, dt, (total_k, nkv, hd), "v"),
+        _ptr(cu_seqlens_q, torch.int32, (B + 1,), "cu_seqlens_q"),
+        _ptr(cu_seqlens_k, torch.int32, (B + 1,), "cu_seqlens_k"),
+        B, total_q, total_k, int(max_seqlen_q), nh, nkv, hd, int(bool(causal)),
+        _ptr(out, dt, (total_q, nh, hd), "out"), _dtype_code(q), _stream(stream),
+    )
+    _check("gqa_attn_prefill_varlen", lib().gqa_attn_prefill_varlen(*args))
 
 
 def gqa_attn_decode_paged(q, k_pages, v_pages, block_table, kv_lens, out, workspace, kv_split: int = 0,

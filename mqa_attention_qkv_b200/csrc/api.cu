@@ -216,6 +216,34 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
   return launch_status(gqa::launch_prefill_simt(p, dtype == GQA_BF16, s));
 }
 
+int gqa_attn_prefill_varlen(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                            const int32_t* cu_seqlens_k, int B, int total_q, int total_k, int max_seqlen_q,
+                            int n_heads, int n_kv_heads, int head_dim, int causal, void* out, int dtype,
+                            void* stream) {
+  if (dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || n_heads <= 0 || n_kv_heads <= 0)
+    return GQA_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)total_q * n_heads * head_dim > kMaxElems || (long long)total_k * n_kv_heads * head_dim > kMaxElems ||
+      B > 65535 || n_heads > 65535 || (long long)B * n_heads * ((max_seqlen_q + 127) / 128) >= kMaxRows)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || total_q == 0 || max_seqlen_q == 0) return GQA_OK;
+  if (!q || !k || !v || !cu_seqlens_q || !cu_seqlens_k || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(cu_seqlens_q) ||
+      !aligned4(cu_seqlens_k))
+    return GQA_ERR_MISALIGNED;
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (!d) return st;
+
+  gqa::PrefillParams p{q, k, v, nullptr, nullptr, B, max_seqlen_q, n_heads, n_kv_heads, head_dim, total_k,
+                       causal ? 1 : 0, out, d->err, cu_seqlens_q, cu_seqlens_k, total_q};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (head_dim == 64) return launch_status(gqa::launch_prefill_pair(p, s));
+  return launch_status(gqa::launch_prefill_fa(p, s));
+}
+
 size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int head_dim,
                                       int cache_cap, int kv_split) {
   if (B < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0 || n_heads % n_kv_heads) return 0;

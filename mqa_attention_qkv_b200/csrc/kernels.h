@@ -30,6 +30,13 @@ struct PrefillParams {
   int B, S, nh, nkv, hd, cap, causal;
   void* out;              // [B, S, nh, hd]
   int* err;
+  // Packed variable-length mode (cu_q != nullptr): q and out [total_q, nh, hd],
+  // k_cache/v_cache [cap, nkv, hd] with cap = total_k; sequence b owns query
+  // rows [cu_q[b], cu_q[b+1]) and key rows [cu_k[b], cu_k[b+1]); S is the
+  // longest query run (it sizes the grid); q_pos and kv_lens are unused.
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int total_q;
 };
 
 struct DecodeParams {
@@ -124,6 +131,11 @@ bool make_tmap_bf16_2d(void* map, const void* base, uint64_t inner, uint64_t out
 // strides (bytes) of dims 1 and 2, box extents.  Zero fill outside the dims.
 bool make_tmap_bf16_3d(void* map, const void* base, const uint64_t dims[3], const uint64_t stride_bytes[2],
                        const uint32_t box[3]);
+// Packed token-major rows [tokens, heads, hd] as a 3-D map whose box is one
+// head's 64 columns of 128 consecutive tokens: the same swizzled 128 x 64
+// tile a 2-D box over head-major rows gives.  tokens == 0 is encoded as 1
+// (nothing may then be loaded).
+bool make_tmap_packed(void* map, const void* base, uint64_t tokens, int heads, int hd);
 
 // Shared by the C-ABI translation units (defined in api.cu).
 int device_check(int** err);  // GQA_OK, or the status for the current device

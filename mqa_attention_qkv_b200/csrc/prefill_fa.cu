@@ -22,6 +22,7 @@
 // when a row's max grows by more than 2^8 (the stale max is exact after the
 // final 1/l and keeps P <= 2^8).
 #include "kernels.h"
+#include "prefill_seq.cuh"
 #include "tc.cuh"
 
 namespace gqa {
@@ -68,7 +69,9 @@ struct Bars {
   int lim_max[2];
 };
 
-template <int HD, int POLY>
+// VARLEN: packed variable-length sequences (3-D tensor maps over
+// [tokens, heads, 64 columns]); otherwise the padded layout (2-D maps).
+template <int HD, int POLY, bool VARLEN>
 __global__ void __launch_bounds__(THREADS, 1)
 prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, PrefillParams p, int n_qt) {
@@ -89,11 +92,9 @@ prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   const int j = h / (p.nh / p.nkv);
   const int s_base = pr * 2 * BQ;   // first query row of tile 0
 
-  int kv_len = p.kv_lens[b];
-  if (kv_len > p.cap || kv_len < 0) {
-    if (threadIdx.x == 0) raise_error(err, GQA_DEVERR_KVLEN_RANGE);
-    kv_len = kv_len > p.cap ? p.cap : 0;
-  }
+  const SeqRange sq = prefill_seq(p, b, err);
+  if (VARLEN && s_base >= sq.S) return;   // a shorter sequence: no query in this pair (whole CTA)
+  const int kv_len = sq.kv_len;
 
   // softmax groups: warps 2-5 -> tile 0, warps 6-9 -> tile 1
   const int grp = warp >= 6 ? 1 : 0;
@@ -127,9 +128,9 @@ prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   __syncthreads();
   if (warp >= 2) {
     const int s = s_base + grp * BQ + row;
-    my_valid = s < p.S;
+    my_valid = s < sq.S;
     if (my_valid) {
-      const int pos = p.q_pos ? p.q_pos[(size_t)b * p.S + s] : kv_len - p.S + s;
+      const int pos = p.q_pos ? p.q_pos[(size_t)b * p.S + s] : kv_len - sq.S + s;
       my_lim = p.causal ? max(0, min(kv_len, pos + 1)) : kv_len;
       atomicMax(&bars->lim_max[grp], my_lim);
     }
@@ -142,7 +143,7 @@ prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   const int n1 = (bars->lim_max[1] + BKV - 1) / BKV;
   const int n_kv = max(n0, n1);
   const bool sanitize = n_kv > 0 && kv_len < n_kv * BKV;
-  const int kv_row0 = (b * p.nkv + j) * p.cap;
+  const int kv_row0 = VARLEN ? 0 : (b * p.nkv + j) * p.cap;
   uint8_t* sQ = smem + C::Q_OFF;
   uint8_t* sK = smem + C::K_OFF;
   uint8_t* sV = smem + C::V_OFF;
@@ -152,10 +153,14 @@ prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     bool ok = true;
     if (lane == 0 && n_kv > 0) {
       mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE);
-      const int qrow = (b * p.nh + h) * p.S + s_base;
+      const int qrow = VARLEN ? 0 : (b * p.nh + h) * p.S + s_base;
       for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < HD / 64; ++c)
-          tc::tma_load_2d(sQ + t * C::TILE + c * 16384, &tmq, c * 64, qrow + t * BQ, &bars->q_full);
+        for (int c = 0; c < HD / 64; ++c) {
+          if (VARLEN)
+            tc::tma_load_3d(sQ + t * C::TILE + c * 16384, &tmq, c * 64, h, sq.q0 + s_base + t * BQ, &bars->q_full);
+          else
+            tc::tma_load_2d(sQ + t * C::TILE + c * 16384, &tmq, c * 64, qrow + t * BQ, &bars->q_full);
+        }
       auto load = [&](int i, bool is_v) {
         const int S = is_v ? C::VS : C::KS;
         const int st = i % S;
@@ -164,8 +169,12 @@ prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         if (!mbar_wait(empty, ((i / S) & 1) ^ 1, err)) return false;
         mbar_arrive_expect_tx(full, C::TILE);
         uint8_t* dst = (is_v ? sV : sK) + st * C::TILE;
-        for (int c = 0; c < HD / 64; ++c)
-          tc::tma_load_2d(dst + c * 16384, is_v ? &tmv : &tmk, c * 64, kv_row0 + i * BKV, full);
+        for (int c = 0; c < HD / 64; ++c) {
+          if (VARLEN)
+            tc::tma_load_3d(dst + c * 16384, is_v ? &tmv : &tmk, c * 64, j, sq.k0 + i * BKV, full);
+          else
+            tc::tma_load_2d(dst + c * 16384, is_v ? &tmv : &tmk, c * 64, kv_row0 + i * BKV, full);
+        }
         return true;
       };
       ok = load(0, false);
@@ -376,7 +385,8 @@ prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     if (ok && n_mine > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done[grp], (n_mine - 1) & 1, err));
     tc::fence_after_sync();
     const int s = s_base + grp * BQ + row;
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + (((size_t)b * p.S + s) * p.nh + h) * HD;
+    const size_t tok = VARLEN ? (size_t)sq.q0 + s : (size_t)b * p.S + s;
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + (tok * p.nh + h) * HD;
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
     for (int c = 0; c < HD / 16; ++c) {
@@ -409,30 +419,38 @@ prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
   }
 }
 
-template <int HD, int POLY>
+template <int HD, int POLY, bool VARLEN>
 cudaError_t launch_hd(const PrefillParams& p, cudaStream_t st) {
   using C = FaCfg<HD>;
   static std::atomic<bool> attr_set[64];
-  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(prefill_fa_kernel<HD, POLY>), C::SMEM);
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(prefill_fa_kernel<HD, POLY, VARLEN>),
+                                     C::SMEM);
       e != cudaSuccess)
     return e;
   CUtensorMap tq, tk, tv;
-  const uint64_t q_rows = (uint64_t)p.B * p.nh * p.S, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
-  if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+  if (VARLEN) {
+    if (!make_tmap_packed(&tq, p.q, p.total_q, p.nh, HD)) return cudaErrorInvalidValue;
+    if (!make_tmap_packed(&tk, p.k_cache, p.cap, p.nkv, HD)) return cudaErrorInvalidValue;
+    if (!make_tmap_packed(&tv, p.v_cache, p.cap, p.nkv, HD)) return cudaErrorInvalidValue;
+  } else {
+    const uint64_t q_rows = (uint64_t)p.B * p.nh * p.S, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
+    if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+  }
   const int n_qt = (p.S + BQ - 1) / BQ;
   const long long grid = (long long)((n_qt + 1) / 2) * p.B * p.nh;
-  prefill_fa_kernel<HD, POLY><<<(unsigned)grid, THREADS, C::SMEM, st>>>(tq, tk, tv, p, n_qt);
+  prefill_fa_kernel<HD, POLY, VARLEN><<<(unsigned)grid, THREADS, C::SMEM, st>>>(tq, tk, tv, p, n_qt);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_prefill_fa(const PrefillParams& p, cudaStream_t st) {
+  const bool packed = p.cu_q != nullptr;
   switch (p.hd) {
-    case 64: return launch_hd<64, kPoly64>(p, st);
-    case 128: return launch_hd<128, kPoly128>(p, st);
+    case 64: return packed ? launch_hd<64, kPoly64, true>(p, st) : launch_hd<64, kPoly64, false>(p, st);
+    case 128: return packed ? launch_hd<128, kPoly128, true>(p, st) : launch_hd<128, kPoly128, false>(p, st);
     default: return cudaErrorInvalidValue;
   }
 }

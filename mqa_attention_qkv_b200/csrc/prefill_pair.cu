@@ -15,6 +15,7 @@
 // max and independent accumulators so the per-row chains stay short.  O is
 // rescaled in TMEM only when a row max grows by more than 2^8.
 #include "kernels.h"
+#include "prefill_seq.cuh"
 #include "tc.cuh"
 
 namespace gqa {
@@ -42,6 +43,10 @@ using tc::fma2;
 using tc::max3;
 using tc::mma_bf16_ts;
 
+// VARLEN: packed variable-length sequences (3-D tensor maps over
+// [tokens, heads, 64 columns]); otherwise the padded layout (2-D maps over
+// [rows, 64 columns]).  Both read the same 128 x 64 swizzled tiles.
+template <bool VARLEN>
 __global__ void __launch_bounds__(THREADS, 2)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, PrefillParams p, int n_qt) {
@@ -59,11 +64,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const int j = h / (p.nh / p.nkv);
   const int s0 = qt * BQ;
 
-  int kv_len = p.kv_lens[b];
-  if (kv_len > p.cap || kv_len < 0) {
-    if (threadIdx.x == 0) raise_error(err, GQA_DEVERR_KVLEN_RANGE);
-    kv_len = kv_len > p.cap ? p.cap : 0;
-  }
+  const SeqRange sq = prefill_seq(p, b, err);
+  if (VARLEN && s0 >= sq.S) return;   // a shorter sequence: no query in this tile (whole CTA)
+  const int kv_len = sq.kv_len;
 
   const int row = (warp & 3) * 32 + lane;
   int my_lim = 0;
@@ -95,9 +98,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   __syncthreads();
   if (warp >= 2) {
     const int s = s0 + row;
-    my_valid = s < p.S;
+    my_valid = s < sq.S;
     if (my_valid) {
-      const int pos = p.q_pos ? p.q_pos[(size_t)b * p.S + s] : kv_len - p.S + s;
+      const int pos = p.q_pos ? p.q_pos[(size_t)b * p.S + s] : kv_len - sq.S + s;
       my_lim = p.causal ? max(0, min(kv_len, pos + 1)) : kv_len;
       atomicMax(&bars->lim_max, my_lim);
     }
@@ -109,7 +112,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const int kv_hi = bars->lim_max < 0 ? 0 : bars->lim_max;
   const int n_kv = (kv_hi + BKV - 1) / BKV;
   const bool sanitize = n_kv > 0 && kv_len < n_kv * BKV;
-  const int kv_row0 = (b * p.nkv + j) * p.cap;
+  const int kv_row0 = VARLEN ? 0 : (b * p.nkv + j) * p.cap;
   uint8_t* sQ = smem + Q_OFF;
   uint8_t* sK = smem + K_OFF;
   uint8_t* sV = smem + V_OFF;
@@ -119,19 +122,28 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     bool ok = true;
     if (lane == 0 && n_kv > 0) {
       mbar_arrive_expect_tx(&bars->q_full, TILE);
-      tc::tma_load_2d(sQ, &tmq, 0, (b * p.nh + h) * p.S + s0, &bars->q_full);
+      if (VARLEN)
+        tc::tma_load_3d(sQ, &tmq, 0, h, sq.q0 + s0, &bars->q_full);
+      else
+        tc::tma_load_2d(sQ, &tmq, 0, (b * p.nh + h) * p.S + s0, &bars->q_full);
       auto load_k = [&](int t) {
         const int st = t % KS;
         if (!mbar_wait(&bars->k_empty[st], ((t / KS) & 1) ^ 1, err)) return false;
         mbar_arrive_expect_tx(&bars->k_full[st], TILE);
-        tc::tma_load_2d(sK + st * TILE, &tmk, 0, kv_row0 + t * BKV, &bars->k_full[st]);
+        if (VARLEN)
+          tc::tma_load_3d(sK + st * TILE, &tmk, 0, j, sq.k0 + t * BKV, &bars->k_full[st]);
+        else
+          tc::tma_load_2d(sK + st * TILE, &tmk, 0, kv_row0 + t * BKV, &bars->k_full[st]);
         return true;
       };
       auto load_v = [&](int t) {
         const int st = t % VS;
         if (!mbar_wait(&bars->v_empty[st], ((t / VS) & 1) ^ 1, err)) return false;
         mbar_arrive_expect_tx(&bars->v_full[st], TILE);
-        tc::tma_load_2d(sV + st * TILE, &tmv, 0, kv_row0 + t * BKV, &bars->v_full[st]);
+        if (VARLEN)
+          tc::tma_load_3d(sV + st * TILE, &tmv, 0, j, sq.k0 + t * BKV, &bars->v_full[st]);
+        else
+          tc::tma_load_2d(sV + st * TILE, &tmv, 0, kv_row0 + t * BKV, &bars->v_full[st]);
         return true;
       };
       ok = load_k(0);
@@ -271,7 +283,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 
     if (ok && n_kv > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (n_kv - 1) & 1, err));
     tc::fence_after_sync();
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + (((size_t)b * p.S + (s0 + row)) * p.nh + h) * HD;
+    const size_t tok = VARLEN ? (size_t)sq.q0 + s0 + row : (size_t)b * p.S + (s0 + row);
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + (tok * p.nh + h) * HD;
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
     for (int c = 0; c < HD / 16; ++c) {
@@ -304,23 +317,34 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   }
 }
 
+template <bool VARLEN>
+cudaError_t launch_pair(const PrefillParams& p, cudaStream_t st) {
+  static std::atomic<bool> attr_set[64];
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(prefill_pair_kernel<VARLEN>), SMEM);
+      e != cudaSuccess)
+    return e;
+  CUtensorMap tq, tk, tv;
+  if (VARLEN) {
+    if (!make_tmap_packed(&tq, p.q, p.total_q, p.nh, HD)) return cudaErrorInvalidValue;
+    if (!make_tmap_packed(&tk, p.k_cache, p.cap, p.nkv, HD)) return cudaErrorInvalidValue;
+    if (!make_tmap_packed(&tv, p.v_cache, p.cap, p.nkv, HD)) return cudaErrorInvalidValue;
+  } else {
+    const uint64_t q_rows = (uint64_t)p.B * p.nh * p.S, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
+    if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
+  }
+  const int n_qt = (p.S + BQ - 1) / BQ;
+  const long long grid = (long long)n_qt * p.B * p.nh;
+  prefill_pair_kernel<VARLEN><<<(unsigned)grid, THREADS, SMEM, st>>>(tq, tk, tv, p, n_qt);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st) {
   if (p.hd != HD) return cudaErrorInvalidValue;
-  static std::atomic<bool> attr_set[64];
-  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(prefill_pair_kernel), SMEM);
-      e != cudaSuccess)
-    return e;
-  CUtensorMap tq, tk, tv;
-  const uint64_t q_rows = (uint64_t)p.B * p.nh * p.S, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
-  if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, kv_rows, HD * 2, 64, 128)) return cudaErrorInvalidValue;
-  const int n_qt = (p.S + BQ - 1) / BQ;
-  const long long grid = (long long)n_qt * p.B * p.nh;
-  prefill_pair_kernel<<<(unsigned)grid, THREADS, SMEM, st>>>(tq, tk, tv, p, n_qt);
-  return cudaGetLastError();
+  return p.cu_q ? launch_pair<true>(p, st) : launch_pair<false>(p, st);
 }
 
 }  // namespace gqa

@@ -60,4 +60,11 @@ bool make_tmap_bf16_3d(void* map, const void* base, const uint64_t dims[3], cons
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_packed(void* map, const void* base, uint64_t tokens, int heads, int hd) {
+  const uint64_t dims[3] = {(uint64_t)hd, (uint64_t)heads, tokens > 0 ? tokens : 1};
+  const uint64_t strides[2] = {(uint64_t)hd * 2, (uint64_t)heads * hd * 2};
+  const uint32_t box[3] = {64, 1, 128};
+  return make_tmap_bf16_3d(map, base, dims, strides, box);
+}
+
 }  // namespace gqa

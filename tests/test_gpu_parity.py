@@ -192,6 +192,100 @@ def test_prefill_explicit_positions_and_empty_rows():
 
 
 # --------------------------------------------------------------------------
+# packed variable-length prefill
+# --------------------------------------------------------------------------
+VARLEN_Q = [1, 127, 128, 129, 300, 0, 64, 257, 10]
+VARLEN_K = [1, 127, 133, 129, 400, 3, 64, 257, 4]     # cached prefixes; the last has fewer keys than queries
+
+
+def varlen_inputs(nh, nkv, hd, q_lens, k_lens, seed):
+    cq = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    ck = np.concatenate([[0], np.cumsum(k_lens)]).astype(np.int32)
+    q = W.normal_tensor((int(cq[-1]), nh, hd), seed, 0, "bf16")
+    k = W.normal_tensor((int(ck[-1]), nkv, hd), seed, 1, "bf16")
+    v = W.normal_tensor((int(ck[-1]), nkv, hd), seed, 2, "bf16")
+    return q, k, v, cq, ck
+
+
+def run_varlen(q, k, v, cq, ck, causal, max_q=None, out=None):
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    max_q = int(np.diff(cq).max()) if max_q is None else max_q
+    gqa.gqa_attn_prefill_varlen(dev(q), dev(k), dev(v), dev_i32(cq), dev_i32(ck), max_q, causal, out)
+    return out
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("hd,g,nkv", [(64, 1, 2), (64, 8, 1), (128, 4, 2), (128, 1, 1)])
+def test_varlen_prefill_parity(hd, g, nkv, causal):
+    """Packed sequences of ragged lengths (tile edges, an empty one, cached
+    prefixes, fewer keys than queries) against the oracle's packed prefill."""
+    nh = g * nkv
+    q, k, v, cq, ck = varlen_inputs(nh, nkv, hd, VARLEN_Q, VARLEN_K, 80 + hd + g)
+    gqa.gqa_device_error()
+    got = host(run_varlen(q, k, v, cq, ck, causal))
+    assert gqa.gqa_device_error() == 0
+    want = ref.varlen_prefill_attention(q.f64, k.f64, v.f64, cq, ck, causal)
+    if causal:   # the last sequence's first 6 queries see no key
+        assert np.all(got[cq[-2]:cq[-2] + 6] == 0)
+    gate(got.reshape(-1, hd), want.reshape(-1, hd), "bf16", f"varlen prefill hd{hd} g{g} causal={causal}",
+         heads=np.tile(np.arange(nh), got.shape[0]))
+
+
+@pytest.mark.parametrize("hd", [64, 128])
+def test_varlen_prefill_matches_padded_bit_for_bit(hd):
+    """The same sequences padded into [B, nh, S, hd] queries and a
+    [B, nkv, cap, hd] cache, with the packed call's positions passed
+    explicitly, give the same bits: only the tiles' addresses differ."""
+    nh, nkv = 8, 2
+    q_lens, k_lens = VARLEN_Q[:-1], VARLEN_K[:-1]
+    q, k, v, cq, ck = varlen_inputs(nh, nkv, hd, q_lens, k_lens, 90 + hd)
+    B, S, cap = len(q_lens), max(q_lens), max(k_lens)
+    qp = np.zeros((B, nh, S, hd), dtype=np.uint16)
+    kp = np.full((B, nkv, cap, hd), SENTINEL["bf16"], dtype=np.uint16)
+    vp = np.full((B, nkv, cap, hd), SENTINEL["bf16"], dtype=np.uint16)
+    pos = np.full((B, S), -1, dtype=np.int32)
+    for b in range(B):
+        qp[b, :, :q_lens[b]] = q.store[cq[b]:cq[b + 1]].transpose(1, 0, 2)
+        kp[b, :, :k_lens[b]] = k.store[ck[b]:ck[b + 1]].transpose(1, 0, 2)
+        vp[b, :, :k_lens[b]] = v.store[ck[b]:ck[b + 1]].transpose(1, 0, 2)
+        pos[b, :q_lens[b]] = k_lens[b] - q_lens[b] + np.arange(q_lens[b])
+    out_p = torch.empty((B, S, nh, hd), dtype=torch.bfloat16, device="cuda")
+    gqa.gqa_attn_prefill(dev(W.Tensor(qp, "bf16")), dev(W.Tensor(kp, "bf16")), dev(W.Tensor(vp, "bf16")),
+                         dev_i32(np.array(k_lens, dtype=np.int32)), True, out_p, q_positions=dev_i32(pos))
+    packed = bits(run_varlen(q, k, v, cq, ck, True))
+    padded = bits(out_p)
+    for b in range(B):
+        np.testing.assert_array_equal(packed[cq[b]:cq[b + 1]], padded[b, :q_lens[b]])
+
+
+def test_varlen_prefill_bad_offsets_are_clamped_and_flagged():
+    """Offsets past the packed tensors are clamped (nothing is written past
+    the output) and flagged; so is a query run longer than max_seqlen_q."""
+    nh, nkv, hd = 4, 1, 64
+    q, k, v, cq, ck = varlen_inputs(nh, nkv, hd, [100, 200], [100, 200], 95)
+    tq = int(cq[-1])
+    big = torch.full((tq + 64, nh, hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    bad_q = cq.copy()
+    bad_q[-1] = tq + 50
+    bad_k = ck.copy()
+    bad_k[-1] = int(ck[-1]) + 77
+    gqa.gqa_device_error()
+    run_varlen(q, k, v, bad_q, bad_k, True, max_q=256, out=big[:tq])
+    assert gqa.gqa_device_error() & 16
+    assert torch.isnan(big[tq:]).all()
+    want = ref.varlen_prefill_attention(q.f64, k.f64, v.f64, cq, ck, True)
+    gate(host(big[:tq]).reshape(-1, hd), want.reshape(-1, hd), "bf16", "clamped offsets",
+         heads=np.tile(np.arange(nh), tq))
+    # max_seqlen_q shorter than a run: flagged; the rows the grid covers are right
+    out = run_varlen(q, k, v, cq, ck, True, max_q=128)
+    assert gqa.gqa_device_error() & 16
+    got = host(out)
+    gate(got[:100].reshape(-1, hd), want[:100].reshape(-1, hd), "bf16", "short max_seqlen_q",
+         heads=np.tile(np.arange(nh), 100))
+
+
+# --------------------------------------------------------------------------
 # a5-a6: decode
 # --------------------------------------------------------------------------
 def run_decode(q, kc, vc, lens, nh, dtype, kv_split=0):
