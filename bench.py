@@ -354,7 +354,8 @@ def measure_workloads(dev, peaks, iters=10, only=None):
     transform on the Llama-2-7B projection (32 -> 8 KV heads): GB/s.  Each
     kernel is timed alone with CUDA events, L2 flushed before every timed call
     (a 512 MB write), median of `iters`.  ``only``: a set of section names
-    (decode, prefill8k, generate, small, meanpool) to measure; None = all."""
+    (decode, prefill8k, generate, small, varlen, meanpool) to measure; None =
+    all."""
     import numpy as np
     import torch
 
@@ -514,6 +515,29 @@ def measure_workloads(dev, peaks, iters=10, only=None):
                                  "attn_ms": round(ms_a, 4), "attn_TFLOP/s": round(fl_a / (ms_a / 1e3) / 1e12, 1),
                                  "tokens_per_s": round(B * S / ((ms_p + ms_a) / 1e3), 1)}
         out["tinyllama_prefill_small"] = small
+
+    # ---- packed variable-length prefill: the TinyLlama layer's attention over
+    # 16 ragged causal sequences of 64..960 tokens, packed without padding
+    if want("varlen"):
+        sh = W.TINYLLAMA_PREFILL.shape
+        nh, nkv, hd = sh.n_heads, sh.n_kv_heads, sh.head_dim
+        seq = W.ragged_lengths(16, 64, 960, W.TINYLLAMA_PREFILL.seed)
+        cu = torch.from_numpy(np.concatenate([[0], np.cumsum(seq)]).astype(np.int32)).to(dev)
+        tot = int(seq.sum())
+        q = torch.randn(tot, nh, hd, generator=gen, device=dev).to(bf)
+        k = torch.randn(tot, nkv, hd, generator=gen, device=dev).to(bf)
+        v = torch.randn(tot, nkv, hd, generator=gen, device=dev).to(bf)
+        o = torch.empty_like(q)
+        try:
+            ms = timed(lambda: gqa.gqa_attn_prefill_varlen(q, k, v, cu, cu, int(seq.max()), True, o, stream=stream))
+            # exact visible (query, key) pairs of the causal sequences
+            fl = 4.0 * nh * hd * float(np.sum(seq.astype(np.float64) * (seq + 1) / 2))
+            tf = fl / (ms / 1e3) / 1e12
+            out["varlen_prefill_tinyllama_16_ragged"] = {
+                "ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_bf16": round(tf / bf16_peak, 4),
+                "tokens": tot, "tokens_per_s": round(tot / (ms / 1e3), 1)}
+        except Exception as exc:   # an auxiliary line: report it, keep the bench line
+            out["varlen_prefill_tinyllama_16_ragged"] = {"error": str(exc)}
 
     # ---- MHA -> GQA weight transform on the Llama-2-7B projection (32 heads -> 8 KV heads)
     if want("meanpool"):

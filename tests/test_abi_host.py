@@ -141,6 +141,27 @@ def test_paged_decode_rejects(kw, code):
     assert _paged(**kw) == code
 
 
+def _varlen(**kw):
+    a = dict(q=P, k=P, v=P, cq=P, ck=P, B=2, tq=300, tk=300, maxq=200, nh=8, nkv=2, hd=64, causal=1, out=P,
+             dtype=1, stream=None)
+    a.update(kw)
+    return gqa.lib().gqa_attn_prefill_varlen(a["q"], a["k"], a["v"], a["cq"], a["ck"], a["B"], a["tq"], a["tk"],
+                                             a["maxq"], a["nh"], a["nkv"], a["hd"], a["causal"], a["out"],
+                                             a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(cq=None), INVALID), (dict(ck=None), INVALID), (dict(k=None), INVALID), (dict(out=None), INVALID),
+    (dict(B=-1), INVALID), (dict(tq=-1), INVALID), (dict(tk=-5), INVALID), (dict(maxq=-1), INVALID),
+    (dict(nh=6, nkv=4), INVALID), (dict(nkv=0), INVALID), (dict(hd=32), SHAPE), (dict(hd=96), SHAPE),
+    (dict(dtype=0), DTYPE), (dict(cq=P + 2), MISALIGNED), (dict(q=MIS), MISALIGNED),
+    (dict(tq=1 << 30, nh=2048, nkv=2048), SHAPE),              # 2^47 query elements
+    (dict(B=60000, maxq=1 << 20, nh=64, nkv=8), SHAPE),        # grid of 2^31 tiles or more
+])
+def test_varlen_prefill_rejects(kw, code):
+    assert _varlen(**kw) == code
+
+
 def test_empty_inputs_are_noops():
     # B == 0 or S == 0 returns OK without launching (pointers may then be NULL)
     assert _qkv(B=0, x=None, w=None, pos=None, q=None, k=None, v=None) == 0
@@ -149,6 +170,9 @@ def test_empty_inputs_are_noops():
     assert _prefill(S=0) == 0
     assert _decode(B=0, q=None, ws=None) == 0
     assert _paged(B=0, q=None, table=None, ws=None) == 0
+    assert _varlen(B=0, q=None, cq=None) == 0
+    assert _varlen(tq=0) == 0
+    assert _varlen(maxq=0) == 0
 
 
 def test_workspace_size_query():
@@ -174,6 +198,8 @@ def test_valid_call_without_gpu_reports_no_device():
     assert _decode() in (NODEV, ARCH)
     assert _meanpool() in (NODEV, ARCH)
     assert _paged() in (NODEV, ARCH)
+    assert _varlen() in (NODEV, ARCH)
+    assert _varlen(tk=0) in (NODEV, ARCH)      # no keys at all: zero rows
 
 
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
