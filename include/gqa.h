@@ -311,6 +311,15 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
                           int kv_split, void* out, void* workspace, size_t workspace_bytes, int dtype,
                           void* stream);
 
+/*
+ * gqa_debug_inject_launch_failures - testing aid (host-side fault
+ * injection): the next n compute calls (projection, prefill, decode,
+ * mean-pool) that pass argument validation return GQA_ERR_LAUNCH_FAILED
+ * without launching anything, as a failed launch would; later calls run
+ * normally.  n = 0 clears pending injections; n < 0 is GQA_ERR_INVALID_ARG.
+ */
+int gqa_debug_inject_launch_failures(int n);
+
 /* Human-readable text of a gqa_status value (static storage). */
 const char* gqa_status_string(int status);
 

@@ -17,7 +17,7 @@ __all__ = [
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
-    "gqa_attn_prefill_varlen", "EXPORTED_SYMBOLS",
+    "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures", "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -27,7 +27,7 @@ EXPORTED_SYMBOLS = (
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
-    "gqa_attn_prefill_varlen",
+    "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
     L.gqa_attn_decode_paged.restype = i32
     L.gqa_attn_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     L.gqa_attn_prefill_varlen.restype = i32
+    L.gqa_debug_inject_launch_failures.argtypes = [i32]
+    L.gqa_debug_inject_launch_failures.restype = i32
     _LIB = L
     return L
 
@@ -238,6 +240,12 @@ def gqa_device_error() -> int:
     v = ctypes.c_int(0)
     _check("gqa_device_error", lib().gqa_device_error(ctypes.byref(v)))
     return v.value
+
+
+def gqa_debug_inject_launch_failures(n: int) -> None:
+    """Testing aid: the next ``n`` compute calls fail as a failed launch would
+    (GQAError with status GQA_ERR_LAUNCH_FAILED), launching nothing."""
+    _check("gqa_debug_inject_launch_failures", lib().gqa_debug_inject_launch_failures(int(n)))
 
 
 def gqa_launch_count() -> int:

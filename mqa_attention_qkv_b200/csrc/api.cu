@@ -54,6 +54,28 @@ const DeviceInfo* device_info(int* status) {
   return &d;
 }
 
+// Launch failures injected by gqa_debug_inject_launch_failures: the next n
+// compute calls that pass validation report GQA_ERR_LAUNCH_FAILED without
+// launching anything.
+std::atomic<int> g_inject_failures{0};
+
+bool take_injected_failure() {
+  int n = g_inject_failures.load(std::memory_order_relaxed);
+  while (n > 0)
+    if (g_inject_failures.compare_exchange_weak(n, n - 1, std::memory_order_relaxed)) return true;
+  return false;
+}
+
+// Device facts for a compute call (an injected failure is reported here,
+// after argument validation and before any launch).
+const DeviceInfo* compute_device(int* status) {
+  if (take_injected_failure()) {
+    *status = GQA_ERR_LAUNCH_FAILED;
+    return nullptr;
+  }
+  return device_info(status);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool hd_ok(int hd) { return hd == 32 || hd == 64 || hd == 128; }
@@ -94,7 +116,7 @@ namespace gqa {
 
 int device_check(int** err) {
   int st;
-  const DeviceInfo* d = device_info(&st);
+  const DeviceInfo* d = compute_device(&st);
   if (d && err) *err = d->err;
   return st;
 }
@@ -171,7 +193,7 @@ int qkv_rope_project(const void* x, const void* w_qkv, const int32_t* positions,
       !aligned16(v_cache) || !aligned4(positions))
     return GQA_ERR_MISALIGNED;
   int st;
-  const DeviceInfo* d = device_info(&st);
+  const DeviceInfo* d = compute_device(&st);
   if (!d) return st;
 
   gqa::QkvParams p{x, w_qkv, positions, B, S, hidden, n_heads, n_kv_heads, head_dim, cache_cap,
@@ -204,7 +226,7 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
       !aligned4(kv_lens) || (q_positions && !aligned4(q_positions)))
     return GQA_ERR_MISALIGNED;
   int st;
-  const DeviceInfo* d = device_info(&st);
+  const DeviceInfo* d = compute_device(&st);
   if (!d) return st;
 
   gqa::PrefillParams p{q, k_cache, v_cache, q_positions, kv_lens, B, S, n_heads, n_kv_heads,
@@ -234,7 +256,7 @@ int gqa_attn_prefill_varlen(const void* q, const void* k, const void* v, const i
       !aligned4(cu_seqlens_k))
     return GQA_ERR_MISALIGNED;
   int st;
-  const DeviceInfo* d = device_info(&st);
+  const DeviceInfo* d = compute_device(&st);
   if (!d) return st;
 
   gqa::PrefillParams p{q, k, v, nullptr, nullptr, B, max_seqlen_q, n_heads, n_kv_heads, head_dim, total_k,
@@ -277,7 +299,7 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
   const size_t need = gqa_attn_decode_workspace_size(B, n_heads, n_kv_heads, head_dim, cache_cap, kv_split);
   if (workspace_bytes < need) return GQA_ERR_WORKSPACE_TOO_SMALL;
   int st;
-  const DeviceInfo* d = device_info(&st);
+  const DeviceInfo* d = compute_device(&st);
   if (!d) return st;
 
   const gqa::DecodeParams p = gqa::decode_params(q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim,
@@ -314,7 +336,7 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
   if (need == 0) return GQA_ERR_UNSUPPORTED_SHAPE;
   if (workspace_bytes < need) return GQA_ERR_WORKSPACE_TOO_SMALL;
   int st;
-  const DeviceInfo* d = device_info(&st);
+  const DeviceInfo* d = compute_device(&st);
   if (!d) return st;
 
   gqa::DecodeParams p = gqa::decode_params(q, k_pages, v_pages, kv_lens, B, n_heads, n_kv_heads, head_dim,
@@ -330,5 +352,11 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
 }
 
 uint64_t gqa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int gqa_debug_inject_launch_failures(int n) {
+  if (n < 0) return GQA_ERR_INVALID_ARG;
+  g_inject_failures.store(n, std::memory_order_relaxed);
+  return GQA_OK;
+}
 
 }  // extern "C"

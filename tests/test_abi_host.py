@@ -226,3 +226,30 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(ValueError, match="CUDA tensor"):
         gqa.gqa_attn_decode_paged(q, kc, kc, torch.zeros(2, 1, dtype=torch.int32), lens, q.clone(),
                                   torch.zeros(1024, dtype=torch.uint8))
+
+
+def test_injected_launch_failures_are_reported_then_clear():
+    """Host-side fault injection: after validation, the next n compute calls
+    report GQA_ERR_LAUNCH_FAILED without launching; invalid calls are still
+    refused first and do not use an injection."""
+    assert gqa.lib().gqa_debug_inject_launch_failures(-1) == INVALID
+    n0 = gqa.gqa_launch_count()
+    gqa.gqa_debug_inject_launch_failures(3)
+    try:
+        assert _decode(dtype=7) == DTYPE
+        assert _decode() == LAUNCH
+        assert _qkv() == LAUNCH
+        assert _meanpool() == LAUNCH
+        if not _gpu_present():
+            assert _decode() in (NODEV, ARCH)     # the injections are used up
+    finally:
+        gqa.gqa_debug_inject_launch_failures(0)
+    assert gqa.gqa_launch_count() == n0            # nothing was launched
+    with pytest.raises(gqa.GQAError) as e:
+        gqa._check("gqa_attn_decode", LAUNCH)
+    assert e.value.status == LAUNCH and "launch failed" in str(e.value)
+
+
+def _gpu_present():
+    import torch
+    return torch.cuda.is_available()

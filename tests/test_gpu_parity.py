@@ -499,6 +499,27 @@ def test_paged_decode_bad_table_entry_flags_and_reads_zeros():
     gate(got, want, "bf16", "zero-read pages")
 
 
+def test_injected_launch_failure_leaves_the_library_usable():
+    """A failure injected on the host surfaces as GQAError (launch failed)
+    and launches nothing; the next call runs and gives the same bits."""
+    dtype, hd, nh, nkv, cap = "bf16", 128, 8, 2, 256
+    lens = np.array([256, 100], dtype=np.int32)
+    q = W.normal_tensor((2, nh, hd), 15, 0, dtype)
+    kc = nan_padded(2, nkv, cap, hd, lens, 15, 1, dtype)
+    vc = nan_padded(2, nkv, cap, hd, lens, 15, 2, dtype)
+    first = bits(run_decode(q, kc, vc, lens, nh, dtype))
+    n0 = gqa.gqa_launch_count()
+    gqa.gqa_debug_inject_launch_failures(1)
+    try:
+        with pytest.raises(gqa.GQAError) as e:
+            run_decode(q, kc, vc, lens, nh, dtype)
+        assert e.value.status == -6
+        assert gqa.gqa_launch_count() == n0
+    finally:
+        gqa.gqa_debug_inject_launch_failures(0)
+    np.testing.assert_array_equal(bits(run_decode(q, kc, vc, lens, nh, dtype)), first)
+
+
 def test_decode_zero_and_clamped_lengths():
     dtype, hd, nh, nkv, cap = "bf16", 64, 4, 2, 128
     lens = np.array([0, 128, 5], dtype=np.int32)
