@@ -99,7 +99,9 @@ enum gqa_device_error_bits {
  *              of every KV head of sequence b is overwritten, all other rows
  *              are left untouched.  A position outside [0, cache_cap) writes
  *              no K/V row and sets GQA_DEVERR_POSITION_RANGE (q is still
- *              written, rotated by that position).
+ *              written, rotated by that position).  Two tokens of one
+ *              sequence with the same position write the same row; which
+ *              one lands is unspecified.
  *
  * The math is float32 (fp32 accumulation of bf16 products for GQA_BF16), with
  * one final rounding of q/k/v to dtype.
