@@ -1,7 +1,8 @@
-"""Host logic of the multi-GPU bench (replicas only: the path has no exchange
-step, so N GPUs run N independent replicas).  Two gloo ranks on the CPU check
-the max-over-ranks timing and the whole-job rate; the reference arm's other
-ranks exit without work."""
+"""Host logic of bench.py that needs no GPU.  Multi-GPU is replicas only
+(the path has no exchange step, so N GPUs run N independent replicas): gloo
+ranks on the CPU check the max-over-ranks timing and the whole-job rate, and
+the reference arm's other ranks exit without work.  The reference arm's JSON
+line is checked on a tiny layer."""
 import os
 import socket
 import subprocess
@@ -70,3 +71,28 @@ def test_reference_arm_other_ranks_exit_without_work():
                         "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    """The reference arm (the float64 oracle on host cores) prints one JSON
+    line with the contract's keys; a tiny layer keeps it quick here."""
+    import json
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setattr(bench, "WORKLOAD", dict(bench.WORKLOAD, S=64, hidden=128, n_heads=4, n_kv_heads=2,
+                                                 head_dim=32, cap=80))
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    bench.run_reference(types.SimpleNamespace(steps=2, warmup=3, gpus=1))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 3 and line["n_gpus"] == 1
+    assert line["value"] > 0 and line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["config"]["workload"] == bench.WORKLOAD["name"]
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
