@@ -253,3 +253,20 @@ def test_injected_launch_failures_are_reported_then_clear():
 def _gpu_present():
     import torch
     return torch.cuda.is_available()
+
+
+def test_binding_argument_lists_match_the_header():
+    """Every declared function is bound with as many arguments as the header
+    gives it (catches drift between include/gqa.h and the ctypes binding)."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decl = re.compile(r"^\s*(?:const\s+)?(?:int|size_t|uint64_t|char\s*\*|void)\s*\*?\s*(\w+)\s*\(([^)]*)\)\s*;",
+                      re.M)
+    L = gqa.lib()
+    seen = 0
+    for name, params in decl.findall(src):
+        params = params.strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        argtypes = getattr(L, name).argtypes
+        assert argtypes is not None and len(argtypes) == n, (name, n, argtypes)
+        seen += 1
+    assert seen == len(gqa.EXPORTED_SYMBOLS)
