@@ -309,12 +309,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->p_full[t & 1]);
     }
-    // O is final once P.V of the last tile has completed.  A parity wait only
-    // tells the newest phase apart from the one before it, and P.V of the
-    // tile before last may still be running here (the last S was issued ahead
-    // of it), so wait for that phase first.
-    if (ok && n_t > 1) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (n_t - 2) & 1, err));
-    if (ok && n_t > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (n_t - 1) & 1, err));
+    // O is final once every MMA has completed, which the single-phase drain
+    // barrier says (the MMA thread commits it after the last P.V).  o_done
+    // cannot say it: a parity wait only tells the newest phase from the one
+    // before it, and here o_done may be one phase short (P.V of the tile
+    // before last still running: the last S went in ahead of it) or already
+    // past both last phases.
+    if (ok && n_t > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->drain, 0, err));
+      // a wait that gave up anywhere (the MMA thread's included) voids O
+      ok = ok && __all_sync(0xffffffffu, !(*reinterpret_cast<volatile int*>(err) & GQA_DEVERR_WAIT_TIMEOUT));
+    }
     tc::fence_after_sync();
     const bool have_o = ok && n_t > 0 && active;
     if (nsp == 1) {
