@@ -123,3 +123,17 @@ def test_incoherent_processing_reduces_fp8_error_with_outliers():
     err_plain = np.sqrt(np.mean((f8.fp8_attention(q, k, v) - exact) ** 2))
     err_rot = np.sqrt(np.mean((f8.fp8_attention(q, k, v, rotation=m) - exact) ** 2))
     assert err_rot * 1.25 <= err_plain, (err_plain, err_rot)
+
+
+def test_round_e4m3_matches_torch_float8_cast_in_range():
+    """Inside the finite range the rounding is the library's e4m3 cast
+    (torch.float8_e4m3fn: nearest, ties to even), checked on random values
+    and on every exact midpoint between neighbouring codes."""
+    import torch
+    grid = f8.e4m3_values()
+    r = np.random.default_rng(12)
+    x = np.concatenate([r.standard_normal(20000) * 50.0, r.standard_normal(5000) * 1e-2, grid,
+                        (grid[1:] + grid[:-1]) / 2.0]).astype(np.float32)
+    x = x[np.abs(x) <= 448.0]
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(f8.round_e4m3(x.astype(np.float64)), lib)
