@@ -539,6 +539,18 @@ def test_round_bf16_matches_bit_level_rounding():
     np.testing.assert_array_equal(ref.round_bf16(a.astype(np.float64)), want)
 
 
+def test_round_bf16_matches_the_library_cast():
+    """A third route: torch's float32 -> bfloat16 cast (nearest, ties to even),
+    on random values and on exact midpoints between neighbouring bf16 values."""
+    import torch
+    r = rng(32)
+    a = np.concatenate([r.standard_normal(100000) * 3, r.standard_normal(1000) * 1e-30]).astype(np.float32)
+    mids = (a.view(np.uint32) & np.uint32(0xFFFF0000)) | np.uint32(0x8000)    # halfway bit patterns
+    a = np.concatenate([a, mids.view(np.float32)])
+    lib = torch.from_numpy(a).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(ref.round_bf16(a.astype(np.float64)), lib)
+
+
 def test_round_bf16_exact_and_ties_to_even():
     exact = np.array([1.0, -2.0, 1.5, 0.00390625, 3.0 * 2 ** 40, 1 + 2 ** -7])
     np.testing.assert_array_equal(ref.round_bf16(exact), exact)
