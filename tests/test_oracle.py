@@ -928,3 +928,37 @@ def test_planted_head_major_concat_is_caught(monkeypatch):
         return orig(np.swapaxes(o, -1, -2).reshape(o.shape), w_o, residual)
     monkeypatch.setattr(ref, "output_projection", channel_major)
     assert _fails(check_output_projection_is_a_sum_over_heads)
+
+
+# --------------------------------------------------------------------------
+# library routine as a special case: torch's scaled_dot_product_attention
+# (float64, CPU) computes the same attention when every sequence is full
+# (top-left and bottom-right causal alignment coincide) and, for decode,
+# per sequence over its first kv_len keys
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("nh,nkv", [(8, 2), (4, 4), (6, 1)])
+def test_prefill_equals_library_sdpa(causal, nh, nkv):
+    import torch
+    import torch.nn.functional as F
+    r = rng(80 + nh + nkv)
+    B, S, hd = 2, 37, 16
+    q, k, v = r.normal(size=(B, nh, S, hd)), r.normal(size=(B, nkv, S, hd)), r.normal(size=(B, nkv, S, hd))
+    lib = F.scaled_dot_product_attention(torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v),
+                                         is_causal=causal, enable_gqa=True).numpy()
+    np.testing.assert_allclose(ref.prefill_attention(q, k, v, np.array([S, S]), causal), lib.transpose(0, 2, 1, 3),
+                               rtol=0, atol=1e-12)
+
+
+def test_decode_equals_library_sdpa_per_sequence():
+    import torch
+    import torch.nn.functional as F
+    r = rng(83)
+    B, nh, nkv, cap, hd = 3, 8, 2, 20, 16
+    lens = np.array([20, 1, 9])
+    q, kc, vc = r.normal(size=(B, nh, hd)), r.normal(size=(B, nkv, cap, hd)), r.normal(size=(B, nkv, cap, hd))
+    got = ref.decode_attention(q, kc, vc, lens)
+    for b, L in enumerate(lens):
+        lib = F.scaled_dot_product_attention(torch.from_numpy(q[b][:, None]), torch.from_numpy(kc[b, :, :L]),
+                                             torch.from_numpy(vc[b, :, :L]), enable_gqa=True).numpy()[:, 0]
+        np.testing.assert_allclose(got[b], lib, rtol=0, atol=1e-12)
