@@ -962,3 +962,25 @@ def test_decode_equals_library_sdpa_per_sequence():
         lib = F.scaled_dot_product_attention(torch.from_numpy(q[b][:, None]), torch.from_numpy(kc[b, :, :L]),
                                              torch.from_numpy(vc[b, :, :L]), enable_gqa=True).numpy()[:, 0]
         np.testing.assert_allclose(got[b], lib, rtol=0, atol=1e-12)
+
+
+def test_rope_matches_the_hf_llama_rotary_embedding():
+    """The RoPE reading (rotate_half pairs, inv_freq = theta^(-2i/hd)) is HF
+    Llama's: its rotary embedding and apply_rotary_pos_emb rotate q and k the
+    same way.  The library forms its angles in float32, so the bound is its
+    angle rounding (position x 2^-24 relative), far below the O(1) gap a
+    different pairing, frequency or sign would leave."""
+    import torch
+    from transformers import LlamaConfig
+    from transformers.models.llama.modeling_llama import LlamaRotaryEmbedding, apply_rotary_pos_emb
+    B, S, nh, nkv, hd = 2, 9, 4, 2, 64
+    cfg = LlamaConfig(hidden_size=nh * hd, num_attention_heads=nh, num_key_value_heads=nkv, head_dim=hd,
+                      rope_theta=10000.0, max_position_embeddings=4096)
+    r = rng(84)
+    q, k = r.normal(size=(B, nh, S, hd)), r.normal(size=(B, nkv, S, hd))
+    pos = np.array([[0, 1, 2, 3, 17, 64, 99, 5, 40], [9, 8, 7, 6, 5, 4, 3, 2, 1]])
+    cos, sin = LlamaRotaryEmbedding(cfg)(torch.from_numpy(q), torch.from_numpy(pos))
+    qe, ke = apply_rotary_pos_emb(torch.from_numpy(q), torch.from_numpy(k), cos.double(), sin.double())
+    for mine, lib in ((ref.apply_rope(q.transpose(0, 2, 1, 3), pos, 10000.0), qe),
+                      (ref.apply_rope(k.transpose(0, 2, 1, 3), pos, 10000.0), ke)):
+        np.testing.assert_allclose(mine.transpose(0, 2, 1, 3), lib.numpy(), rtol=0, atol=2e-4)
