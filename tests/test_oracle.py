@@ -984,3 +984,37 @@ def test_rope_matches_the_hf_llama_rotary_embedding():
     for mine, lib in ((ref.apply_rope(q.transpose(0, 2, 1, 3), pos, 10000.0), qe),
                       (ref.apply_rope(k.transpose(0, 2, 1, 3), pos, 10000.0), ke)):
         np.testing.assert_allclose(mine.transpose(0, 2, 1, 3), lib.numpy(), rtol=0, atol=2e-4)
+
+
+@pytest.mark.parametrize("nh,nkv", [(4, 2), (4, 4), (4, 1)])
+def test_layer_equals_hf_llama_attention(nh, nkv):
+    """The whole layer as the pages state it (fused projection sliced into
+    q/k/v, RoPE on q and k, causal attention with the h -> h/g map, output
+    projection) equals HF's LlamaAttention (eager, float64; its rotary
+    angles are float32, hence the bound) with q/k/v_proj cut from W_qkv."""
+    import torch
+    from transformers import LlamaConfig
+    from transformers.models.llama.modeling_llama import LlamaAttention, LlamaRotaryEmbedding
+    B, S, D, hd = 2, 11, 64, 16
+    cfg = LlamaConfig(hidden_size=D, num_attention_heads=nh, num_key_value_heads=nkv, head_dim=hd,
+                      rope_theta=10000.0, attention_bias=False, max_position_embeddings=512)
+    cfg._attn_implementation = "eager"
+    att = LlamaAttention(cfg, layer_idx=0).double()
+    r = rng(85 + nkv)
+    x = r.normal(size=(B, S, D))
+    w = r.normal(size=((nh + 2 * nkv) * hd, D)) * 0.3
+    wo = r.normal(size=(D, nh * hd)) * 0.3
+    q_end, k_end = nh * hd, (nh + nkv) * hd
+    with torch.no_grad():
+        att.q_proj.weight.copy_(torch.from_numpy(w[:q_end]))
+        att.k_proj.weight.copy_(torch.from_numpy(w[q_end:k_end]))
+        att.v_proj.weight.copy_(torch.from_numpy(w[k_end:]))
+        att.o_proj.weight.copy_(torch.from_numpy(wo))
+        pos = np.tile(np.arange(S), (B, 1))
+        cos, sin = LlamaRotaryEmbedding(cfg)(torch.from_numpy(x), torch.from_numpy(pos))
+        mask = torch.full((S, S), float("-inf"), dtype=torch.float64).triu(1)[None, None].expand(B, 1, S, S)
+        lib, _ = att(torch.from_numpy(x), (cos.double(), sin.double()), mask)
+    z = np.zeros((B, nkv, S, hd))
+    q, kc, vc = ref.qkv_rope_project(x, w, pos, nh, nkv, hd, 10000.0, z, z)
+    mine = ref.output_projection(ref.prefill_attention(q, kc, vc, np.full(B, S), True), wo)
+    np.testing.assert_allclose(mine, lib.numpy(), rtol=0, atol=1e-6 * np.max(np.abs(mine)))
