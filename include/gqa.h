@@ -228,19 +228,23 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
  * host framework hands only the op's tensors (no allocator interface), or a
  * latency-critical path on which an allocation, which may synchronise the
  * device, is not allowed.  The caller still passes every input and output;
- * arguments, layouts, results and errors are those of gqa_attn_decode.
+ * arguments, layouts, results and argument checks are those of
+ * gqa_attn_decode (both run the same validation), except that a problem too
+ * large for the static scratch returns GQA_ERR_WORKSPACE_TOO_SMALL.
  *
- * The split-KV partials live in a fixed 64 MiB array of static device memory
- * inside the library, which every GPU that loads the library holds until the
- * process exits.  A problem whose partials (gqa_attn_decode_workspace_size)
- * exceed 64 MiB is rejected with GQA_ERR_WORKSPACE_TOO_SMALL; a larger
- * kv_split needs fewer partials.  The first call on each device looks up the
- * array's device address (with that device current) and zeroes the array
- * once (a synchronous cudaMemset), so make that first call before any stream
- * capture.  All calls share the array; each leaves its counter block at zero,
- * as the next call needs it.  Calls that overlap on the GPU (e.g. on two
- * streams) race, so order them on one stream or with events.  It allocates
- * nothing.
+ * The split counters and partials live in a fixed 64 MiB array of static
+ * device memory inside the library, which every GPU that loads the library
+ * holds until the process exits.  A problem whose workspace
+ * (gqa_attn_decode_workspace_size) exceeds 64 MiB is rejected with
+ * GQA_ERR_WORKSPACE_TOO_SMALL; a larger kv_split needs fewer partials.
+ * The first call on each device looks up the array's device address, with
+ * that device current (a host-side runtime query; make that first call
+ * before any stream capture).  Every call then clears the counter block at
+ * the front of the array with cudaMemsetAsync on `stream`, before its decode
+ * kernel on the same stream, because the array keeps whatever the previous
+ * call left there.  All calls share the array: calls that overlap on the
+ * GPU (e.g. on two streams) race, so order them on one stream or with
+ * events.  It allocates nothing.
  */
 int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,

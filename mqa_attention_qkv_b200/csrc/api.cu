@@ -127,6 +127,23 @@ int decode_split_len(int B, int nh, int nkv, int cache_cap, int kv_split) {
   return kv_split ? kv_split : auto_split(B, nkv, decode_n_hgrp(nh, nkv), cache_cap);
 }
 
+int decode_check_args(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens, int B,
+                      int nh, int nkv, int hd, int cap, int kv_split, const void* out, int dtype) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+  if (B < 0 || nh <= 0 || nkv <= 0 || cap <= 0) return GQA_ERR_INVALID_ARG;
+  if (nh % nkv != 0) return GQA_ERR_INVALID_ARG;
+  if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;
+  if (kv_split > 0 && (cap + kv_split - 1) / kv_split > kMaxSplits) return GQA_ERR_INVALID_ARG;
+  if (!hd_ok(hd)) return GQA_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * nkv * cap * hd > kMaxElems || B > 65535 || nkv > 65535 || (long long)B * nkv * cap >= kMaxRows)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return GQA_OK;
+  if (!q || !k_cache || !v_cache || !kv_lens || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned4(kv_lens))
+    return GQA_ERR_MISALIGNED;
+  return GQA_OK;
+}
+
 DecodeParams decode_params(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens,
                            int B, int nh, int nkv, int hd, int cap, int kv_split, void* out, void* workspace,
                            int* err) {
@@ -282,20 +299,12 @@ int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,
                     const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,
                     int cache_cap, int kv_split, void* out, void* workspace,
                     size_t workspace_bytes, int dtype, void* stream) {
-  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
-  if (B < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0) return GQA_ERR_INVALID_ARG;
-  if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
-  if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;
-  if (kv_split > 0 && (cache_cap + kv_split - 1) / kv_split > kMaxSplits) return GQA_ERR_INVALID_ARG;
-  if (!hd_ok(head_dim)) return GQA_ERR_UNSUPPORTED_SHAPE;
-  if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems || B > 65535 || n_kv_heads > 65535 ||
-      (long long)B * n_kv_heads * cache_cap >= kMaxRows)
-    return GQA_ERR_UNSUPPORTED_SHAPE;
-  if (B == 0) return GQA_OK;
-  if (!q || !k_cache || !v_cache || !kv_lens || !out || !workspace) return GQA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
-      !aligned16(workspace) || !aligned4(kv_lens))
-    return GQA_ERR_MISALIGNED;
+  if (const int v = gqa::decode_check_args(q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim,
+                                           cache_cap, kv_split, out, dtype);
+      v != GQA_OK || B == 0)
+    return v;
+  if (!workspace) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
   const size_t need = gqa_attn_decode_workspace_size(B, n_heads, n_kv_heads, head_dim, cache_cap, kv_split);
   if (workspace_bytes < need) return GQA_ERR_WORKSPACE_TOO_SMALL;
   int st;

@@ -12,7 +12,8 @@
 // The scratch array is kNoAllocScratchBytes (64 MiB) of device memory that
 // every GPU which loads this library holds until the process exits.  Its
 // device address is looked up once per device (cudaGetSymbolAddress with that
-// device current) on the first call made on that device.
+// device current) on the first call made on that device; each call clears the
+// split counters at its front with an asynchronous memset on its own stream.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -36,9 +37,10 @@ struct ScratchSlot {
 };
 ScratchSlot g_slot[kMaxDevices];
 
-// Device address of g_decode_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in: a kernel given it would fault (or
-// silently use the wrong memory), so the real address is looked up here.
+// Device address of g_decode_scratch on the current device, looked up once
+// per device with that device current.  In host code the array's name is only
+// a host-side stand-in: a kernel given it would fault (or silently use the
+// wrong memory), so the real address is taken from the runtime.
 void* scratch_ptr() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -48,8 +50,6 @@ void* scratch_ptr() {
   ScratchSlot& s = g_slot[dev];
   std::call_once(s.once, [&] {
     s.status = cudaGetSymbolAddress(&s.ptr, g_decode_scratch);
-    // the split counters at the front must start at zero; every call leaves them so
-    if (s.status == cudaSuccess) s.status = cudaMemset(s.ptr, 0, kNoAllocScratchBytes);
     if (s.status != cudaSuccess) {
       s.ptr = nullptr;
       cudaGetLastError();
@@ -65,21 +65,13 @@ extern "C" {
 int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* kv_lens, int B, int n_heads, int n_kv_heads, int head_dim,
                             int cache_cap, int kv_split, void* out, int dtype, void* stream) {
-  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
-  if (B < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0) return GQA_ERR_INVALID_ARG;
-  if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
-  if (kv_split < 0 || (kv_split > 0 && kv_split % 64)) return GQA_ERR_INVALID_ARG;
-  if (head_dim != 32 && head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED_SHAPE;
-  if ((long long)B * n_kv_heads * cache_cap * head_dim > (1ll << 40) || B > 65535 || n_kv_heads > 65535 ||
-      (long long)B * n_kv_heads * cache_cap >= (1ll << 31))   // 32-bit cache row coordinates
-    return GQA_ERR_UNSUPPORTED_SHAPE;
-  if (B == 0) return GQA_OK;
-  if (!q || !k_cache || !v_cache || !kv_lens || !out) return GQA_ERR_INVALID_ARG;
-  const auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-  if (!a16(q) || !a16(k_cache) || !a16(v_cache) || !a16(out) || (reinterpret_cast<uintptr_t>(kv_lens) & 3u))
-    return GQA_ERR_MISALIGNED;
-  // The problem's partials must fit the fixed scratch; larger problems are
-  // rejected (a larger kv_split needs fewer partials).
+  // the same validation as gqa_attn_decode, minus the workspace arguments
+  if (const int v = gqa::decode_check_args(q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim,
+                                           cache_cap, kv_split, out, dtype);
+      v != GQA_OK || B == 0)
+    return v;
+  // The problem's counters and partials must fit the fixed scratch; larger
+  // problems are rejected (a larger kv_split needs fewer partials).
   const size_t need = gqa_attn_decode_workspace_size(B, n_heads, n_kv_heads, head_dim, cache_cap, kv_split);
   if (need == 0 || need > kNoAllocScratchBytes) return GQA_ERR_WORKSPACE_TOO_SMALL;
   int* err = nullptr;
@@ -88,15 +80,23 @@ int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
   void* ws = scratch_ptr();
   if (!ws) return GQA_ERR_NO_DEVICE;
 
-  // The scratch starts with the per-(sequence, KV head) split counters, which
-  // must be zero: the set-up above zeroes the array once and every call leaves
-  // the counters at zero again.  The partials need no clearing (each one the
-  // merge reads is written by the same call first).  Calls that overlap on the
-  // GPU (other streams) share the array and race; order them on one stream or
-  // with events.
+  // The scratch starts with the per-(sequence, KV head, head group) split
+  // counters, which must start at zero.  The array keeps whatever the last
+  // call left, so they are cleared here, on the caller's stream, ahead of the
+  // decode kernel (stream order makes the clear finish first whatever kind of
+  // stream the caller uses).  The partials need no clearing: every partial
+  // the merge reads is written by the same call first.  Calls that overlap on
+  // the GPU (other streams) share the array and race; order them on one
+  // stream or with events.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t counter_bytes =
+      gqa::decode_counter_bytes(B, n_kv_heads, gqa::decode_n_hgrp(n_heads, n_kv_heads));
+  if (cudaMemsetAsync(ws, 0, counter_bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_LAUNCH_FAILED;
+  }
   const gqa::DecodeParams p = gqa::decode_params(q, k_cache, v_cache, kv_lens, B, n_heads, n_kv_heads, head_dim,
                                                  cache_cap, kv_split, out, ws, err);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   gqa::count_launches(gqa::launch_decode(p, dtype == GQA_BF16, s, &e));
   if (e != cudaSuccess) {

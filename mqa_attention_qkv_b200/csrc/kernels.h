@@ -141,6 +141,10 @@ bool make_tmap_packed(void* map, const void* base, uint64_t tokens, int heads, i
 int device_check(int** err);  // GQA_OK, or the status for the current device
 void count_launches(int n);
 int decode_split_len(int B, int nh, int nkv, int cache_cap, int kv_split);
+// Host-side validation shared by the decode entry points (everything but the
+// workspace): GQA_OK or the status to return.  B == 0 passes (a no-op).
+int decode_check_args(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens, int B,
+                      int nh, int nkv, int hd, int cap, int kv_split, const void* out, int dtype);
 // Decode parameters over a workspace laid out as counters, then partials.
 DecodeParams decode_params(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens,
                            int B, int nh, int nkv, int hd, int cap, int kv_split, void* out, void* workspace,

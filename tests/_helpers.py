@@ -4,16 +4,18 @@ and the tolerance gates.
 Gates (fixed by the spec of the path; readings stated in the design notes):
 
 * float32: max|err| <= 1e-4 * max|ref| over the output tensor.
-* bfloat16: "2e-2 absolute on unit-scale outputs".  The scale of an output is
-  taken per output row (the head_dim-vector of one head at one token) as its
-  RMS, and an element larger than that scale is held to 2e-2 of itself (no
-  bf16 value is closer than 2^-8 relative to its reference):
-  |err| <= 2e-2 * max(RMS(ref_row), |ref|).  On a unit-scale row with
-  elements up to 1 this is exactly 2e-2 absolute; decode outputs (RMS ~0.05)
-  are held to ~1e-3.  Where V has outlier channels (x20 in the long-context
-  workload) an output channel has a scale of its own, so attention outputs
-  compared as [rows, hd] also take the RMS of their (head, channel) over the
-  compared rows into the max.
+* bfloat16: "2e-2 absolute on unit-scale outputs", held on every element and
+  never loosened above it: |err| <= 2e-2 * min(1, RMS(ref_row)), where a row
+  is the head_dim-vector of one head at one token.  On a row of unit (or
+  larger) scale this is the spec's 2e-2 absolute; on a smaller row it is the
+  same 2% of the row's own scale (decode outputs, RMS ~0.05, are held to
+  ~1e-3), so every output tensor also meets max|err| <= 2e-2 * max|ref|.
+  A correct bf16 result stays well inside it: one rounding costs at most
+  2^-9 of the value, so an element up to ~10x its row's RMS still fits.
+  ``col_scale`` names channels that the inputs scaled on purpose (the
+  long-context workload multiplies 0.1% of V's channels by 20); attention
+  is linear in V, so such an output channel is that factor times a
+  unit-scale output, and its row RMS and its bound are taken on that scale.
 * KV-cache layout: bit-exact (integer inputs with exact fp32 sums).
 """
 from __future__ import annotations
@@ -52,10 +54,10 @@ def bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy().view(np.uint32)
 
 
-def gate(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = "", heads=None):
-    """Assert the spec's tolerance; rows are the last axis.  ``heads`` (one id
-    per row of a 2-D ``[rows, hd]`` comparison) groups rows by attention head
-    so that each (head, channel) also gets its own RMS scale."""
+def gate(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = "", col_scale=None):
+    """Assert the spec's tolerance; rows are the last axis.  ``col_scale``
+    (broadcastable to ``ref``) is the factor by which the inputs scaled an
+    output channel on purpose (1 elsewhere)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
@@ -66,20 +68,15 @@ def gate(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = "", heads=Non
         worst = float(err.max()) if err.size else 0.0
         assert worst <= bound, f"{what}: max|err| {worst:.3e} > {bound:.3e}"
         return worst / bound if bound else 0.0
-    rms = np.sqrt(np.mean(ref * ref, axis=-1, keepdims=True))
-    scale = np.maximum(rms, np.abs(ref))
-    if heads is not None:
-        heads = np.asarray(heads)
-        col = np.zeros_like(ref)
-        for hid in np.unique(heads):
-            sel = heads == hid
-            col[sel] = np.sqrt(np.mean(ref[sel] ** 2, axis=0, keepdims=True))
-        scale = np.maximum(scale, col)
-    lim = BF16_TOL * np.maximum(scale, 1e-6)
-    ratio = err / lim
-    worst = float(ratio.max()) if ratio.size else 0.0
-    if worst > 1.0:
-        idx = np.unravel_index(np.argmax(ratio), ratio.shape)
-        raise AssertionError(f"{what}: err {err[idx]:.3e} at {idx} exceeds 2e-2 x row RMS "
-                             f"{float(rms[idx[:-1]][0]):.3e} (ref {ref[idx]:.4f}, got {got[idx]:.4f})")
-    return worst
+    scale = np.ones_like(ref) if col_scale is None else np.broadcast_to(np.asarray(col_scale, np.float64), ref.shape)
+    unit = ref / scale
+    rms = np.sqrt(np.mean(unit * unit, axis=-1, keepdims=True))
+    lim = BF16_TOL * scale * np.minimum(1.0, rms)
+    over = err > lim
+    if np.any(over):
+        ratio = np.where(lim > 0, err / np.where(lim > 0, lim, 1.0), np.inf)
+        idx = np.unravel_index(np.argmax(np.where(over, ratio, -1.0)), ratio.shape)
+        raise AssertionError(f"{what}: err {err[idx]:.3e} at {idx} exceeds 2e-2 x min(1, row RMS) = {lim[idx]:.3e} "
+                             f"(row RMS {float(rms[idx[:-1]][0]):.3e}, ref {ref[idx]:.4f}, got {got[idx]:.4f})")
+    ok = lim > 0
+    return float((err[ok] / lim[ok]).max()) if np.any(ok) else 0.0

@@ -102,6 +102,27 @@ def test_decode_rejects(kw, code):
     assert _decode(**kw) == code
 
 
+def _decode_noalloc(**kw):
+    a = dict(q=P, k=P, v=P, lens=P, B=2, nh=4, nkv=2, hd=64, cap=16, split=0, out=P, dtype=1, stream=None)
+    a.update(kw)
+    return gqa.lib().gqa_attn_decode_noalloc(a["q"], a["k"], a["v"], a["lens"], a["B"], a["nh"], a["nkv"],
+                                             a["hd"], a["cap"], a["split"], a["out"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=None), dict(k=None), dict(v=None), dict(lens=None), dict(out=None), dict(split=100),
+    dict(split=-64), dict(nh=4, nkv=3), dict(nkv=0), dict(B=-1), dict(cap=0), dict(hd=48),
+    dict(q=MIS), dict(out=MIS), dict(lens=P + 2), dict(dtype=7),
+    dict(cap=64 * 600, split=64),                                    # 600 splits > 512
+    dict(B=2, nkv=2, nh=4, cap=1 << 29, split=1 << 21),              # 2^31 cache rows
+])
+def test_noalloc_decode_validates_like_decode(kw):
+    """Both decode entry points run the same argument checks."""
+    want = _decode(**kw)
+    assert want < 0
+    assert _decode_noalloc(**kw) == want
+
+
 def _meanpool(**kw):
     a = dict(w=P, hidden=64, nh=8, nkv=2, hd=64, out=P + (1 << 24), dtype=1, stream=None)
     a.update(kw)

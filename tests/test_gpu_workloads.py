@@ -188,6 +188,12 @@ def test_long_prefill_outliers(nkv, causal):
     rows = [(int(r.integers(B)), h, int(r.integers(S))) for h in range(nh) for _ in range(8)]
     rows += [(0, 0, 0), (1, nh - 1, S - 1), (0, 3, 127), (1, 5, 128), (0, 7, 4095)]
     want = ref.prefill_attention(q.f64, k.f64, v.f64, np.full(B, S), causal, rows=rows)
+    # V's outlier channels (x20) give the output channels of every query head
+    # reading that KV head a 20x scale (attention is linear in V)
+    vscale = np.ones(nkv * hd)
+    vscale[W.outlier_channels(nkv * hd, 0.001, wl.seed + nkv, 2)] = 20.0
+    vscale = vscale.reshape(nkv, hd)
+    g = nh // nkv
     gate(np.stack([got[b, s, h] for b, h, s in rows]), want, "bf16", f"long prefill nkv={nkv} causal={causal}",
-         heads=[h for _, h, _ in rows])
+         col_scale=np.stack([vscale[h // g] for _, h, _ in rows]))
     assert np.all(np.isfinite(got))
