@@ -251,6 +251,41 @@ int gqa_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_ca
                             int cache_cap, int kv_split, void* out, int dtype, void* stream);
 
 /*
+ * gqa_o_proj_residual - the attention layer's output projection with the
+ * residual add (the step after a4 / a5).
+ *
+ * Source: the "custom op overhead" gist (youkaichao), toy model:
+ * LlamaAttention.forward ends in output = self.output_projection(attn_output),
+ * a linear layer from the n_heads * head_dim concatenated head outputs back to
+ * the hidden size, and LlamaDecoderLayer adds that output to the residual
+ * stream.  (The toy's linear layers carry a bias; the layer here has none, as
+ * W_qkv has none.)
+ *
+ *   attn      [T, n_heads, head_dim] dtype: per token the heads in order,
+ *             i.e. [T, n_heads * head_dim] (gqa_attn_prefill's out
+ *             [B, S, n_heads, head_dim] with T = B * S, or gqa_attn_decode's
+ *             out [B, n_heads, head_dim] with T = B)
+ *   w_o       [hidden, n_heads * head_dim] dtype (nn.Linear storage: y = x w^T)
+ *   residual  [T, hidden] dtype, or NULL for none
+ *   out       [T, hidden] dtype: out = attn . w_o^T + residual, accumulated in
+ *             float32 (the residual added in float32) and rounded once.  out
+ *             may be the residual buffer itself (an in-place update of the
+ *             residual stream); it must not overlap attn or w_o.
+ *
+ * bf16 with hidden % 8 == 0 runs on the tensor cores (tcgen05): 128-token
+ * tiles, or for T <= 64 tiles whose rows are 128 rows of w_o with the
+ * reduction split over a thread-block cluster.  float32 (FFMA, no TF32) and
+ * other bf16 widths run a SIMT kernel.  T == 0 is a no-op.
+ * Errors: GQA_ERR_INVALID_ARG (null pointers, non-positive sizes, out
+ * overlapping attn or w_o, or partly overlapping the residual),
+ * GQA_ERR_UNSUPPORTED_SHAPE (head_dim, sizes), GQA_ERR_MISALIGNED,
+ * GQA_ERR_UNSUPPORTED_DTYPE and the device/launch statuses.  Asynchronous on
+ * `stream`; allocates nothing.
+ */
+int gqa_o_proj_residual(const void* attn, const void* w_o, const void* residual, int T, int n_heads,
+                        int head_dim, int hidden, void* out, int dtype, void* stream);
+
+/*
  * gqa_meanpool_kv_heads - MHA -> GQA weight transform ("MHA -> GQA: 提升 LLM
  * 推理效率", section 4.3: the new KV projection of each group of heads is
  * initialised by mean pooling the group's projections).
@@ -325,6 +360,26 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
  * normally.  n = 0 clears pending injections; n < 0 is GQA_ERR_INVALID_ARG.
  */
 int gqa_debug_inject_launch_failures(int n);
+
+/*
+ * gqa_debug_set_wait_limit_ns - testing aid for the bounded waits: every
+ * pipeline wait in the library's kernels gives up after this many
+ * nanoseconds (ns = 0 restores the default of 2 s), sets
+ * GQA_DEVERR_WAIT_TIMEOUT, lets the copies and MMAs its CTA has in flight
+ * land, frees its tensor memory and returns.  Applies to the current device
+ * from the next launch on; synchronous (a host-to-device copy).
+ */
+int gqa_debug_set_wait_limit_ns(uint64_t ns);
+
+/*
+ * gqa_debug_skip_next_kv_tile - testing aid (a wait that runs out, made on
+ * purpose): in the next gqa_attn_prefill call that takes the head_dim-64
+ * bf16 tensor-core kernel, the first CTA's copy thread does not load key
+ * tile `tile` (of 128 keys), so the waits for it run out after the wait
+ * limit; the call still returns and later calls run normally.  tile = -1
+ * disarms; tile < -1 is GQA_ERR_INVALID_ARG.
+ */
+int gqa_debug_skip_next_kv_tile(int tile);
 
 /* Human-readable text of a gqa_status value (static storage). */
 const char* gqa_status_string(int status);

@@ -17,7 +17,8 @@ __all__ = [
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
-    "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures", "EXPORTED_SYMBOLS",
+    "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures", "gqa_o_proj_residual",
+    "gqa_debug_set_wait_limit_ns", "gqa_debug_skip_next_kv_tile", "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -27,7 +28,8 @@ EXPORTED_SYMBOLS = (
     "qkv_rope_project", "gqa_attn_prefill", "gqa_attn_decode",
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
-    "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures",
+    "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures", "gqa_o_proj_residual",
+    "gqa_debug_set_wait_limit_ns", "gqa_debug_skip_next_kv_tile",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +80,12 @@ def lib() -> ctypes.CDLL:
     L.gqa_attn_decode_paged.restype = i32
     L.gqa_attn_prefill_varlen.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     L.gqa_attn_prefill_varlen.restype = i32
+    L.gqa_o_proj_residual.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp]
+    L.gqa_o_proj_residual.restype = i32
+    L.gqa_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    L.gqa_debug_set_wait_limit_ns.restype = i32
+    L.gqa_debug_skip_next_kv_tile.argtypes = [i32]
+    L.gqa_debug_skip_next_kv_tile.restype = i32
     L.gqa_debug_inject_launch_failures.argtypes = [i32]
     L.gqa_debug_inject_launch_failures.restype = i32
     _LIB = L
@@ -235,6 +243,26 @@ def gqa_attn_decode_paged(q, k_pages, v_pages, block_table, kv_lens, out, worksp
     _check("gqa_attn_decode_paged", lib().gqa_attn_decode_paged(*args))
 
 
+def gqa_o_proj_residual(attn, w_o, out, residual=None, stream=None) -> None:
+    """Output projection + residual: attn [..., nh, hd] (the heads of each
+    token in order), w_o [hidden, nh*hd], residual None or [..., hidden] ->
+    out [..., hidden] = attn . w_o^T + residual.  ``out`` may be ``residual``
+    (in place)."""
+    *lead, nh, hd = attn.shape
+    T = 1
+    for d in lead:
+        T *= int(d)
+    hidden = w_o.shape[0]
+    dt = attn.dtype
+    oshape = (*lead, hidden)
+    args = (
+        _ptr(attn, dt, name="attn"), _ptr(w_o, dt, (hidden, nh * hd), "w_o"),
+        _ptr(residual, dt, oshape, "residual"), T, nh, hd, hidden,
+        _ptr(out, dt, oshape, "out"), _dtype_code(attn), _stream(stream),
+    )
+    _check("gqa_o_proj_residual", lib().gqa_o_proj_residual(*args))
+
+
 def gqa_device_error() -> int:
     """Read and clear the device error word (synchronises the device)."""
     v = ctypes.c_int(0)
@@ -246,6 +274,18 @@ def gqa_debug_inject_launch_failures(n: int) -> None:
     """Testing aid: the next ``n`` compute calls fail as a failed launch would
     (GQAError with status GQA_ERR_LAUNCH_FAILED), launching nothing."""
     _check("gqa_debug_inject_launch_failures", lib().gqa_debug_inject_launch_failures(int(n)))
+
+
+def gqa_debug_set_wait_limit_ns(ns: int) -> None:
+    """Testing aid: pipeline waits give up after ``ns`` nanoseconds (0 = the
+    default 2 s) on the current device, from the next launch on."""
+    _check("gqa_debug_set_wait_limit_ns", lib().gqa_debug_set_wait_limit_ns(int(ns)))
+
+
+def gqa_debug_skip_next_kv_tile(tile: int) -> None:
+    """Testing aid: the next head_dim-64 bf16 prefill leaves key tile ``tile``
+    unloaded in its first CTA, so that the waits on it run out (-1 disarms)."""
+    _check("gqa_debug_skip_next_kv_tile", lib().gqa_debug_skip_next_kv_tile(int(tile)))
 
 
 def gqa_launch_count() -> int:

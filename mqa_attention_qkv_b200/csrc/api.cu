@@ -11,8 +11,10 @@
 
 namespace {
 
-// Device error word: one per device, in the library's static device memory.
-__device__ int g_device_error;
+// Device error block, one per device in the library's static device memory:
+// word 0 the GQA_DEVERR_* bits, words 2-3 a wait-limit override in ns (0 =
+// the default; set only by gqa_debug_set_wait_limit_ns).
+__device__ __align__(16) int g_device_error[4];
 
 constexpr int kMaxDevices = 64;
 
@@ -58,6 +60,9 @@ const DeviceInfo* device_info(int* status) {
 // compute calls that pass validation report GQA_ERR_LAUNCH_FAILED without
 // launching anything.
 std::atomic<int> g_inject_failures{0};
+// gqa_debug_skip_next_kv_tile: K tile + 1 that the next head-dim-64 prefill's
+// first CTA does not load (0 = none); taken by that call.
+std::atomic<int> g_skip_kv_tile{0};
 
 bool take_injected_failure() {
   int n = g_inject_failures.load(std::memory_order_relaxed);
@@ -248,6 +253,7 @@ int gqa_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
 
   gqa::PrefillParams p{q, k_cache, v_cache, q_positions, kv_lens, B, S, n_heads, n_kv_heads,
                        head_dim, cache_cap, causal ? 1 : 0, out, d->err};
+  if (dtype == GQA_BF16 && head_dim == 64) p.dbg_skip_tile1 = g_skip_kv_tile.exchange(0);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // head_dim 64: two CTAs per SM (measured fastest there); 128: two query tiles per CTA
   if (dtype == GQA_BF16 && head_dim == 64) return launch_status(gqa::launch_prefill_pair(p, s));
@@ -360,7 +366,61 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
   return launch_status(e, n);
 }
 
+int gqa_o_proj_residual(const void* attn, const void* w_o, const void* residual, int T, int n_heads,
+                        int head_dim, int hidden, void* out, int dtype, void* stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED_DTYPE;
+  if (T < 0 || n_heads <= 0 || hidden <= 0) return GQA_ERR_INVALID_ARG;
+  if (!hd_ok(head_dim)) return GQA_ERR_UNSUPPORTED_SHAPE;
+  const long long K = (long long)n_heads * head_dim;
+  if ((long long)T * K > kMaxElems || (long long)T * hidden > kMaxElems || K * hidden > kMaxElems ||
+      K >= kMaxRows || (long long)T >= kMaxRows)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return GQA_OK;
+  if (!attn || !w_o || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(attn) || !aligned16(w_o) || !aligned16(out) || (residual && !aligned16(residual)))
+    return GQA_ERR_MISALIGNED;
+  // out may be the residual itself (in place); no other overlap is allowed
+  const size_t es = dtype == GQA_BF16 ? 2 : 4;
+  const char* ob = static_cast<const char*>(out);
+  const size_t ob_n = (size_t)T * hidden * es;
+  auto overlaps = [&](const void* q, size_t n) {
+    const char* qb = static_cast<const char*>(q);
+    return qb < ob + ob_n && ob < qb + n;
+  };
+  if (overlaps(attn, (size_t)T * K * es) || overlaps(w_o, (size_t)K * hidden * es) ||
+      (residual && residual != out && overlaps(residual, ob_n)))
+    return GQA_ERR_INVALID_ARG;
+  int st;
+  const DeviceInfo* d = compute_device(&st);
+  if (!d) return st;
+
+  const gqa::OprojParams p{attn, w_o, residual, out, T, (int)K, hidden, d->err};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == GQA_BF16 && hidden % 8 == 0) {
+    if (T <= 64) return launch_status(gqa::launch_oproj_smallt(p, d->num_sms, s));
+    return launch_status(gqa::launch_oproj_tc(p, d->num_sms, s));
+  }
+  return launch_status(gqa::launch_oproj_simt(p, dtype == GQA_BF16, s));
+}
+
 uint64_t gqa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int gqa_debug_set_wait_limit_ns(uint64_t ns) {
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (!d) return st;
+  if (cudaMemcpy(d->err + 2, &ns, sizeof(ns), cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_LAUNCH_FAILED;
+  }
+  return GQA_OK;
+}
+
+int gqa_debug_skip_next_kv_tile(int tile) {
+  if (tile < -1) return GQA_ERR_INVALID_ARG;
+  g_skip_kv_tile.store(tile + 1);
+  return GQA_OK;
+}
 
 int gqa_debug_inject_launch_failures(int n) {
   if (n < 0) return GQA_ERR_INVALID_ARG;

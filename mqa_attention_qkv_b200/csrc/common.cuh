@@ -52,11 +52,19 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
 }
 
 // ---------------------------------------------------------------------------
-// Time-bounded waits.  A wait that has not succeeded after kWaitLimitNs gives
+// Time-bounded waits.  A wait that has not succeeded after its limit gives
 // up, records GQA_DEVERR_WAIT_TIMEOUT and returns false; the caller then skips
-// the rest of its work and goes straight to its teardown.
+// the rest of its work and goes straight to its teardown.  The limit is
+// kWaitLimitNs unless the device error word's companion (words 2-3 of the
+// 16-byte block `err` points at) holds a shorter one, which the failure-path
+// tests set through gqa_debug_set_wait_limit_ns.
 // ---------------------------------------------------------------------------
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint64_t wait_limit_ns(const int* err) {
+  const uint64_t v = err ? *reinterpret_cast<const volatile uint64_t*>(err + 2) : 0ull;
+  return v ? v : kWaitLimitNs;
+}
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
@@ -102,11 +110,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
+  uint64_t limit = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (err && (*reinterpret_cast<volatile int*>(err) & GQA_DEVERR_WAIT_TIMEOUT)) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (!limit) limit = wait_limit_ns(err);
+      if (global_timer_ns() - t0 > limit) {
+        raise_error(err, GQA_DEVERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Teardown wait for work this thread itself issued (copies or MMAs in
+// flight), which completes on its own: bounded by the limit alone, not cut
+// short when another wait has already given up, so that a role that stops
+// early still lets its asynchronous work land before shared memory or TMEM
+// is released.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int* err) {
+  const uint64_t t0 = global_timer_ns();
+  uint64_t limit = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u) {
+      if (!limit) limit = wait_limit_ns(err);
+      if (global_timer_ns() - t0 > limit) {
         raise_error(err, GQA_DEVERR_WAIT_TIMEOUT);
         return false;
       }

@@ -21,6 +21,16 @@ struct QkvParams {
   int* err;
 };
 
+// Output projection with residual: out[T, N] = x[T, K] . w[N, K]^T (+ residual[T, N]).
+struct OprojParams {
+  const void* x;          // [T, K]   attention output, heads concatenated (K = nh * hd)
+  const void* w;          // [N, K]   W_o, nn.Linear layout
+  const void* residual;   // [T, N] or nullptr
+  void* out;              // [T, N]   may be the residual itself (in place)
+  int T, K, N;
+  int* err;
+};
+
 struct PrefillParams {
   const void* q;          // [B, nh, S, hd]
   const void* k_cache;    // [B, nkv, cap, hd]
@@ -37,6 +47,10 @@ struct PrefillParams {
   const int32_t* cu_q;
   const int32_t* cu_k;
   int total_q;
+  // failure-path testing (gqa_debug_skip_next_kv_tile): K tile + 1 that the
+  // first CTA's TMA thread does not load, so that the waits on it run out;
+  // 0 = none
+  int dbg_skip_tile1;
 };
 
 struct DecodeParams {
@@ -90,6 +104,12 @@ cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t
 // Tensor-core (tcgen05 + TMA) kernels, bf16 only.
 cudaError_t launch_qkv_tc(const QkvParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_qkv_smallm(const QkvParams& p, int num_sms, cudaStream_t st);  // B*S <= 64
+// Output projection + residual: tcgen05 GEMM (128-token tiles) and, for at
+// most 64 tokens, W-streaming tcgen05 tiles (W rows as M, tokens as N) with
+// the reduction dimension split over a thread-block cluster; SIMT for fp32.
+cudaError_t launch_oproj_tc(const OprojParams& p, int num_sms, cudaStream_t st);
+cudaError_t launch_oproj_smallt(const OprojParams& p, int num_sms, cudaStream_t st);   // T <= 64
+cudaError_t launch_oproj_simt(const OprojParams& p, bool bf16, cudaStream_t st);
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
 cudaError_t launch_prefill_fa(const PrefillParams& p, cudaStream_t st);    // head_dim 64/128, 2 Q tiles/CTA
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128

@@ -8,6 +8,8 @@
 //                  positions of one head; decode: 16 of the g heads of one KV
 //                  head over one key split, writing an unnormalised partial)
 //  decode_combine  log-sum-exp merge of the decode partials
+//  oproj_simt      output projection + residual, one output element per
+//                  thread (float32, and bf16 widths the tensor path skips)
 #include "common.cuh"
 #include "kernels.h"
 
@@ -309,6 +311,36 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p) {
   for (int d = 0; d < PER; ++d) out[lane + 32 * d] = from_f32<T>(o[d] * inv);
 }
 
+// ---------------------------------------------------------------------------
+// oproj_simt: out[t, n] = sum_k x[t, k] w[n, k] (+ residual[t, n]); a block of
+// 128 threads takes 128 consecutive outputs n of one token t and stages the
+// token's row of x through shared memory in chunks.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void __launch_bounds__(128) oproj_simt_kernel(OprojParams p) {
+  constexpr int CH = 256;
+  __shared__ float xs[CH];
+  const int n = blockIdx.x * 128 + threadIdx.x;
+  const T* w = static_cast<const T*>(p.w) + (size_t)(n < p.N ? n : 0) * p.K;
+  for (int t = blockIdx.y; t < p.T; t += gridDim.y) {
+    const T* x = static_cast<const T*>(p.x) + (size_t)t * p.K;
+    float acc = 0.f;
+    for (int k0 = 0; k0 < p.K; k0 += CH) {
+      const int kn = min(CH, p.K - k0);
+      __syncthreads();
+      for (int k = threadIdx.x; k < kn; k += 128) xs[k] = to_f32(x[k0 + k]);
+      __syncthreads();
+      if (n < p.N)
+        for (int k = 0; k < kn; ++k) acc = fmaf(xs[k], to_f32(w[k0 + k]), acc);
+    }
+    if (n < p.N) {
+      const size_t o = (size_t)t * p.N + n;
+      if (p.residual) acc += to_f32(static_cast<const T*>(p.residual)[o]);
+      static_cast<T*>(p.out)[o] = from_f32<T>(acc);
+    }
+  }
+}
+
 template <typename T>
 cudaError_t qkv_dispatch(const QkvParams& p, cudaStream_t st) {
   const int T_tot = p.B * p.S;
@@ -366,6 +398,15 @@ cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, cudaStream_t st
   PrefillParams none{};
   return bf16 ? attn_dispatch<__nv_bfloat16, true>(none, p, grid, p.hd, st)
               : attn_dispatch<float, true>(none, p, grid, p.hd, st);
+}
+
+cudaError_t launch_oproj_simt(const OprojParams& p, bool bf16, cudaStream_t st) {
+  dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)(p.T < 65535 ? p.T : 65535));
+  if (bf16)
+    oproj_simt_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(p);
+  else
+    oproj_simt_kernel<float><<<grid, 128, 0, st>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_decode_combine(const DecodeParams& p, bool bf16, cudaStream_t st) {

@@ -249,6 +249,11 @@ def test_binding_rejects_host_tensors():
                                   torch.zeros(1024, dtype=torch.uint8))
 
 
+def test_skip_tile_knob_validates_on_the_host():
+    assert gqa.lib().gqa_debug_skip_next_kv_tile(-2) == INVALID
+    assert gqa.lib().gqa_debug_skip_next_kv_tile(-1) == 0     # disarm
+
+
 def test_injected_launch_failures_are_reported_then_clear():
     """Host-side fault injection: after validation, the next n compute calls
     report GQA_ERR_LAUNCH_FAILED without launching; invalid calls are still

@@ -159,8 +159,13 @@ def test_qkv_gemm_protocol(n_tiles, n_kb):
 
 
 # ---------------------------------------------------------------- prefill_pair.cu
-def prefill_pair(n, KS=3, VS=2, warps=4, rescale_at=()):
-    bars = {"q_full": Bar(1), "s_full": Bar(1), "p_full": Bar(warps), "o_done": Bar(1), "drain": Bar(1)}
+def prefill_pair(n, KS=3, VS=2, warps=4, rescale_at=(), p_before_pv_wait=True):
+    """S | P | O in TMEM: the softmax frees S once it holds it in registers
+    (s_free), the MMA lane issues the next S at once, and the softmax writes
+    P(t) only after P(t-1).V has read the P columns.  ``p_before_pv_wait``
+    False plants the mistake of storing P without that wait."""
+    bars = {"q_full": Bar(1), "s_full": Bar(1), "s_free": Bar(warps), "p_full": Bar(warps), "o_done": Bar(1),
+            "drain": Bar(1)}
     for i in range(KS):
         bars[f"k_full{i}"], bars[f"k_empty{i}"] = Bar(1), Bar(1)
     for i in range(VS):
@@ -176,14 +181,18 @@ def prefill_pair(n, KS=3, VS=2, warps=4, rescale_at=()):
                 yield from ring_load("k", t + 2, KS, None)
             yield from ring_load("v", t, VS, None)
 
+    def issue_s(t):
+        yield ("wait", f"k_full{t % KS}", t // KS)
+        yield ("event", f"S{t}_start")
+        yield ("issue", f"S{t}", [f"k_empty{t % KS}", "s_full"])
+
     def mma():
         yield ("wait", "q_full", 0)
+        yield from issue_s(0)
         for t in range(n):
-            yield ("wait", f"k_full{t % KS}", t // KS)
-            if t > 0:                       # S/P columns free once P(t-1).V has read them
-                yield ("wait", "o_done", t - 1)
-            yield ("event", f"S{t}_start")
-            yield ("issue", f"S{t}", [f"k_empty{t % KS}", "s_full"])
+            if t + 1 < n:                   # S columns free once every warp holds S(t)
+                yield ("wait", "s_free", t)
+                yield from issue_s(t + 1)
             yield ("wait", "p_full", t)
             yield ("wait", f"v_full{t % VS}", t // VS)
             yield ("event", f"PV{t}_start")
@@ -195,8 +204,10 @@ def prefill_pair(n, KS=3, VS=2, warps=4, rescale_at=()):
         for t in range(n):
             yield ("wait", "s_full", t)
             yield ("event", f"readS{t}_{w}")
-            if t in rescale_at:
+            yield ("arrive", "s_free")
+            if t > 0 and (p_before_pv_wait or t in rescale_at):
                 yield ("wait", "o_done", t - 1)
+            if t in rescale_at:
                 yield ("event", f"rescale{t}_{w}")
             yield ("event", f"writeP{t}_{w}")
             yield ("arrive", "p_full")
@@ -209,20 +220,40 @@ def prefill_pair(n, KS=3, VS=2, warps=4, rescale_at=()):
     return roles, bars
 
 
+def check_pair(n, pos):
+    for t in range(n):
+        for w in range(4):
+            assert pos[("done", f"S{t}")] < pos[("event", f"readS{t}_{w}")]
+            assert pos[("event", f"writeP{t}_{w}")] < pos[("event", f"PV{t}_start")]
+            if t + 1 < n:   # S(t+1) overwrites S only after every warp read S(t)
+                assert pos[("event", f"readS{t}_{w}")] < pos[("event", f"S{t + 1}_start")]
+            if t > 0:       # P(t) overwrites P(t-1) only after P(t-1).V has read it
+                assert pos[("done", f"PV{t - 1}")] < pos[("event", f"writeP{t}_{w}")]
+                if ("event", f"rescale{t}_{w}") in pos:
+                    assert pos[("done", f"PV{t - 1}")] < pos[("event", f"rescale{t}_{w}")]
+        if t >= 3:
+            assert pos[("done", f"S{t - 3}")] < pos[("issue", f"load_k{t}")]
+    assert all(pos[("done", f"PV{n - 1}")] < pos[("event", f"readO_{w}")] for w in range(4))
+
+
 @pytest.mark.parametrize("n", [1, 2, 3, 6])
 def test_prefill_pair_protocol(n):
     for seed in range(60):
         roles, bars = prefill_pair(n, rescale_at=tuple(range(1, n, 2)))
-        pos = first(run(roles, bars, seed))
-        for t in range(n):
-            for w in range(4):
-                assert pos[("done", f"S{t}")] < pos[("event", f"readS{t}_{w}")]
-                assert pos[("event", f"writeP{t}_{w}")] < pos[("event", f"PV{t}_start")]
-                if t + 1 < n:   # P(t) lives in S's columns until P(t).V is done
-                    assert pos[("done", f"PV{t}")] < pos[("event", f"S{t + 1}_start")]
-            if t >= 3:
-                assert pos[("done", f"S{t - 3}")] < pos[("issue", f"load_k{t}")]
-        assert all(pos[("done", f"PV{n - 1}")] < pos[("event", f"readO_{w}")] for w in range(4))
+        check_pair(n, first(run(roles, bars, seed)))
+
+
+def test_prefill_pair_protocol_flags_p_written_before_pv_read_it():
+    """Planted mistake: P(t) stored without waiting for P(t-1).V."""
+    failed = False
+    for seed in range(200):
+        roles, bars = prefill_pair(4, p_before_pv_wait=False)
+        try:
+            check_pair(4, first(run(roles, bars, seed)))
+        except AssertionError:
+            failed = True
+            break
+    assert failed
 
 
 # ---------------------------------------------------------------- prefill_fa.cu

@@ -12,6 +12,8 @@ the rounded value, so input rounding is never counted as kernel error):
 * hidden states ``x``: N(0, 1)
 * fused weight ``W_qkv`` ``[(n_heads + 2 n_kv_heads) * head_dim, hidden]``
   (``nn.Linear`` storage, rows = output features): N(0, 0.02)
+* output projection ``W_o`` ``[hidden, n_heads * head_dim]``: N(0, 0.02); the
+  residual stream is the layer's own hidden states
 * decode queries and KV-cache rows: N(0, 1); cache slots at or beyond a
   sequence's KV length hold NaN, so any read of padding shows in the output
 * long-context Q/K/V: N(0, 1) with 0.1 % of the feature channels of each
@@ -165,6 +167,12 @@ def layer_inputs(shape: LayerShape, B: int, S: int, seed: int, dtype: str,
 def weight(shape: LayerShape, seed: int, dtype: str) -> Tensor:
     rng = np.random.default_rng([seed, 1])
     return _make(_normal(rng, (shape.n_qkv, shape.hidden), 0.02), dtype)
+
+
+def output_weight(shape: LayerShape, seed: int, dtype: str) -> Tensor:
+    """W_o ``[hidden, n_heads * head_dim]`` ~ N(0, 0.02), from its own stream."""
+    rng = np.random.default_rng([seed, 8])
+    return _make(_normal(rng, (shape.hidden, shape.n_heads * shape.head_dim), 0.02), dtype)
 
 
 def hidden_states(shape: LayerShape, B: int, S: int, seed: int, stream: int, dtype: str) -> Tensor:
