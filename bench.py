@@ -1,13 +1,16 @@
 """Benchmark of the fused-QKV + grouped-query attention path on B200.
 
-One step = the whole path over one batch of the TinyLlama-1.1B-shaped layer
-(hidden 2048, 32 query heads, 4 KV heads, head_dim 64, bf16, RoPE theta 1e4):
+One step = the whole attention layer over one batch of the TinyLlama-1.1B-
+shaped layer (hidden 2048, 32 query heads, 4 KV heads, head_dim 64, bf16,
+RoPE theta 1e4):
 
-  1. qkv_rope_project   prompt  x [4, 2048, 2048] -> q, K/V cache slots 0..2047
-  2. gqa_attn_prefill   causal, 4 x 2048 queries over their 2048 keys
-  3. qkv_rope_project   one new token per sequence at position 2048
-  4. gqa_attn_decode    4 sequences x 32 heads over 2049 cached keys
-                        (split-KV partials + log-sum-exp combine)
+  1. qkv_rope_project     prompt  x [4, 2048, 2048] -> q, K/V cache slots 0..2047
+  2. gqa_attn_prefill     causal, 4 x 2048 queries over their 2048 keys
+  3. gqa_o_proj_residual  attention output . W_o^T + x -> y [4, 2048, 2048]
+  4. qkv_rope_project     one new token per sequence at position 2048
+  5. gqa_attn_decode      4 sequences x 32 heads over 2049 cached keys
+                          (split-KV partials + log-sum-exp combine)
+  6. gqa_o_proj_residual  the new tokens' layer output
 
 value = tokens processed per second (8192 prompt + 4 decode tokens per step,
 summed over all GPUs).  Inputs are seeded synthetic tensors resident in HBM;
@@ -34,7 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "prefill attn TFLOPS & % BF16 peak; decode KV GB/s & % HBM; tokens/s per layer"
-WORKLOAD = dict(name="tinyllama-1.1b-layer-prefill4x2048+decode", B=4, S=2048, hidden=2048,
+WORKLOAD = dict(name="tinyllama-1.1b-attention-layer-prefill4x2048+decode", B=4, S=2048, hidden=2048,
                 n_heads=32, n_kv_heads=4, head_dim=64, theta=10000.0, cap=2112, causal=True)
 N_ROT = 4
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -175,6 +178,8 @@ def run_ours(args):
     for _ in range(N_ROT):
         st = dict(
             x=randn(B, S, D), w=randn(shape.n_qkv, D, std=0.02), x_dec=randn(B, 1, D),
+            w_o=randn(D, nh * hd, std=0.02),
+            y=torch.empty(B, S, D, dtype=bf, device=dev), y_dec=torch.empty(B, 1, D, dtype=bf, device=dev),
             q=torch.empty(B, nh, S, hd, dtype=bf, device=dev),
             kc=torch.zeros(B, nkv, cap, hd, dtype=bf, device=dev),
             vc=torch.zeros(B, nkv, cap, hd, dtype=bf, device=dev),
@@ -191,7 +196,7 @@ def run_ours(args):
     ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    names = ("qkv_prefill", "attn_prefill", "qkv_decode", "attn_decode")
+    names = ("qkv_prefill", "attn_prefill", "oproj_prefill", "qkv_decode", "attn_decode", "oproj_decode")
 
     def step(st, evs=None):
         def mark(i):
@@ -203,10 +208,15 @@ def run_ours(args):
         mark(1)
         gqa.gqa_attn_prefill(st["q"], st["kc"], st["vc"], lens, True, st["o"], stream=stream)
         mark(2)
-        gqa.qkv_rope_project(st["x_dec"], st["w"], pos_dec, nh, nkv, hd, wl["theta"], st["q_dec"], st["kc"], st["vc"], stream)
+        gqa.gqa_o_proj_residual(st["o"], st["w_o"], st["y"], residual=st["x"], stream=stream)
         mark(3)
-        gqa.gqa_attn_decode(st["q_dec"].view(B, nh, hd), st["kc"], st["vc"], lens_dec, st["o_dec"], ws, stream=stream)
+        gqa.qkv_rope_project(st["x_dec"], st["w"], pos_dec, nh, nkv, hd, wl["theta"], st["q_dec"], st["kc"], st["vc"], stream)
         mark(4)
+        gqa.gqa_attn_decode(st["q_dec"].view(B, nh, hd), st["kc"], st["vc"], lens_dec, st["o_dec"], ws, stream=stream)
+        mark(5)
+        gqa.gqa_o_proj_residual(st["o_dec"].view(B, 1, nh, hd), st["w_o"], st["y_dec"], residual=st["x_dec"],
+                                stream=stream)
+        mark(6)
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -219,7 +229,7 @@ def run_ours(args):
     barrier()
 
     # timed region: K steps; per-kernel events on the launching stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
@@ -245,10 +255,12 @@ def run_ours(args):
     flops = {
         "qkv_prefill": 2.0 * B * S * D * shape.n_qkv,
         "attn_prefill": 4.0 * B * nh * S * S * hd / 2,           # causal counted as half
+        "oproj_prefill": 2.0 * B * S * nh * hd * D,
     }
     bytes_ = {
         "qkv_decode": 2.0 * (shape.n_qkv * D + B * D + B * shape.n_qkv),
         "attn_decode": 2.0 * (2 * B * nkv * (S + 1) * hd + 2 * B * nh * hd),
+        "oproj_decode": 2.0 * (D * nh * hd + B * nh * hd + 2 * B * D),
     }
     mean_ms = {n: statistics.mean(v) for n, v in per_kernel.items()}
     dominant = max(mean_ms, key=mean_ms.get)
@@ -278,8 +290,8 @@ def run_ours(args):
     if not args.no_e2e:
         hx = [sets[i]["x"].cpu().pin_memory() for i in range(N_ROT)]
         hxd = [sets[i]["x_dec"].cpu().pin_memory() for i in range(N_ROT)]
-        ho = [torch.empty(B, S, nh, hd, dtype=bf).pin_memory() for _ in range(N_ROT)]
-        hod = [torch.empty(B, nh, hd, dtype=bf).pin_memory() for _ in range(N_ROT)]
+        ho = [torch.empty(B, S, D, dtype=bf).pin_memory() for _ in range(N_ROT)]
+        hod = [torch.empty(B, 1, D, dtype=bf).pin_memory() for _ in range(N_ROT)]
         hpos = pos.cpu().pin_memory()
         for st in sets:
             st["pos"] = torch.empty_like(pos)
@@ -306,8 +318,8 @@ def run_ours(args):
             ev_done[k].record(stream)
             with torch.cuda.stream(out_st):
                 out_st.wait_event(ev_done[k])
-                ho[k].copy_(st["o"], non_blocking=True)
-                hod[k].copy_(st["o_dec"], non_blocking=True)
+                ho[k].copy_(st["y"], non_blocking=True)         # the layer's output
+                hod[k].copy_(st["y_dec"], non_blocking=True)
                 ev_out[k].record(out_st)
             used[k] = True
 
@@ -332,9 +344,12 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(budget_s=args.cpu_budget)
     wls = None
+    step_check = None
     if rank == 0 and world == 1 and not args.no_workloads:
+        step_check = check_layer_step(sets[0], B, S, nh, nkv, hd, wl["theta"])
         del sets
         wls = measure_workloads(dev, {"hbm_gbs": hbm_peak, "bf16_tflops": bf16_peak})
+        wls["tiny_fp32_layer"] = check_tiny_fp32(dev)
 
     if world > 1:
         dist.barrier(device_ids=[local])
@@ -354,7 +369,7 @@ def run_ours(args):
                    "l2": f"{N_ROT} rotating input/output sets of ~{set_mb:.0f} MB (> 126 MB L2)"},
         "prefill_attn_tflops": attn["achieved"], "prefill_attn_frac_bf16_peak": attn["frac"],
         "decode_kv_gbs": dec["achieved"], "decode_frac_hbm": dec["frac"],
-        "kernels": kernels, "roofline": roofline, "gpu_launches": int(launches),
+        "kernels": kernels, "roofline": roofline, "gpu_launches": int(launches), "parity": step_check,
         "clocks": clk, "e2e": e2e, "cpu_baseline": cpu, "workloads": wls,
     }
     print(json.dumps(line))
@@ -367,7 +382,7 @@ def _set_mb(st):
 # ---------------------------------------------------------------------------
 # the other workloads of the metric, measured kernel by kernel
 # ---------------------------------------------------------------------------
-def measure_workloads(dev, peaks, iters=10, only=None):
+def measure_workloads(dev, peaks, iters=10, only=None, checks=True):
     """Llama-2-7B-shaped batched decode (B 64, 32 query heads, hd 128, ragged
     KV 512..8192, MHA/GQA/MQA caches, contiguous and in shuffled 64-key
     pages): KV GB/s; 8K-token prefill (B 2, 16
@@ -379,7 +394,9 @@ def measure_workloads(dev, peaks, iters=10, only=None):
     kernel is timed alone with CUDA events, L2 flushed before every timed call
     (a 512 MB write), median of `iters`.  ``only``: a set of section names
     (decode, prefill8k, generate, small, varlen, meanpool) to measure; None =
-    all."""
+    all.  ``checks``: also compare sampled outputs of each config with the
+    float64 oracle and time the oracle on the host cores (scaled linearly
+    from the sample to the whole config)."""
     import numpy as np
     import torch
 
@@ -392,10 +409,11 @@ def measure_workloads(dev, peaks, iters=10, only=None):
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
 
-    def timed(fn):
+    def timed(fn, flush_l2=True):
         ts = []
         for i in range(iters + 2):
-            flush.fill_(i & 0xFF)
+            if flush_l2:
+                flush.fill_(i & 0xFF)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             fn()
@@ -429,6 +447,12 @@ def measure_workloads(dev, peaks, iters=10, only=None):
             gbs = nbytes / (ms / 1e3) / 1e9
             dec[f"nkv{nkv}"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
                                 "bytes": int(nbytes)}
+            if nkv == 1:   # MQA: 143 MB of K/V fits in L2, so the warm figure differs
+                ms_w = timed(lambda: gqa.gqa_attn_decode(q, kc, vc, lens, o, ws, stream=stream), flush_l2=False)
+                dec["nkv1"].update({"ms_warm_l2": round(ms_w, 4),
+                                    "GB/s_warm_l2": round(nbytes / (ms_w / 1e3) / 1e9, 1)})
+            if checks:
+                dec[f"nkv{nkv}"].update(check_decode(q, kc, vc, lens_np, o, nkv))
             # the same cache cut into 64-key pages, shuffled over the page pool
             ps, maxp = 64, cap // 64
             perm = torch.randperm(B * maxp, generator=torch.Generator().manual_seed(nkv)).to(dev)
@@ -455,17 +479,24 @@ def measure_workloads(dev, peaks, iters=10, only=None):
         nh, hd = wl.shape.n_heads, wl.shape.head_dim
         lp = {}
         for nkv in wl.extra["n_kv_heads_cases"]:
-            q = torch.randn(B, nh, S, hd, generator=gen, device=dev).to(bf)
-            k = torch.randn(B, nkv, S, hd, generator=gen, device=dev).to(bf)
-            v = torch.randn(B, nkv, S, hd, generator=gen, device=dev).to(bf)
+            qkv = []
+            for tid, H in enumerate((nh, nkv, nkv)):   # N(0,1), 0.1% of each tensor's channels x20
+                t = torch.randn(B, H, S, hd, generator=gen, device=dev)
+                for c in W.outlier_channels(H * hd, wl.extra["outlier_frac"], wl.seed + nkv, tid):
+                    hh, d = divmod(int(c), hd)
+                    t[:, hh, :, d] *= wl.extra["outlier_scale"]
+                qkv.append(t.to(bf))
+            q, k, v = qkv
             o = torch.empty(B, S, nh, hd, dtype=bf, device=dev)
             ln = torch.full((B,), S, dtype=torch.int32, device=dev)
             for causal in (True, False):
                 ms = timed(lambda: gqa.gqa_attn_prefill(q, k, v, ln, causal, o, stream=stream))
                 fl = 4.0 * B * nh * S * S * hd * (0.5 if causal else 1.0)
                 tf = fl / (ms / 1e3) / 1e12
-                lp[f"nkv{nkv}_{'causal' if causal else 'full'}"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
-                                                                     "frac_bf16": round(tf / bf16_peak, 4)}
+                key = f"nkv{nkv}_{'causal' if causal else 'full'}"
+                lp[key] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_bf16": round(tf / bf16_peak, 4)}
+                if checks:
+                    lp[key].update(check_long_prefill(q, k, v, o, causal, nkv, wl))
         out["long_prefill_2x8192"] = lp
 
     # ---- MQA generation loop (prompt 16, 1024 steps), one timed region
@@ -506,13 +537,27 @@ def measure_workloads(dev, peaks, iters=10, only=None):
         ms_graph = timed_once(graph.replay, stream)
         toks = B * (P + T)
         per_step_bytes = 2.0 * sh.n_qkv * sh.hidden
+        # one step (t = 512) alone after an L2 flush: the cold counterpart of
+        # the graph loop, in which W_qkv can stay L2-resident from step to step
+        t_mid = T // 2
+
+        def one_step():
+            gqa.qkv_rope_project(xs[t_mid], w, pos_steps[t_mid], nh, nkv, hd, sh.rope_theta, qt, kc, vc, stream)
+            gqa.gqa_attn_decode(qt.view(B, nh, hd), kc, vc, len_steps[t_mid], ot[t_mid], ws, stream=stream)
+
+        us_cold = timed(one_step) * 1e3
         out["mqa_generate_b8_p16_g1024"] = {
             "ms_direct": round(ms_direct, 3), "ms_graph": round(ms_graph, 3),
             "tokens_per_s_direct": round(toks / (ms_direct / 1e3), 1),
             "tokens_per_s_graph": round(toks / (ms_graph / 1e3), 1),
+            "us_per_step_graph_warm_l2": round(ms_graph * 1e3 / T, 2),
+            "us_per_step_cold_l2": round(us_cold, 2),
             "weight_stream_GB/s_graph": round(per_step_bytes * T / (ms_graph / 1e3) / 1e9, 1),
-            "note": "W_qkv (78.6 MB) is re-read every step and may stay partly L2-resident across steps"}
-        del graph
+            "note": "W_qkv (78.6 MB) is re-read every step and may stay L2-resident across steps in the graph loop"}
+        del graph            # every replay and the single step recompute the same values
+        torch.cuda.synchronize(dev)
+        if checks:
+            out["mqa_generate_b8_p16_g1024"].update(check_generation(xp, xs, w, ot, sh, P, T))
 
     # ---- TinyLlama layer, the smaller prefill shapes of the same config
     if want("small"):
@@ -576,6 +621,230 @@ def measure_workloads(dev, peaks, iters=10, only=None):
     return out
 
 
+# ---------------------------------------------------------------------------
+# per-config parity against the oracle, and the oracle's own timing
+# ---------------------------------------------------------------------------
+def err_over_tol(got, want, dtype, col_scale=None):
+    """(max |err|, max of |err| / tolerance) under the parity tests' gates:
+    float32 |err| <= 1e-4 max|ref|; bf16 |err| <= 2e-2 min(1, RMS of the
+    row) + half a bf16 ulp of the reference, per element (rows = last axis),
+    outlier channels on their own scale."""
+    import numpy as np
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    err = np.abs(got - want)
+    if dtype == "f32":
+        tol = 1e-4 * max(float(np.max(np.abs(want))), 1e-30)
+        return float(err.max()), float(err.max()) / tol
+    sc = np.ones_like(want) if col_scale is None else np.broadcast_to(col_scale, want.shape)
+    unit = want / sc
+    _, ex = np.frexp(np.abs(want))
+    half_ulp = np.where(want != 0, np.ldexp(1.0, ex - 9), 0.0)
+    lim = 2e-2 * sc * np.minimum(1.0, np.sqrt(np.mean(unit * unit, axis=-1, keepdims=True))) + half_ulp
+    return float(err.max()), float(np.max(err / np.maximum(lim, 1e-30)))
+
+
+def _to64(t):
+    import numpy as np
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def oracle_seconds(fn, threads=None):
+    """Wall time of ``fn()`` on the host cores (``threads``: BLAS thread cap)."""
+    from threadpoolctl import threadpool_limits
+    if threads is None:
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+    with threadpool_limits(limits=threads):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+
+def check_tiny_fp32(dev, iters=20):
+    """The tiny fp32 layer: projection, causal prefill and output projection,
+    every element against the oracle; GPU microseconds (median of `iters`
+    runs), oracle seconds with all host cores and with one thread."""
+    import numpy as np
+    import torch
+
+    import mqa_attention_qkv_b200 as gqa
+    import workloads as W
+    from oracle import gqa_ref as ref
+    wl = W.TINY_FP32
+    sh = wl.shape
+    B, S = wl.batch_seq[0]
+    nh, nkv, hd = sh.n_heads, sh.n_kv_heads, sh.head_dim
+    x, w, pos = W.layer_inputs(sh, B, S, seed=wl.seed, dtype="f32")
+    w_o = W.output_weight(sh, wl.seed, "f32")
+    f32 = torch.float32
+    xd, wd, wod = (torch.from_numpy(t.store).to(dev) for t in (x, w, w_o))
+    posd = torch.from_numpy(pos).to(dev)
+    kc = torch.zeros(B, nkv, S, hd, dtype=f32, device=dev)
+    vc = torch.zeros_like(kc)
+    q = torch.empty(B, nh, S, hd, dtype=f32, device=dev)
+    o = torch.empty(B, S, nh, hd, dtype=f32, device=dev)
+    y = torch.empty(B, S, sh.hidden, dtype=f32, device=dev)
+    lens = torch.full((B,), S, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def layer():
+        gqa.qkv_rope_project(xd, wd, posd, nh, nkv, hd, sh.rope_theta, q, kc, vc, stream)
+        gqa.gqa_attn_prefill(q, kc, vc, lens, True, o, stream=stream)
+        gqa.gqa_o_proj_residual(o, wod, y, residual=xd, stream=stream)
+
+    layer()
+    ts = []
+    for _ in range(iters):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        layer()
+        b.record(stream)
+        b.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+
+    z = np.zeros((B, nkv, S, hd))
+
+    def oracle():
+        q_r, kc_r, vc_r = ref.qkv_rope_project(x.f64, w.f64, pos, nh, nkv, hd, sh.rope_theta, z, z)
+        o_r = ref.prefill_attention(q_r, kc_r, vc_r, np.full(B, S), True)
+        return o_r, ref.output_projection(o_r, w_o.f64, x.f64)
+
+    o_r, y_r = oracle()
+    e_o = err_over_tol(_to64(o), o_r, "f32")
+    e_y = err_over_tol(_to64(y), y_r, "f32")
+    return {"us": round(statistics.median(ts), 2), "max_err": max(e_o[0], e_y[0]),
+            "err_over_tol": round(max(e_o[1], e_y[1]), 4), "checked": "every element of o and y",
+            "oracle_s": round(oracle_seconds(oracle), 4), "oracle_s_1thread": round(oracle_seconds(oracle, 1), 4)}
+
+
+def check_layer_step(st, B, S, nh, nkv, hd, theta, rows=48):
+    """The bench step's layer output on sampled tokens of sequence 0 and the
+    decode token, against the oracle's chain on the same (device-drawn)
+    inputs; plus the oracle's time for the whole 4 x 2048 step, scaled
+    linearly from sampled query rows (all cores and one thread)."""
+    import numpy as np
+
+    from oracle import gqa_ref as ref
+    x, w, w_o, xd = _to64(st["x"][0:1]), _to64(st["w"]), _to64(st["w_o"]), _to64(st["x_dec"][0:1])
+    cap = S + 1
+    z = np.zeros((1, nkv, cap, hd))
+    pos = np.arange(S, dtype=np.int32)[None]
+    rb = ref.round_bf16
+
+    def chain(n_rows):
+        srows = np.linspace(0, S - 1, n_rows).round().astype(int)
+        q, kc, vc = ref.qkv_rope_project(x, w, pos, nh, nkv, hd, theta, z, z)
+        rr = [(0, h, int(s)) for s in srows for h in range(nh)]
+        o = np.asarray(ref.prefill_attention(rb(q), rb(kc), rb(vc), np.array([S]), True, rows=rr))
+        y = ref.output_projection(rb(o.reshape(n_rows, nh, hd)), w_o, x[0, srows])
+        qd, kc, vc = ref.qkv_rope_project(xd, w, np.array([[S]], dtype=np.int32), nh, nkv, hd, theta, kc, vc)
+        od = ref.decode_attention(rb(qd[:, :, 0]), rb(kc), rb(vc), np.array([S + 1]))
+        yd = ref.output_projection(rb(od)[:, None], w_o, xd[:, 0:1])
+        return srows, y, yd
+
+    srows, y_r, yd_r = chain(rows)
+    e1 = err_over_tol(_to64(st["y"][0])[srows], y_r, "bf16")
+    e2 = err_over_tol(_to64(st["y_dec"][0:1]), yd_r, "bf16")
+    out = {"max_err": max(e1[0], e2[0]), "err_over_tol": round(max(e1[1], e2[1]), 4),
+           "checked": f"layer output of {rows} query rows of sequence 0 and the decode token"}
+    for key, th in (("oracle_s", None), ("oracle_s_1thread", 1)):
+        t16, t64 = oracle_seconds(lambda: chain(16), th), oracle_seconds(lambda: chain(64), th)
+        per_row = max(0.0, (t64 - t16) / 48)
+        out[key] = round(B * (t16 - 16 * per_row + S * per_row), 2)
+    out["oracle_note"] = "whole 4 x 2048 step, scaled linearly from 16- and 64-row samples of one sequence"
+    return out
+
+
+def check_decode(q, kc, vc, lens_np, o, nkv, pairs=8):
+    """Sampled (sequence, head) rows of the batched decode against the oracle
+    (inputs copied from the device); oracle time for all B x 32 rows, scaled
+    by the keys each row reads (all cores and one thread)."""
+    import numpy as np
+
+    from oracle import gqa_ref as ref
+    B, nh, hd = q.shape
+    g = nh // nkv
+    r = np.random.default_rng(11)
+    sel = [(int(np.argmax(lens_np)), 0), (int(np.argmin(lens_np)), nh - 1)]
+    sel += [(int(r.integers(B)), int(r.integers(nh))) for _ in range(pairs - 2)]
+    data = [(_to64(q[b, h]), _to64(kc[b, h // g, :int(lens_np[b])]), _to64(vc[b, h // g, :int(lens_np[b])]))
+            for b, h in sel]
+    got = np.stack([_to64(o[b, h]) for b, h in sel])
+    rows = lambda: [ref.attend_row(qv, K, V)[0] for qv, K, V in data]   # noqa: E731
+    want = np.stack(rows())
+    e = err_over_tol(got, want, "bf16")
+    scale = nh * float(lens_np.sum()) / sum(int(lens_np[b]) for b, _ in sel)
+    return {"max_err": e[0], "err_over_tol": round(e[1], 4), "checked": f"{len(sel)} (sequence, head) rows",
+            "oracle_s": round(oracle_seconds(rows) * scale, 3),
+            "oracle_s_1thread": round(oracle_seconds(rows, 1) * scale, 3)}
+
+
+def check_long_prefill(q, k, v, o, causal, nkv, wl, n=12):
+    """Sampled query rows of the 8K prefill (outlier inputs) against the
+    oracle, outlier V channels on their x20 scale; oracle time for every row,
+    scaled by the keys each row sees."""
+    import numpy as np
+
+    import workloads as W
+    from oracle import gqa_ref as ref
+    B, nh, S, hd = q.shape
+    g = nh // nkv
+    r = np.random.default_rng(13)
+    sel = [(0, 0, 0), (B - 1, nh - 1, S - 1)] + [(int(r.integers(B)), int(r.integers(nh)), int(r.integers(S)))
+                                                  for _ in range(n - 2)]
+    vis = [s + 1 if causal else S for _, _, s in sel]
+    data = [(_to64(q[b, h, s]), _to64(k[b, h // g, :L]), _to64(v[b, h // g, :L])) for (b, h, s), L in zip(sel, vis)]
+    rows = lambda: [ref.attend_row(qv, K, V)[0] for qv, K, V in data]   # noqa: E731
+    want = np.stack(rows())
+    got = np.stack([_to64(o[b, s, h]) for b, h, s in sel])
+    vscale = np.ones(nkv * hd)
+    vscale[W.outlier_channels(nkv * hd, wl.extra["outlier_frac"], wl.seed + nkv, 2)] = wl.extra["outlier_scale"]
+    vscale = vscale.reshape(nkv, hd)
+    e = err_over_tol(got, want, "bf16", np.stack([vscale[h // g] for _, h, _ in sel]))
+    total = B * nh * (S * (S + 1) / 2 if causal else S * S)
+    scale = total / sum(vis)
+    return {"max_err": e[0], "err_over_tol": round(e[1], 4), "checked": f"{len(sel)} query rows",
+            "oracle_s": round(oracle_seconds(rows) * scale, 2)}
+
+
+def check_generation(xp, xs, w, ot, sh, P, T, seqs=(0, 7), steps=(0, 511, 1023)):
+    """Decode outputs of sampled steps of the generation loop against the
+    oracle, which projects the sequence's own tokens (inputs copied from the
+    device) to rebuild its K/V cache; oracle time for the whole loop (all
+    8 x 1040 tokens projected, every step's attention), scaled from one
+    sequence."""
+    import numpy as np
+
+    from oracle import gqa_ref as ref
+    nh, nkv, hd = sh.n_heads, sh.n_kv_heads, sh.head_dim
+    W_ = _to64(w)
+    rb = ref.round_bf16
+    errs = []
+
+    def one_seq(b, which, check):
+        x = np.concatenate([_to64(xp[b]), _to64(xs[:, b, 0])], axis=0)[None]      # [1, P + T, hidden]
+        pos = np.arange(P + T, dtype=np.int32)[None]
+        z = np.zeros((1, nkv, P + T, hd))
+        q, kc, vc = ref.qkv_rope_project(x, W_, pos, nh, nkv, hd, sh.rope_theta, z, z)
+        for t in which:
+            want = ref.decode_attention(rb(q[:, :, P + t]), rb(kc), rb(vc), np.array([P + t + 1]))
+            if check:
+                errs.append(err_over_tol(_to64(ot[t, b]), want[0], "bf16"))
+
+    for b in seqs:
+        one_seq(b, steps, True)
+    # one sequence with every 32nd step; the steps' attention scaled to all 1024
+    sample = list(range(0, T, 32))
+    t_proj = oracle_seconds(lambda: one_seq(0, [], False))
+    t_some = oracle_seconds(lambda: one_seq(0, sample, False))
+    t_seq = t_proj + (t_some - t_proj) * T / len(sample)
+    return {"max_err": max(e[0] for e in errs), "err_over_tol": round(max(e[1] for e in errs), 4),
+            "checked": f"steps {list(steps)} of sequences {list(seqs)}", "oracle_s": round(t_seq * 8, 2),
+            "oracle_note": "one sequence's projection and every 32nd step timed, scaled to 8 sequences x 1024 steps"}
+
+
 def timed_once(fn, stream):
     import torch
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -592,7 +861,8 @@ def timed_once(fn, stream):
 def oracle_sample_step(rows_per_seq: int, seed: int = 1):
     """The float64 oracle on one of the workload's sequences: projection of its
     2048 prompt tokens, causal attention for `rows_per_seq` evenly spaced query
-    rows (all 32 heads), then the decode step.  Returns tokens covered."""
+    rows (all 32 heads) and their output projection + residual, then the
+    decode step through the same layer.  Returns tokens covered."""
     import numpy as np
 
     import workloads as W
@@ -606,10 +876,14 @@ def oracle_sample_step(rows_per_seq: int, seed: int = 1):
     q, kc, vc = ref.qkv_rope_project(x.f64, w.f64, pos, nh, nkv, hd, wl["theta"], zeros, zeros)
     srows = np.linspace(0, S - 1, rows_per_seq).round().astype(int)
     rows = [(0, h, int(s)) for h in range(nh) for s in srows]
-    ref.prefill_attention(q, kc, vc, np.array([S]), True, rows=rows)
+    w_o = W.output_weight(shape, seed, "bf16")
+    o = np.asarray(ref.prefill_attention(q, kc, vc, np.array([S]), True, rows=rows))
+    o = o.reshape(nh, rows_per_seq, hd).transpose(1, 0, 2)                  # [tokens, heads, hd]
+    ref.output_projection(o, w_o.f64, x.f64[0, srows])
     qd, kc, vc = ref.qkv_rope_project(xd.f64, w.f64, np.array([[S]], dtype=np.int32), nh, nkv, hd,
                                       wl["theta"], kc, vc)
-    ref.decode_attention(qd[:, :, 0], kc, vc, np.array([S + 1]))
+    od = ref.decode_attention(qd[:, :, 0], kc, vc, np.array([S + 1]))
+    ref.output_projection(od[:, None], w_o.f64, xd.f64[:, 0:1])
     return rows_per_seq + 1
 
 
@@ -634,8 +908,8 @@ def cpu_baseline(budget_s: float = 20.0, rows_per_seq: int | None = None):
     threads, affinity = _cores()
     return {"value": round(tok / dt, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": (f"float64 numpy oracle, 1 of 4 sequences: projection of its 2048 prompt tokens, "
-                       f"causal attention of {rows_per_seq} evenly spaced query rows x 32 heads, "
-                       f"1 decode token; {dt:.1f} s; host affinity {affinity} cores"),
+                       f"causal attention of {rows_per_seq} evenly spaced query rows x 32 heads and their "
+                       f"output projection, 1 decode token; {dt:.1f} s; host affinity {affinity} cores"),
             "seconds": round(dt, 2)}
 
 
@@ -662,8 +936,8 @@ def run_reference(args):
     threads, affinity = _cores()
     cpu = {"value": round(value, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
            "sample": (f"float64 numpy oracle per step: 1 sequence, projection of 2048 prompt tokens, "
-                      f"causal attention of {rows} evenly spaced query rows x 32 heads, 1 decode token; "
-                      f"host affinity {affinity} cores")}
+                      f"causal attention of {rows} evenly spaced query rows x 32 heads and their output "
+                      f"projection, 1 decode token; host affinity {affinity} cores")}
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
