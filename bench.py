@@ -497,6 +497,26 @@ def measure_workloads(dev, peaks, iters=10, only=None, checks=True):
                 lp[key] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_bf16": round(tf / bf16_peak, 4)}
                 if checks:
                     lp[key].update(check_long_prefill(q, k, v, o, causal, nkv, wl))
+            # FP8 (e4m3) with incoherent processing: quantise (rotation, amax, codes), then attention
+            q8 = torch.empty(B, nh, S, hd, dtype=torch.uint8, device=dev)
+            k8 = torch.empty(B, nkv, S, hd, dtype=torch.uint8, device=dev)
+            v8t = torch.empty(B, nkv, hd, S, dtype=torch.uint8, device=dev)
+            amax = torch.empty(3, device=dev)
+            signs = np.where(np.random.default_rng([wl.seed, 9]).integers(0, 2, hd) == 1, -1, 1).tolist()
+            ms_q = timed(lambda: gqa.gqa_fp8_quantize_qkv(q, k, v, ln, q8, k8, v8t, amax, signs=signs, stream=stream))
+            qbytes = 2.0 * 2 * (q.numel() + 2 * k.numel()) + (q.numel() + 2 * k.numel())   # two bf16 passes + codes
+            fp8_peak = 2.0 * bf16_peak
+            for causal in (True, False):
+                ms = timed(lambda: gqa.gqa_attn_prefill_fp8(q8, k8, v8t, amax, ln, causal, o, stream=stream))
+                fl = 4.0 * B * nh * S * S * hd * (0.5 if causal else 1.0)
+                tf = fl / (ms / 1e3) / 1e12
+                key = f"fp8_nkv{nkv}_{'causal' if causal else 'full'}"
+                lp[key] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_fp8": round(tf / fp8_peak, 4),
+                           "quantize_ms": round(ms_q, 4),
+                           "quantize_GB/s": round(qbytes / (ms_q / 1e3) / 1e9, 1),
+                           "fp8_peak_note": "2 x the bf16 peak (the nominal fp8/bf16 ratio)"}
+                if checks:
+                    lp[key].update(check_fp8_error(q, k, v, o, ln, causal, nkv, signs, q8, k8, v8t, amax, stream))
         out["long_prefill_2x8192"] = lp
 
     # ---- MQA generation loop (prompt 16, 1024 steps), one timed region
@@ -843,6 +863,36 @@ def check_generation(xp, xs, w, ot, sh, P, T, seqs=(0, 7), steps=(0, 511, 1023))
     return {"max_err": max(e[0] for e in errs), "err_over_tol": round(max(e[1] for e in errs), 4),
             "checked": f"steps {list(steps)} of sequences {list(seqs)}", "oracle_s": round(t_seq * 8, 2),
             "oracle_note": "one sequence's projection and every 32nd step timed, scaled to 8 sequences x 1024 steps"}
+
+
+def check_fp8_error(q, k, v, o, ln, causal, nkv, signs, q8, k8, v8t, amax, stream, n=12):
+    """FP8 output on sampled rows against exact attention on the bf16 inputs
+    (float64 oracle), with the random-sign Hadamard rotation (the output in
+    ``o``) and without it: the error the rotation removes."""
+    import numpy as np
+
+    import mqa_attention_qkv_b200 as gqa
+    from oracle import gqa_ref as ref
+    B, nh, S, hd = q.shape
+    g = nh // nkv
+    r = np.random.default_rng(17)
+    sel = [(int(r.integers(B)), int(r.integers(nh)), int(r.integers(S))) for _ in range(n)]
+    vis = [s + 1 if causal else S for _, _, s in sel]
+    want = np.stack([ref.attend_row(_to64(q[b, h, s]), _to64(k[b, h // g, :L]), _to64(v[b, h // g, :L]))[0]
+                     for (b, h, s), L in zip(sel, vis)])
+
+    def rms_err(out):
+        got = np.stack([_to64(out[b, s, h]) for b, h, s in sel])
+        return float(np.sqrt(np.mean((got - want) ** 2)))
+
+    e_rot = rms_err(o)
+    o2 = o.clone()
+    gqa.gqa_fp8_quantize_qkv(q, k, v, ln, q8, k8, v8t, amax, signs=None, stream=stream)
+    gqa.gqa_attn_prefill_fp8(q8, k8, v8t, amax, ln, causal, o2, stream=stream)
+    e_plain = rms_err(o2)
+    gqa.gqa_fp8_quantize_qkv(q, k, v, ln, q8, k8, v8t, amax, signs=signs, stream=stream)   # rotated codes again
+    return {"rms_err_vs_exact": round(e_rot, 5), "rms_err_vs_exact_no_rotation": round(e_plain, 5),
+            "checked": f"{n} query rows against float64 attention on the bf16 inputs"}
 
 
 def timed_once(fn, stream):

@@ -353,6 +353,66 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
                           void* stream);
 
 /*
+ * gqa_fp8_quantize_qkv - FP8 (e4m3) inputs for gqa_attn_prefill_fp8, with
+ * incoherent processing.
+ *
+ * Source: "FlashAttention-3" (together.ai summary), section "FP8低精度と
+ * incoherent processing": FP8 doubles the tensor-core rate, but outlier
+ * features inflate the rounding error; multiplying queries and keys by one
+ * random orthogonal matrix, a Hadamard transform with random signs, spreads
+ * the outliers over the features before quantising, and leaves every score
+ * q.k unchanged.  Here M = H diag(signs) / sqrt(head_dim), H the Sylvester
+ * Hadamard matrix; q and k rows become x M, v is not rotated.  Each tensor is
+ * then scaled by 448 / amax (its largest magnitude after the rotation) and
+ * rounded to e4m3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+ * nearest, ties to even, saturating at 448).
+ *
+ *   q          [B, n_heads, S, head_dim] bf16
+ *   k_cache,
+ *   v_cache    [B, n_kv_heads, cache_cap, head_dim] bf16; rows at or beyond
+ *              kv_lens[b] are not read (they may hold NaN)
+ *   kv_lens    [B] int32, clamped to [0, cache_cap]
+ *   signs      HOST array of head_dim values, each +1 or -1 (read during the
+ *              call), or NULL for no rotation
+ *   q8         [B, n_heads, S, head_dim] e4m3 codes, written
+ *   k8         [B, n_kv_heads, cache_cap, head_dim] e4m3, written (rows at or
+ *              beyond kv_len are zero)
+ *   v8t        [B, n_kv_heads, head_dim, cache_cap] e4m3, written TRANSPOSED
+ *              (per KV head, one row of cache_cap keys per feature; keys at
+ *              or beyond kv_len are zero)
+ *   amax       DEVICE float[3], written: the largest magnitude of the
+ *              rotated q, the rotated k and v; tensor t's scale is
+ *              amax[t] / 448 (a zero tensor has amax 0 and codes 0)
+ *
+ * head_dim 64 or 128; cache_cap a multiple of 16.  Asynchronous on `stream`
+ * (a memset of amax and three kernels); allocates nothing.
+ */
+int gqa_fp8_quantize_qkv(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens, int B,
+                         int S, int n_heads, int n_kv_heads, int head_dim, int cache_cap, const int8_t* signs,
+                         void* q8, void* k8, void* v8t, float* amax, void* stream);
+
+/*
+ * gqa_attn_prefill_fp8 - gqa_attn_prefill on FP8 inputs: the tiled online
+ * softmax with S = Q K^T and O = P V both on the tensor cores in e4m3
+ * (tcgen05 kind::f8f6f4, float32 accumulation).  The probabilities P are
+ * rounded to e4m3 for P V (offset by 2^4 so that values down to 2^-10 of a
+ * row's maximum keep full e4m3 precision); the row sums use the unrounded
+ * float32 probabilities.  Source as gqa_fp8_quantize_qkv and gqa_attn_prefill.
+ *
+ *   q8, k8, v8t, amax  as written by gqa_fp8_quantize_qkv (with or without
+ *                      the rotation: scores are the same either way)
+ *   kv_lens            [B] int32; queries sit at positions kv_len - S + s
+ *   causal             nonzero: key t visible to a query at position p iff t <= p
+ *   out                [B, S, n_heads, head_dim] bf16
+ *
+ * head_dim 128 only; cache_cap a multiple of 16.  Statuses as
+ * gqa_attn_prefill; asynchronous on `stream`; allocates nothing.
+ */
+int gqa_attn_prefill_fp8(const void* q8, const void* k8, const void* v8t, const float* amax, const int32_t* kv_lens,
+                         int B, int S, int n_heads, int n_kv_heads, int head_dim, int cache_cap, int causal, void* out,
+                         void* stream);
+
+/*
  * gqa_debug_inject_launch_failures - testing aid (host-side fault
  * injection): the next n compute calls (projection, prefill, decode,
  * mean-pool) that pass argument validation return GQA_ERR_LAUNCH_FAILED

@@ -18,7 +18,8 @@ __all__ = [
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
     "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures", "gqa_o_proj_residual",
-    "gqa_debug_set_wait_limit_ns", "gqa_debug_skip_next_kv_tile", "EXPORTED_SYMBOLS",
+    "gqa_debug_set_wait_limit_ns", "gqa_debug_skip_next_kv_tile", "gqa_fp8_quantize_qkv",
+    "gqa_attn_prefill_fp8", "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -29,7 +30,8 @@ EXPORTED_SYMBOLS = (
     "gqa_attn_decode_workspace_size", "gqa_status_string", "gqa_device_error",
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
     "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures", "gqa_o_proj_residual",
-    "gqa_debug_set_wait_limit_ns", "gqa_debug_skip_next_kv_tile",
+    "gqa_debug_set_wait_limit_ns", "gqa_debug_skip_next_kv_tile", "gqa_fp8_quantize_qkv",
+    "gqa_attn_prefill_fp8",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -82,6 +84,10 @@ def lib() -> ctypes.CDLL:
     L.gqa_attn_prefill_varlen.restype = i32
     L.gqa_o_proj_residual.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp]
     L.gqa_o_proj_residual.restype = i32
+    L.gqa_fp8_quantize_qkv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
+    L.gqa_fp8_quantize_qkv.restype = i32
+    L.gqa_attn_prefill_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    L.gqa_attn_prefill_fp8.restype = i32
     L.gqa_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     L.gqa_debug_set_wait_limit_ns.restype = i32
     L.gqa_debug_skip_next_kv_tile.argtypes = [i32]
@@ -261,6 +267,42 @@ def gqa_o_proj_residual(attn, w_o, out, residual=None, stream=None) -> None:
         _ptr(out, dt, oshape, "out"), _dtype_code(attn), _stream(stream),
     )
     _check("gqa_o_proj_residual", lib().gqa_o_proj_residual(*args))
+
+
+def gqa_fp8_quantize_qkv(q, k_cache, v_cache, kv_lens, q8, k8, v8t, amax, signs=None, stream=None) -> None:
+    """FP8 inputs for gqa_attn_prefill_fp8: q [B,nh,S,hd], caches [B,nkv,cap,hd]
+    bf16 -> q8 [B,nh,S,hd], k8 [B,nkv,cap,hd], v8t [B,nkv,hd,cap] (uint8
+    tensors holding e4m3 codes) and amax [3] float32; ``signs`` (hd values
+    +-1, a host sequence) selects the random-sign Hadamard rotation of q and
+    k, None for none."""
+    import torch
+    B, nh, S, hd = q.shape
+    nkv, cap = k_cache.shape[1], k_cache.shape[2]
+    sg = None
+    if signs is not None:
+        sg = (ctypes.c_int8 * hd)(*[int(v) for v in signs])
+    args = (
+        _ptr(q, torch.bfloat16, name="q"), _ptr(k_cache, torch.bfloat16, (B, nkv, cap, hd), "k_cache"),
+        _ptr(v_cache, torch.bfloat16, (B, nkv, cap, hd), "v_cache"), _ptr(kv_lens, torch.int32, (B,), "kv_lens"),
+        B, S, nh, nkv, hd, cap, ctypes.cast(sg, ctypes.c_void_p) if sg is not None else None,
+        _ptr(q8, torch.uint8, (B, nh, S, hd), "q8"), _ptr(k8, torch.uint8, (B, nkv, cap, hd), "k8"),
+        _ptr(v8t, torch.uint8, (B, nkv, hd, cap), "v8t"), _ptr(amax, torch.float32, (3,), "amax"), _stream(stream),
+    )
+    _check("gqa_fp8_quantize_qkv", lib().gqa_fp8_quantize_qkv(*args))
+
+
+def gqa_attn_prefill_fp8(q8, k8, v8t, amax, kv_lens, causal: bool, out, stream=None) -> None:
+    """FP8 prefill: the tensors of gqa_fp8_quantize_qkv -> out [B,S,nh,hd] bf16."""
+    import torch
+    B, nh, S, hd = q8.shape
+    nkv, cap = k8.shape[1], k8.shape[2]
+    args = (
+        _ptr(q8, torch.uint8, name="q8"), _ptr(k8, torch.uint8, (B, nkv, cap, hd), "k8"),
+        _ptr(v8t, torch.uint8, (B, nkv, hd, cap), "v8t"), _ptr(amax, torch.float32, (3,), "amax"),
+        _ptr(kv_lens, torch.int32, (B,), "kv_lens"), B, S, nh, nkv, hd, cap, 1 if causal else 0,
+        _ptr(out, torch.bfloat16, (B, S, nh, hd), "out"), _stream(stream),
+    )
+    _check("gqa_attn_prefill_fp8", lib().gqa_attn_prefill_fp8(*args))
 
 
 def gqa_device_error() -> int:

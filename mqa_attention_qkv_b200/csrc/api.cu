@@ -405,6 +405,58 @@ int gqa_o_proj_residual(const void* attn, const void* w_o, const void* residual,
 
 uint64_t gqa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int gqa_fp8_quantize_qkv(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens, int B,
+                         int S, int n_heads, int n_kv_heads, int head_dim, int cache_cap, const int8_t* signs,
+                         void* q8, void* k8, void* v8t, float* amax, void* stream) {
+  if (B < 0 || S < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0) return GQA_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (cache_cap % 16 != 0) return GQA_ERR_UNSUPPORTED_SHAPE;   // 16-byte rows of the transposed V
+  if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems || (long long)B * n_heads * S * head_dim > kMaxElems ||
+      (long long)B * n_kv_heads * cache_cap >= kMaxRows || (long long)B * n_heads * S >= kMaxRows)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return GQA_OK;
+  if (!q || !k_cache || !v_cache || !kv_lens || !q8 || !k8 || !v8t || !amax) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q8) || !aligned16(k8) ||
+      !aligned16(v8t) || !aligned4(kv_lens) || !aligned4(amax))
+    return GQA_ERR_MISALIGNED;
+  gqa::Fp8QuantParams p{q, k_cache, v_cache, kv_lens, B, S, n_heads, n_kv_heads, head_dim, cache_cap,
+                        signs != nullptr, {0u, 0u, 0u, 0u}, q8, k8, v8t, amax, nullptr};
+  if (signs) {
+    for (int c = 0; c < head_dim; ++c) {
+      if (signs[c] != 1 && signs[c] != -1) return GQA_ERR_INVALID_ARG;
+      if (signs[c] < 0) p.signs[c >> 5] |= 1u << (c & 31);
+    }
+  }
+  int st;
+  const DeviceInfo* d = compute_device(&st);
+  if (!d) return st;
+  p.err = d->err;
+  return launch_status(gqa::launch_fp8_quantize(p, d->num_sms, static_cast<cudaStream_t>(stream)), 3);
+}
+
+int gqa_attn_prefill_fp8(const void* q8, const void* k8, const void* v8t, const float* amax, const int32_t* kv_lens,
+                         int B, int S, int n_heads, int n_kv_heads, int head_dim, int cache_cap, int causal, void* out,
+                         void* stream) {
+  if (B < 0 || S < 0 || n_heads <= 0 || n_kv_heads <= 0 || cache_cap <= 0) return GQA_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads != 0) return GQA_ERR_INVALID_ARG;
+  if (head_dim != 128 || cache_cap % 16 != 0) return GQA_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)B * n_kv_heads * cache_cap * head_dim > kMaxElems || (long long)B * n_heads * S * head_dim > kMaxElems ||
+      B > 65535 || n_heads > 65535 || (long long)B * n_kv_heads * cache_cap >= kMaxRows ||
+      (long long)B * n_heads * S >= kMaxRows)
+    return GQA_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || S == 0) return GQA_OK;
+  if (!q8 || !k8 || !v8t || !amax || !kv_lens || !out) return GQA_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t) || !aligned16(out) || !aligned4(amax) || !aligned4(kv_lens))
+    return GQA_ERR_MISALIGNED;
+  int st;
+  const DeviceInfo* d = compute_device(&st);
+  if (!d) return st;
+  const gqa::Fp8AttnParams p{q8, k8, v8t, amax, kv_lens, B, S, n_heads, n_kv_heads, head_dim, cache_cap,
+                             causal ? 1 : 0, out, d->err};
+  return launch_status(gqa::launch_prefill_fp8(p, static_cast<cudaStream_t>(stream)));
+}
+
 int gqa_debug_set_wait_limit_ns(uint64_t ns) {
   int st;
   const DeviceInfo* d = device_info(&st);

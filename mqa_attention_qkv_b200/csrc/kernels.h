@@ -31,6 +31,34 @@ struct OprojParams {
   int* err;
 };
 
+// FP8 quantisation of the attention inputs (random-sign Hadamard on q and k).
+struct Fp8QuantParams {
+  const void* q;          // [B, nh, S, hd] bf16
+  const void* k;          // [B, nkv, cap, hd] bf16
+  const void* v;
+  const int32_t* kv_lens; // [B]
+  int B, S, nh, nkv, hd, cap;
+  int rotate;             // apply the rotation to q and k
+  uint32_t signs[4];      // bit c set: sign of rotation column c is -1
+  void* q8;               // [B, nh, S, hd] e4m3
+  void* k8;               // [B, nkv, cap, hd] e4m3
+  void* v8t;              // [B, nkv, hd, cap] e4m3 (transposed)
+  float* amax;            // [3] device: max |value| of rotated q, rotated k, v
+  int* err;
+};
+
+// FP8 prefill attention over the quantised tensors.
+struct Fp8AttnParams {
+  const void* q8;         // [B, nh, S, hd] e4m3
+  const void* k8;         // [B, nkv, cap, hd] e4m3
+  const void* v8t;        // [B, nkv, hd, cap] e4m3
+  const float* amax;      // [3] device: the scales are amax / 448
+  const int32_t* kv_lens; // [B]
+  int B, S, nh, nkv, hd, cap, causal;
+  void* out;              // [B, S, nh, hd] bf16
+  int* err;
+};
+
 struct PrefillParams {
   const void* q;          // [B, nh, S, hd]
   const void* k_cache;    // [B, nkv, cap, hd]
@@ -110,6 +138,9 @@ cudaError_t launch_qkv_smallm(const QkvParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_oproj_tc(const OprojParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_oproj_smallt(const OprojParams& p, int num_sms, cudaStream_t st);   // T <= 64
 cudaError_t launch_oproj_simt(const OprojParams& p, bool bf16, cudaStream_t st);
+// FP8 path: amax + quantisation passes, and the tcgen05 kind::f8f6f4 prefill (head_dim 128).
+cudaError_t launch_fp8_quantize(const Fp8QuantParams& p, int num_sms, cudaStream_t st);
+cudaError_t launch_prefill_fp8(const Fp8AttnParams& p, cudaStream_t st);
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
 cudaError_t launch_prefill_fa(const PrefillParams& p, cudaStream_t st);    // head_dim 64/128, 2 Q tiles/CTA
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128
@@ -156,6 +187,9 @@ bool make_tmap_bf16_3d(void* map, const void* base, const uint64_t dims[3], cons
 // tile a 2-D box over head-major rows gives.  tokens == 0 is encoded as 1
 // (nothing may then be loaded).
 bool make_tmap_packed(void* map, const void* base, uint64_t tokens, int heads, int hd);
+// 2-D byte (e4m3) descriptor with 128-byte swizzle, zero fill outside the dims.
+bool make_tmap_u8_2d(void* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer);
 
 // Shared by the C-ABI translation units (defined in api.cu).
 int device_check(int** err);  // GQA_OK, or the status for the current device

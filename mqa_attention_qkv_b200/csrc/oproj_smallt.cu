@@ -12,7 +12,8 @@
 // NT = 16, 32 or 64), so a tile wastes nothing on padding rows of W.  A
 // 128-row block of W_o alone would keep only N / 128 SMs busy, so its
 // reduction dimension is split over a thread-block cluster of `split` CTAs
-// (one per SM, split <= 8, as many as the SM count allows): each CTA streams
+// (one per SM, split <= 8, the largest for which every cluster is resident at
+// once): each CTA streams
 // its K range of the block through a TMA ring into tcgen05.mma.kind::f16
 // with the fp32 partial in TMEM, writes the partial to its shared memory,
 // and after a cluster barrier every CTA sums its share of the block's rows
@@ -165,14 +166,21 @@ oproj_smallt_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_consta
       const int tok = e / quads, r = r0 + 4 * (e % quads);
       const int n = m0 + r;
       if (n >= p.N) continue;   // N % 8 == 0: a quad is wholly inside or outside
+      // every CTA's partial: all remote loads issued before the first add
+      float4 part[kMaxSplit];
+      const uint32_t a = red_u + (uint32_t)(tok * BM + r) * 4u;
+#pragma unroll
+      for (int q = 0; q < kMaxSplit; ++q)
+        if (q < split) part[q] = tc::ld_dsmem_f32x4(tc::mapa_shared(a, (uint32_t)q));
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q = 0; q < split; ++q) {
-        const float4 v = tc::ld_dsmem_f32x4(tc::mapa_shared(red_u + (uint32_t)(tok * BM + r) * 4u, (uint32_t)q));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
-      }
+#pragma unroll
+      for (int q = 0; q < kMaxSplit; ++q)
+        if (q < split) {
+          acc.x += part[q].x;
+          acc.y += part[q].y;
+          acc.z += part[q].z;
+          acc.w += part[q].w;
+        }
       const size_t o = (size_t)tok * p.N + n;
       if (res) {
         const uint2 rv = *reinterpret_cast<const uint2*>(res + o);
@@ -207,10 +215,42 @@ cudaError_t launch_nt(const OprojParams& p, int num_sms, cudaStream_t st) {
     return e;
   const int n_mblk = (p.N + BM - 1) / BM;
   const int n_kb = (p.K + BK - 1) / BK;
-  int split = num_sms / n_mblk;
-  if (split > kMaxSplit) split = kMaxSplit;
-  if (split > n_kb) split = n_kb;
-  if (split < 1) split = 1;
+  // The largest split whose clusters all fit on the GPU at once (measured on
+  // B200: at most 15 clusters of 8 are resident, so 16 row blocks x 8 would
+  // take two waves), found once per device and split from the occupancy API.
+  static std::atomic<int> max_clusters[64][kMaxSplit + 1];   // 0 unknown, else clusters + 1
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    dev = -1;
+  }
+  int split = 1;
+  for (int sp = kMaxSplit; sp >= 1; --sp) {
+    if (sp > n_kb || n_mblk * sp > num_sms) continue;
+    int fit = dev >= 0 ? max_clusters[dev][sp].load(std::memory_order_relaxed) - 1 : -1;
+    if (fit < 0) {
+      cudaLaunchConfig_t q = {};
+      q.gridDim = dim3((unsigned)(n_mblk * sp), 1, 1);
+      q.blockDim = dim3(THREADS, 1, 1);
+      q.dynamicSmemBytes = C::SMEM;
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = (unsigned)sp;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&fit, oproj_smallt_kernel<NT>, &q) != cudaSuccess) {
+        cudaGetLastError();
+        fit = 0;
+      }
+      if (dev >= 0) max_clusters[dev][sp].store(fit + 1, std::memory_order_relaxed);
+    }
+    if (fit >= n_mblk) {
+      split = sp;
+      break;
+    }
+  }
   CUtensorMap tw, tx;
   if (!make_tmap_bf16_2d(&tw, p.w, p.K, p.N, (uint64_t)p.K * 2, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tx, p.x, p.K, p.T, (uint64_t)p.K * 2, BK, NT)) return cudaErrorInvalidValue;

@@ -43,6 +43,9 @@ constexpr int kPoly = GQA_PAIR_POLY;
 #ifndef GQA_PAIR_PACK
 #define GQA_PAIR_PACK 0
 #endif
+#ifndef GQA_PAIR_F2
+#define GQA_PAIR_F2 0
+#endif
 
 // Two probabilities (finite, >= 0) -> packed bf16 pair, rounded to nearest.
 __device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
@@ -348,6 +351,26 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           }
           tc::tmem_st16(tmem + lane_base + kPCol + c * 16, w);
         }
+      } else if constexpr (GQA_PAIR_F2) {
+        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(neg_m, neg_m);
+        float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < BKV / 32; ++c) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float2 pp = __ffma2_rn(make_float2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), sc2, nm2);
+            pp.x = tc::ex2(pp.x);
+            pp.y = tc::ex2(pp.y);
+            if (i & 1) acc_b = __fadd2_rn(acc_b, pp); else acc_a = __fadd2_rn(acc_a, pp);
+            w[i] = pack_p(pp.x, pp.y);
+          }
+          tc::tmem_st16(tmem + lane_base + kPCol + c * 16, w);
+        }
+        sa0 = acc_a.x;
+        sa1 = acc_a.y;
+        sb0 = acc_b.x;
+        sb1 = acc_b.y;
       } else {
 #pragma unroll
         for (int c = 0; c < BKV / 32; ++c) {

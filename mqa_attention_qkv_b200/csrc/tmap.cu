@@ -60,6 +60,20 @@ bool make_tmap_bf16_3d(void* map, const void* base, const uint64_t dims[3], cons
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_u8_2d(void* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer) {
+  if (!load_encoder()) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_packed(void* map, const void* base, uint64_t tokens, int heads, int hd) {
   const uint64_t dims[3] = {(uint64_t)hd, (uint64_t)heads, tokens > 0 ? tokens : 1};
   const uint64_t strides[2] = {(uint64_t)hd * 2, (uint64_t)heads * hd * 2};
