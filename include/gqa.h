@@ -441,6 +441,15 @@ int gqa_debug_set_wait_limit_ns(uint64_t ns);
  */
 int gqa_debug_skip_next_kv_tile(int tile);
 
+/*
+ * gqa_debug_exp2_poly - testing aid: evaluates, for n device floats x, the
+ * polynomial 2^x that the prefill softmax can run on the FMA pipe (range
+ * reduction to n + f with |f| <= 1/2, a degree-3 minimax fit of 2^f in
+ * relative error, inputs below -125 clamped) into poly[i], and CUDA's
+ * exp2f(x[i]) into ref[i].  Device pointers; asynchronous on `stream`.
+ */
+int gqa_debug_exp2_poly(const float* x, int n, float* poly, float* ref, void* stream);
+
 /* Human-readable text of a gqa_status value (static storage). */
 const char* gqa_status_string(int status);
 

@@ -19,7 +19,7 @@ __all__ = [
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
     "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures", "gqa_o_proj_residual",
     "gqa_debug_set_wait_limit_ns", "gqa_debug_skip_next_kv_tile", "gqa_fp8_quantize_qkv",
-    "gqa_attn_prefill_fp8", "EXPORTED_SYMBOLS",
+    "gqa_attn_prefill_fp8", "gqa_debug_exp2_poly", "EXPORTED_SYMBOLS",
 ]
 
 GQA_F32 = 0
@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = (
     "gqa_launch_count", "gqa_attn_decode_noalloc", "gqa_meanpool_kv_heads", "gqa_attn_decode_paged",
     "gqa_attn_prefill_varlen", "gqa_debug_inject_launch_failures", "gqa_o_proj_residual",
     "gqa_debug_set_wait_limit_ns", "gqa_debug_skip_next_kv_tile", "gqa_fp8_quantize_qkv",
-    "gqa_attn_prefill_fp8",
+    "gqa_attn_prefill_fp8", "gqa_debug_exp2_poly",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -88,6 +88,8 @@ def lib() -> ctypes.CDLL:
     L.gqa_fp8_quantize_qkv.restype = i32
     L.gqa_attn_prefill_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
     L.gqa_attn_prefill_fp8.restype = i32
+    L.gqa_debug_exp2_poly.argtypes = [vp, i32, vp, vp, vp]
+    L.gqa_debug_exp2_poly.restype = i32
     L.gqa_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     L.gqa_debug_set_wait_limit_ns.restype = i32
     L.gqa_debug_skip_next_kv_tile.argtypes = [i32]
@@ -328,6 +330,16 @@ def gqa_debug_skip_next_kv_tile(tile: int) -> None:
     """Testing aid: the next head_dim-64 bf16 prefill leaves key tile ``tile``
     unloaded in its first CTA, so that the waits on it run out (-1 disarms)."""
     _check("gqa_debug_skip_next_kv_tile", lib().gqa_debug_skip_next_kv_tile(int(tile)))
+
+
+def gqa_debug_exp2_poly(x, poly, ref, stream=None) -> None:
+    """Testing aid: the softmax's polynomial 2^x (poly) and CUDA's exp2f (ref)
+    for the float32 CUDA tensor x."""
+    import torch
+    n = x.numel()
+    args = (_ptr(x, torch.float32, name="x"), n, _ptr(poly, torch.float32, (n,), "poly"),
+            _ptr(ref, torch.float32, (n,), "ref"), _stream(stream))
+    _check("gqa_debug_exp2_poly", lib().gqa_debug_exp2_poly(*args))
 
 
 def gqa_launch_count() -> int:

@@ -397,7 +397,12 @@ int gqa_o_proj_residual(const void* attn, const void* w_o, const void* residual,
   const gqa::OprojParams p{attn, w_o, residual, out, T, (int)K, hidden, d->err};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == GQA_BF16 && hidden % 8 == 0) {
-    if (T <= 64) return launch_status(gqa::launch_oproj_smallt(p, d->num_sms, s));
+    if (T <= 64) {
+      // W_o-bound: the few-token projection's streaming kernel where its
+      // shape rules hold, else the cluster-split tensor-core kernel
+      if (gqa::oproj_stream_fits(p)) return launch_status(gqa::launch_oproj_stream(p, d->num_sms, s));
+      return launch_status(gqa::launch_oproj_smallt(p, d->num_sms, s));
+    }
     return launch_status(gqa::launch_oproj_tc(p, d->num_sms, s));
   }
   return launch_status(gqa::launch_oproj_simt(p, dtype == GQA_BF16, s));
@@ -466,6 +471,17 @@ int gqa_debug_set_wait_limit_ns(uint64_t ns) {
     return GQA_ERR_LAUNCH_FAILED;
   }
   return GQA_OK;
+}
+
+int gqa_debug_exp2_poly(const float* x, int n, float* poly, float* ref, void* stream) {
+  if (n < 0) return GQA_ERR_INVALID_ARG;
+  if (n == 0) return GQA_OK;
+  if (!x || !poly || !ref) return GQA_ERR_INVALID_ARG;
+  if (!aligned4(x) || !aligned4(poly) || !aligned4(ref)) return GQA_ERR_MISALIGNED;
+  int st;
+  const DeviceInfo* d = device_info(&st);
+  if (!d) return st;
+  return launch_status(gqa::launch_exp2_check(x, n, poly, ref, static_cast<cudaStream_t>(stream)));
 }
 
 int gqa_debug_skip_next_kv_tile(int tile) {

@@ -137,10 +137,16 @@ cudaError_t launch_qkv_smallm(const QkvParams& p, int num_sms, cudaStream_t st);
 // the reduction dimension split over a thread-block cluster; SIMT for fp32.
 cudaError_t launch_oproj_tc(const OprojParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_oproj_smallt(const OprojParams& p, int num_sms, cudaStream_t st);   // T <= 64
+// the few-token QKV projection's W-streaming kernel with a residual epilogue
+// (T <= 64, K % 64 == 0, N % 16 == 0, tokens' rows fit in shared memory)
+bool oproj_stream_fits(const OprojParams& p);
+cudaError_t launch_oproj_stream(const OprojParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_oproj_simt(const OprojParams& p, bool bf16, cudaStream_t st);
 // FP8 path: amax + quantisation passes, and the tcgen05 kind::f8f6f4 prefill (head_dim 128).
 cudaError_t launch_fp8_quantize(const Fp8QuantParams& p, int num_sms, cudaStream_t st);
 cudaError_t launch_prefill_fp8(const Fp8AttnParams& p, cudaStream_t st);
+// testing aid: tc::exp2_poly2 and exp2f on the same inputs
+cudaError_t launch_exp2_check(const float* x, int n, float* poly, float* ref, cudaStream_t st);
 cudaError_t launch_prefill_pair(const PrefillParams& p, cudaStream_t st);  // head_dim 64, 2 CTAs/SM
 cudaError_t launch_prefill_fa(const PrefillParams& p, cudaStream_t st);    // head_dim 64/128, 2 Q tiles/CTA
 cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head_dim 64 or 128

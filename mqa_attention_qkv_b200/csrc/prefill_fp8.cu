@@ -34,6 +34,13 @@ constexpr int Q_OFF = 0, K_OFF = 2 * TILE, V_OFF = K_OFF + KS * TILE, BAR_OFF = 
 constexpr int SMEM = BAR_OFF + 1024 + 1024;
 constexpr uint32_t O_COL = 256;
 constexpr float kRescaleThreshold = 4.0f, kPOffset = 4.0f;
+// Quads out of every 8 of a row chunk whose 2^x runs as a polynomial on the
+// FMA pipe (tc::exp2_poly2) instead of the MUFU unit, on tiles without a
+// masked key.
+#ifndef GQA_FP8_POLY
+#define GQA_FP8_POLY 0
+#endif
+constexpr int kPoly = GQA_FP8_POLY;
 
 // Instruction descriptor, kind::f8f6f4: e4m3 A and B (format 0), f32
 // accumulator (bits 4-5 = 1), both K-major, N >> 3 at bit 17, M >> 4 at 24.
@@ -299,6 +306,7 @@ prefill_fp8_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
       // P = 2^(s * scale - m + offset) -> e4m3, 4 per column, over S's first 32 columns
       const float neg_m = m_used == -INFINITY ? 0.f : kPOffset - m_used;
       float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+      const bool poly = kPoly > 0 && __all_sync(0xffffffffu, k0 + BKV <= my_lim);   // warp-uniform
 #pragma unroll
       for (int c = 0; c < BKV / 64; ++c) {
         uint32_t w[16];
@@ -308,10 +316,15 @@ prefill_fp8_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constan
           float p2 = s[c * 64 + 4 * e + 2], p3 = s[c * 64 + 4 * e + 3];
           tc::fma2(p0, p1, scale_log2, neg_m);
           tc::fma2(p2, p3, scale_log2, neg_m);
-          p0 = tc::ex2(p0);
-          p1 = tc::ex2(p1);
-          p2 = tc::ex2(p2);
-          p3 = tc::ex2(p3);
+          if (poly && (e & 7) < kPoly) {
+            tc::exp2_poly2(p0, p1);
+            tc::exp2_poly2(p2, p3);
+          } else {
+            p0 = tc::ex2(p0);
+            p1 = tc::ex2(p1);
+            p2 = tc::ex2(p2);
+            p3 = tc::ex2(p3);
+          }
           tc::add2(sa0, sa1, p0, p1);
           tc::add2(sb0, sb1, p2, p3);
           w[e] = pack_e4m3x4(p0, p1, p2, p3);

@@ -40,33 +40,6 @@ constexpr uint32_t kTmemCols = 256, kPCol = 128, kOCol = 192;
 #define GQA_PAIR_POLY 0
 #endif
 constexpr int kPoly = GQA_PAIR_POLY;
-#ifndef GQA_PAIR_PACK
-#define GQA_PAIR_PACK 0
-#endif
-#ifndef GQA_PAIR_F2
-#define GQA_PAIR_F2 0
-#endif
-
-// Two probabilities (finite, >= 0) -> packed bf16 pair, rounded to nearest.
-__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
-  if constexpr (GQA_PAIR_PACK == 1) {
-    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-    a += 0x7FFFu + ((a >> 16) & 1u);
-    b += 0x7FFFu + ((b >> 16) & 1u);
-    return __byte_perm(a, b, 0x7632);
-  } else if constexpr (GQA_PAIR_PACK == 2) {
-    float g0 = lo, g1 = hi;
-    tc::fma2(g0, g1, 65537.0f, 0.0f);
-    float d0 = g0, d1 = g1;
-    tc::fma2v(d0, d1, -1.0f, -1.0f, lo, hi);
-    tc::add2(g0, g1, d0, d1);
-    return __byte_perm(__float_as_uint(g0), __float_as_uint(g1), 0x7632);
-  } else if constexpr (GQA_PAIR_PACK == 3) {
-    return __byte_perm(__float_as_uint(lo), __float_as_uint(hi), 0x7632);
-  } else {
-    return pack_bf16x2(lo, hi);
-  }
-}
 constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t IDESC_S = tc::idesc_bf16(128, 128, false, false);
 constexpr uint32_t IDESC_O = tc::idesc_bf16(128, HD, false, true);
@@ -347,30 +320,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
               p1 = tc::ex2(p1);
             }
             if (i & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
-            w[i] = pack_p(p0, p1);
+            w[i] = pack_bf16x2(p0, p1);
           }
           tc::tmem_st16(tmem + lane_base + kPCol + c * 16, w);
         }
-      } else if constexpr (GQA_PAIR_F2) {
-        const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(neg_m, neg_m);
-        float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < BKV / 32; ++c) {
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float2 pp = __ffma2_rn(make_float2(s[c * 32 + 2 * i], s[c * 32 + 2 * i + 1]), sc2, nm2);
-            pp.x = tc::ex2(pp.x);
-            pp.y = tc::ex2(pp.y);
-            if (i & 1) acc_b = __fadd2_rn(acc_b, pp); else acc_a = __fadd2_rn(acc_a, pp);
-            w[i] = pack_p(pp.x, pp.y);
-          }
-          tc::tmem_st16(tmem + lane_base + kPCol + c * 16, w);
-        }
-        sa0 = acc_a.x;
-        sa1 = acc_a.y;
-        sb0 = acc_b.x;
-        sb1 = acc_b.y;
       } else {
 #pragma unroll
         for (int c = 0; c < BKV / 32; ++c) {
@@ -382,7 +335,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
             p0 = tc::ex2(p0);
             p1 = tc::ex2(p1);
             if (i & 1) add2(sb0, sb1, p0, p1); else add2(sa0, sa1, p0, p1);
-            w[i] = pack_p(p0, p1);
+            w[i] = pack_bf16x2(p0, p1);
           }
           tc::tmem_st16(tmem + lane_base + kPCol + c * 16, w);
         }

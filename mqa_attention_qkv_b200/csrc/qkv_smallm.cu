@@ -206,16 +206,60 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
 }
 
-template <int NT, int HD>
+// Epilogues of the streaming kernel.  A work unit is 16 rows of W: 8 "lo"
+// rows at unit_row(u) and 8 "hi" rows HD/2 further on (HD = 16: 16
+// consecutive rows).  store() gets the finished dot products of lo row
+// unit_row(u) + r and its hi partner with token `tok`.
+template <int HD_>
+struct StreamQkv {                         // QKV projection: RoPE pair + scatter
+  static constexpr int HD = HD_;
+  using Params = QkvParams;
+  __device__ static int T(const Params& p) { return p.B * p.S; }
+  __device__ static int K(const Params& p) { return p.hidden; }
+  __device__ static const void* X(const Params& p) { return p.x; }
+  __device__ static int* err(const Params& p) { return p.err; }
+  __device__ static void init(const Params& p, double* table) {
+    for (int f = threadIdx.x; f < HD / 2; f += SW_WARPS * 32) table[f] = rope_inv_freq(f, HD, p.theta);
+  }
+  __device__ static void store(const Params& p, int u, int r, int tok, float lo, float hi, const double* table) {
+    constexpr int GROUPS = HD / 16;
+    const int hb = u / GROUPS, i0 = (u % GROUPS) * 8;
+    rope_store_pair<HD>(p, hb, i0, r, tok, lo, hi, table[i0 + r]);
+  }
+};
+
+struct StreamResidual {                    // output projection: + residual, round once
+  static constexpr int HD = 16;
+  using Params = OprojParams;
+  __device__ static int T(const Params& p) { return p.T; }
+  __device__ static int K(const Params& p) { return p.K; }
+  __device__ static const void* X(const Params& p) { return p.x; }
+  __device__ static int* err(const Params& p) { return p.err; }
+  __device__ static void init(const Params&, double*) {}
+  __device__ static void store(const Params& p, int u, int r, int tok, float lo, float hi, const double*) {
+    const size_t o = (size_t)tok * p.N + u * 16 + r;
+    const __nv_bfloat16* res = static_cast<const __nv_bfloat16*>(p.residual);
+    if (res) {
+      lo += __bfloat162float(res[o]);
+      hi += __bfloat162float(res[o + 8]);
+    }
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
+    out[o] = __float2bfloat16_rn(lo);
+    out[o + 8] = __float2bfloat16_rn(hi);
+  }
+};
+
+template <int NT, class Epi>
 __global__ void __launch_bounds__((SW_WARPS + 1) * 32, 1)
-qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
-                  int n_units, int nstages) {
+w_stream_kernel(const __grid_constant__ CUtensorMap tmw, typename Epi::Params p,
+                int n_units, int nstages) {
   constexpr int TP = NT * 8;
+  constexpr int HD = Epi::HD;
   constexpr int GROUPS = HD / 16;
   constexpr int XBOX = TP * 128;                   // one 64-column block of X
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int nblk = p.hidden / 64;
+  const int nblk = Epi::K(p) / 64;
   const int nst = (nblk + SW_KB - 1) / SW_KB;
   uint8_t* ring = smem;
   uint8_t* xs = smem + nstages * SW_STAGE;
@@ -224,8 +268,8 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
   uint64_t* empty = full + SW_STAGES;
   double* inv_freq = reinterpret_cast<double*>(empty + SW_STAGES);   // [HD / 2]
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int T = p.B * p.S;
-  int* err = p.err;
+  const int T = Epi::T(p);
+  int* err = Epi::err(p);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstages; ++s) {
@@ -285,7 +329,8 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
     // rows; rows past T zero) by the consumer threads, 8 vectors in flight
     // each, while the producer fills the W ring.  (Fetched by TMA next to
     // the W slabs, the same X measured markedly slower on B200.)
-    const __nv_bfloat16* X = static_cast<const __nv_bfloat16*>(p.x);
+    const __nv_bfloat16* X = static_cast<const __nv_bfloat16*>(Epi::X(p));
+    const int hidden = Epi::K(p);
     const int nchunk = nblk * TP * 8;
     for (int e0 = threadIdx.x; e0 < nchunk; e0 += SW_WARPS * 32 * 8) {
       uint4 v[8];
@@ -295,7 +340,7 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
         const int kb = e / (TP * 8), rem = e % (TP * 8), row = rem / 8, ch = rem % 8;
         v[i] = make_uint4(0, 0, 0, 0);
         if (e < nchunk && row < T)
-          v[i] = *reinterpret_cast<const uint4*>(X + (size_t)row * p.hidden + kb * 64 + ch * 8);
+          v[i] = *reinterpret_cast<const uint4*>(X + (size_t)row * hidden + kb * 64 + ch * 8);
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -304,8 +349,8 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
         if (e < nchunk) *reinterpret_cast<uint4*>(xs + kb * XBOX + row * 128 + ((ch ^ (row & 7)) << 4)) = v[i];
       }
     }
-    // the RoPE frequencies of the head dimension, once per CTA
-    for (int f = threadIdx.x; f < HD / 2; f += SW_WARPS * 32) inv_freq[f] = rope_inv_freq(f, HD, p.theta);
+    // the epilogue's per-CTA table (the RoPE frequencies of the head dimension)
+    Epi::init(p, inv_freq);
     asm volatile("bar.sync 1, %0;" ::"n"(SW_WARPS * 32) : "memory");
   }
   bool dead = false;
@@ -374,7 +419,6 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
       rw[(g + 8) * (TP + 1) + n * 8 + 2 * tq + 1] = acc[n][3];
     }
     asm volatile("bar.sync 1, %0;" ::"n"(SW_WARPS * 32) : "memory");
-    const int hb = u / GROUPS, i0 = (u % GROUPS) * 8;
     for (int e = threadIdx.x; e < 8 * T; e += SW_WARPS * 32) {
       const int r = e & 7, tok = e >> 3;
       float lo = 0.f, hi = 0.f;
@@ -383,20 +427,20 @@ qkv_stream_kernel(const __grid_constant__ CUtensorMap tmw, QkvParams p,
         lo += red[(w * 16 + r) * (TP + 1) + tok];
         hi += red[(w * 16 + r + 8) * (TP + 1) + tok];
       }
-      if (!dead) rope_store_pair<HD>(p, hb, i0, r, tok, lo, hi, inv_freq[i0 + r]);
+      if (!dead) Epi::store(p, u, r, tok, lo, hi, inv_freq);
     }
     asm volatile("bar.sync 1, %0;" ::"n"(SW_WARPS * 32) : "memory");
   }
 }
 
-template <int NT, int HD>
-cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
-  const int nblk = p.hidden / 64;
+template <int NT, class Epi>
+cudaError_t launch_stream_epi(const typename Epi::Params& p, const void* w, int K, int N, int num_sms,
+                              cudaStream_t st) {
+  const int nblk = K / 64;
   static std::atomic<bool> attr_set[64];
-  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(qkv_stream_kernel<NT, HD>), SW_SMEM_MAX);
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(w_stream_kernel<NT, Epi>), SW_SMEM_MAX);
       e != cudaSuccess)
     return e;
-  const int N = (p.nh + 2 * p.nkv) * HD;
   const int n_units = N / 16;
   // More units than SMs and small hidden states: two CTAs per SM with a
   // shorter ring each, so that a few hundred units run in one wave instead
@@ -412,7 +456,7 @@ cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
       known = -1;
       for (int s2 = SW_STAGES; s2 >= 3; --s2) {
         int fit = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, qkv_stream_kernel<NT, HD>, (SW_WARPS + 1) * 32,
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, w_stream_kernel<NT, Epi>, (SW_WARPS + 1) * 32,
                                                           stream_smem(NT, nblk, s2)) != cudaSuccess) {
           cudaGetLastError();
           break;
@@ -433,12 +477,17 @@ cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
   CUtensorMap tw;
   // W viewed as [column block][row][64 columns]: a box is 8 blocks x 8 rows
   const uint64_t wd[3] = {64, (uint64_t)N, (uint64_t)nblk};
-  const uint64_t ws[2] = {(uint64_t)p.hidden * 2, 128};
+  const uint64_t ws[2] = {(uint64_t)K * 2, 128};
   const uint32_t wbox[3] = {64, 8, SW_KB};
-  if (!make_tmap_bf16_3d(&tw, p.w, wd, ws, wbox)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_3d(&tw, w, wd, ws, wbox)) return cudaErrorInvalidValue;
   const int grid = n_units < per_sm * num_sms ? n_units : per_sm * num_sms;
-  qkv_stream_kernel<NT, HD><<<grid, (SW_WARPS + 1) * 32, smem, st>>>(tw, p, n_units, stages);
+  w_stream_kernel<NT, Epi><<<grid, (SW_WARPS + 1) * 32, smem, st>>>(tw, p, n_units, stages);
   return cudaGetLastError();
+}
+
+template <int NT, int HD>
+cudaError_t launch_stream_hd(const QkvParams& p, int num_sms, cudaStream_t st) {
+  return launch_stream_epi<NT, StreamQkv<HD>>(p, p.w, p.hidden, (p.nh + 2 * p.nkv) * HD, num_sms, st);
 }
 
 template <int NT>
@@ -465,6 +514,22 @@ cudaError_t launch_nt(const QkvParams& p, cudaStream_t st) {
 }
 
 }  // namespace
+
+bool oproj_stream_fits(const OprojParams& p) {
+  if (p.T > 64 || p.K % 64 != 0 || p.N % 16 != 0) return false;
+  const int nt = p.T <= 8 ? 1 : p.T <= 16 ? 2 : p.T <= 32 ? 4 : 8;
+  return stream_smem(nt, p.K / 64) <= (size_t)SW_SMEM_MAX;
+}
+
+cudaError_t launch_oproj_stream(const OprojParams& p, int num_sms, cudaStream_t st) {
+  if (!oproj_stream_fits(p)) return cudaErrorInvalidValue;
+  switch (p.T <= 8 ? 1 : p.T <= 16 ? 2 : p.T <= 32 ? 4 : 8) {
+    case 1: return launch_stream_epi<1, StreamResidual>(p, p.w, p.K, p.N, num_sms, st);
+    case 2: return launch_stream_epi<2, StreamResidual>(p, p.w, p.K, p.N, num_sms, st);
+    case 4: return launch_stream_epi<4, StreamResidual>(p, p.w, p.K, p.N, num_sms, st);
+    default: return launch_stream_epi<8, StreamResidual>(p, p.w, p.K, p.N, num_sms, st);
+  }
+}
 
 cudaError_t launch_qkv_smallm(const QkvParams& p, int num_sms, cudaStream_t st) {
   const int T = p.B * p.S;

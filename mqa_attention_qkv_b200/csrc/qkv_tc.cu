@@ -30,14 +30,24 @@
 namespace gqa {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int TMEM_COLS = 2 * BN;
+constexpr int BM = 128, BK = 64, MAX_STAGES = 8;
 constexpr int THREADS = 192;
-constexpr uint32_t IDESC = tc::idesc_bf16(BM, BN, false, false);
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*barriers, tables*/;
+
+// Tile width and ring depth.  Wide (N 256, 4 stages) for many-token
+// problems; narrow (N 64 or 128, 8 or 6 stages) when the wide tiles would
+// leave most SMs idle (a 128-token projection is 10 tiles wide): more, thinner
+// tiles and more bytes in flight per SM.
+template <int BN_, int STAGES_>
+struct GemmCfg {
+  static constexpr int BN = BN_, STAGES = STAGES_;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;     // two accumulators
+  static constexpr uint32_t IDESC = tc::idesc_bf16(BM, BN, false, false);
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*barriers, tables*/;
+  static_assert(STAGES <= MAX_STAGES, "barrier arrays");
+};
 
 template <class P>
 struct TcArgs {
@@ -46,7 +56,7 @@ struct TcArgs {
 };
 
 struct Bars {
-  uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain;
+  uint64_t full[MAX_STAGES], empty[MAX_STAGES], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
   int abort;
   double inv_freq[64];
@@ -62,8 +72,10 @@ struct QkvEpilogue {
     if (threadIdx.x >= 64 && threadIdx.x < 64 + HD / 2)
       bars->inv_freq[threadIdx.x - 64] = rope_inv_freq(threadIdx.x - 64, HD, p.theta);
   }
+  template <int BN>
   __device__ static void tile(const TcArgs<Params>& a, const Bars* bars, uint32_t tbase, int m0, int n0, int row) {
     constexpr int HALF = HD / 2, CHUNKS = HALF / 16, HEADS = BN / HD;
+    static_assert(BN % HD == 0, "tiles hold whole heads");
     const Params& p = a.p;
     int* err = p.err;
     const int t = m0 + row;
@@ -137,6 +149,7 @@ struct QkvEpilogue {
 struct ResidualEpilogue {
   using Params = OprojParams;
   __device__ static void init(const Params&, Bars*) {}
+  template <int BN>
   __device__ static void tile(const TcArgs<Params>& a, const Bars*, uint32_t tbase, int m0, int n0, int row) {
     const Params& p = a.p;
     const int t = m0 + row;
@@ -175,10 +188,13 @@ struct ResidualEpilogue {
   }
 };
 
-template <class Epi>
+template <class Epi, class Cfg>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
                TcArgs<typename Epi::Params> a) {
+  constexpr int BN = Cfg::BN, STAGES = Cfg::STAGES, A_BYTES = Cfg::A_BYTES, STAGE_BYTES = Cfg::STAGE_BYTES;
+  constexpr int TMEM_COLS = Cfg::TMEM_COLS;
+  constexpr uint32_t IDESC = Cfg::IDESC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
@@ -231,7 +247,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
       for (int s = 0; s < STAGES; ++s) {
         int st = (stage + s) % STAGES;
         uint32_t ph = (st < stage) ? phase : phase ^ 1;  // phase of the last load issued into st
-        mbar_wait(&bars->full[st], ph, err);
+        mbar_wait_drain(&bars->full[st], ph, err);
       }
     }
   } else if (warp == 1) {
@@ -265,7 +281,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
       if (!ok) atomicExch(&bars->abort, 1);
       // all MMAs done before TMEM is released
       tc::mma_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0, err);
+      mbar_wait_drain(&bars->drain, 0, err);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -279,7 +295,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
       tc::fence_after_sync();
       const int m0 = (tile / a.num_n) * BM, n0 = (tile % a.num_n) * BN;
       const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + buf * BN;
-      Epi::tile(a, bars, tbase, m0, n0, row);
+      Epi::template tile<BN>(a, bars, tbase, m0, n0, row);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
@@ -295,26 +311,40 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
   }
 }
 
-template <class Epi>
-cudaError_t launch_gemm(const typename Epi::Params& p, const void* x, const void* w, int T, int K, int N, int n_heads_total,
-                        int num_sms, cudaStream_t st) {
+template <class Epi, class Cfg>
+cudaError_t launch_cfg(const typename Epi::Params& p, const void* x, const void* w, int T, int K, int N,
+                       int n_heads_total, int num_sms, cudaStream_t st) {
   static std::atomic<bool> attr_set[64];
-  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(gemm_tc_kernel<Epi>), SMEM_BYTES);
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(gemm_tc_kernel<Epi, Cfg>),
+                                     Cfg::SMEM_BYTES);
       e != cudaSuccess)
     return e;
   TcArgs<typename Epi::Params> a;
   a.p = p;
   a.T = T;
   a.n_heads_total = n_heads_total;
-  a.num_n = (N + BN - 1) / BN;
+  a.num_n = (N + Cfg::BN - 1) / Cfg::BN;
   a.num_tiles = ((T + BM - 1) / BM) * a.num_n;
   a.num_kb = (K + BK - 1) / BK;
   CUtensorMap tx, tw;
   if (!make_tmap_bf16_2d(&tx, x, K, T, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16_2d(&tw, w, K, N, (uint64_t)K * 2, BK, BN)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16_2d(&tw, w, K, N, (uint64_t)K * 2, BK, Cfg::BN)) return cudaErrorInvalidValue;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
-  gemm_tc_kernel<Epi><<<grid, THREADS, SMEM_BYTES, st>>>(tx, tw, a);
+  gemm_tc_kernel<Epi, Cfg><<<grid, THREADS, Cfg::SMEM_BYTES, st>>>(tx, tw, a);
   return cudaGetLastError();
+}
+
+// Wide tiles unless they would leave more than half of the SMs idle; then
+// the narrowest tile that still holds whole heads (`min_bn`).
+template <class Epi, int MIN_BN>
+cudaError_t launch_gemm(const typename Epi::Params& p, const void* x, const void* w, int T, int K, int N,
+                        int n_heads_total, int num_sms, cudaStream_t st) {
+  const long long wide_tiles = (long long)((T + BM - 1) / BM) * ((N + 255) / 256);
+  if (2 * wide_tiles >= num_sms) return launch_cfg<Epi, GemmCfg<256, 4>>(p, x, w, T, K, N, n_heads_total, num_sms, st);
+  if constexpr (MIN_BN <= 64)
+    return launch_cfg<Epi, GemmCfg<64, 8>>(p, x, w, T, K, N, n_heads_total, num_sms, st);
+  else
+    return launch_cfg<Epi, GemmCfg<128, 6>>(p, x, w, T, K, N, n_heads_total, num_sms, st);
 }
 
 }  // namespace
@@ -322,15 +352,15 @@ cudaError_t launch_gemm(const typename Epi::Params& p, const void* x, const void
 cudaError_t launch_qkv_tc(const QkvParams& p, int num_sms, cudaStream_t st) {
   const int T = p.B * p.S, heads = p.nh + 2 * p.nkv, N = heads * p.hd;
   switch (p.hd) {
-    case 32: return launch_gemm<QkvEpilogue<32>>(p, p.x, p.w, T, p.hidden, N, heads, num_sms, st);
-    case 64: return launch_gemm<QkvEpilogue<64>>(p, p.x, p.w, T, p.hidden, N, heads, num_sms, st);
-    case 128: return launch_gemm<QkvEpilogue<128>>(p, p.x, p.w, T, p.hidden, N, heads, num_sms, st);
+    case 32: return launch_gemm<QkvEpilogue<32>, 64>(p, p.x, p.w, T, p.hidden, N, heads, num_sms, st);
+    case 64: return launch_gemm<QkvEpilogue<64>, 64>(p, p.x, p.w, T, p.hidden, N, heads, num_sms, st);
+    case 128: return launch_gemm<QkvEpilogue<128>, 128>(p, p.x, p.w, T, p.hidden, N, heads, num_sms, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
 cudaError_t launch_oproj_tc(const OprojParams& p, int num_sms, cudaStream_t st) {
-  return launch_gemm<ResidualEpilogue>(p, p.x, p.w, p.T, p.K, p.N, 0, num_sms, st);
+  return launch_gemm<ResidualEpilogue, 64>(p, p.x, p.w, p.T, p.K, p.N, 0, num_sms, st);
 }
 
 }  // namespace gqa

@@ -12,6 +12,7 @@
 //                  thread (float32, and bf16 widths the tensor path skips)
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace gqa {
 namespace {
@@ -406,6 +407,28 @@ cudaError_t launch_oproj_simt(const OprojParams& p, bool bf16, cudaStream_t st) 
     oproj_simt_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(p);
   else
     oproj_simt_kernel<float><<<grid, 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+namespace {
+// testing aid: the prefill softmax's polynomial 2^x next to CUDA's exp2f
+__global__ void exp2_check_kernel(const float* x, int n, float* poly, float* ref) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  float a = x[i], b = i + 1 < n ? x[i + 1] : 0.f;
+  const float ra = exp2f(a), rb = exp2f(b);
+  tc::exp2_poly2(a, b);
+  poly[i] = a;
+  ref[i] = ra;
+  if (i + 1 < n) {
+    poly[i + 1] = b;
+    ref[i + 1] = rb;
+  }
+}
+}  // namespace
+
+cudaError_t launch_exp2_check(const float* x, int n, float* poly, float* ref, cudaStream_t st) {
+  exp2_check_kernel<<<(unsigned)((n + 511) / 512), 256, 0, st>>>(x, n, poly, ref);
   return cudaGetLastError();
 }
 

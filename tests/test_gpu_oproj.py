@@ -25,8 +25,10 @@ def _inputs(seed, T, nh, hd, hidden, dtype):
 
 
 CASES = [
-    # T, n_heads, head_dim, hidden
+    # T, n_heads, head_dim, hidden (T <= 64: the W-streaming kernel when nh*hd % 64 == 0 and hidden % 16 == 0,
+    # else the cluster-split tensor-core kernel: (13, 5, 32, 264), (33, 8, 128, 1032), (40, 8, 64, 2056))
     (1, 32, 64, 2048), (8, 32, 64, 2048), (13, 5, 32, 264), (33, 8, 128, 1032), (64, 32, 64, 2048),
+    (40, 8, 64, 2056), (20, 6, 32, 1040),
     (8, 48, 128, 6144),                               # MQA generation step shape
     (65, 32, 64, 2048), (200, 5, 32, 264), (300, 8, 128, 1032), (1000, 16, 64, 1024),
 ]
