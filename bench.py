@@ -348,8 +348,10 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_workloads:
         step_check = check_layer_step(sets[0], B, S, nh, nkv, hd, wl["theta"])
         del sets
-        wls = measure_workloads(dev, {"hbm_gbs": hbm_peak, "bf16_tflops": bf16_peak})
-        wls["tiny_fp32_layer"] = check_tiny_fp32(dev)
+        only = set(args.workloads.split(",")) if args.workloads else None
+        wls = measure_workloads(dev, {"hbm_gbs": hbm_peak, "bf16_tflops": bf16_peak}, only=only)
+        if only is None or "tiny" in only:
+            wls["tiny_fp32_layer"] = check_tiny_fp32(dev)
 
     if world > 1:
         dist.barrier(device_ids=[local])
@@ -1011,6 +1013,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the per-kernel measurements of the decode, 8K-prefill and generation workloads")
+    ap.add_argument("--workloads", default=None,
+                    help="comma-separated workload sections to measure (decode, prefill8k, generate, small, "
+                         "varlen, meanpool, tiny); default all")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, always
