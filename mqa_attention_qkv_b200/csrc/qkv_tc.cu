@@ -19,11 +19,13 @@
 //               fp32 accumulators in TMEM (double buffered across tiles)
 //   warps 2-5   epilogue: thread = token row; tcgen05.ld the accumulator.
 //               QKV: rotate q/k feature pairs (i, i + hd/2) in fp32, round to
-//               bf16 once and store each head straight to q_out
-//               [B, nh, S, hd] or to the cache row [b, j, position]; tiles are
-//               128 tokens x 256 fused features, i.e. whole heads, so a
-//               rotation pair never leaves the thread that holds it.
+//               bf16 once and store each head to q_out [B, nh, S, hd] or to
+//               the cache row [b, j, position]; tiles are 128 tokens x 256
+//               fused features, i.e. whole heads, so a rotation pair never
+//               leaves the thread that holds it.
 //               Output projection: add the residual row in fp32, round once.
+//               Both stage their rows in shared memory and write whole
+//               128-byte lines (see the staging note below).
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -59,25 +61,62 @@ struct Bars {
   uint64_t full[MAX_STAGES], empty[MAX_STAGES], acc_full[2], acc_empty[2], drain;
   uint32_t tmem_base;
   int abort;
-  double inv_freq[64];
+  unsigned long long rope_step[64];   // RoPE angle steps in fixed-point turns (rope_turn_step)
 };
+static_assert(sizeof(Bars) <= 1024, "barrier block");
+
+// Epilogue staging.  Each epilogue warp owns 32 accumulator rows (its TMEM
+// lane quarter) and a shared-memory staging area of 32 rows.  A thread first
+// writes its own row there (16-byte chunk c of row r at chunk c ^ (r & 7), so
+// the 32 rows of a warp spread over all banks); the warp then copies the rows
+// out with consecutive lanes on consecutive 16-byte chunks of one row, so
+// every store instruction writes whole 128-byte lines of 4 (or 2) rows.
+// Row-per-thread stores of 16 bytes would touch 32 lines per instruction,
+// and on B200 those partial-line requests slowed the concurrent operand
+// stream of the main loop through L2.
+__device__ __forceinline__ uint32_t stage_chunk(uint32_t row_base, int r, int c, int mask) {
+  return row_base + (uint32_t)((c ^ (r & mask)) * 16);
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a)
+               : "memory");
+  return v;
+}
+// 16 bytes global -> shared without registers; src_bytes 0 writes zeros
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Epilogue of the QKV projection: RoPE on q/k, head-major scatter.  One
-// thread owns token row `row` of the 128 x 256 tile at (m0, n0); `tbase` is
-// its TMEM lane in the accumulator buffer.
+// thread owns token row `row` of the 128 x BN tile at (m0, n0); `tbase` is
+// its TMEM lane in the accumulator buffer; `stage` is its warp's staging
+// area (32 rows of one head).  A tile holds whole heads, so a rotation pair
+// (i, i + hd/2) never leaves the thread that holds it.
 template <int HD>
 struct QkvEpilogue {
   using Params = QkvParams;
+  static constexpr int kStageBytes = 32 * HD * 2;   // per warp: 32 rows of one head
   __device__ static void init(const Params& p, Bars* bars) {
     if (threadIdx.x >= 64 && threadIdx.x < 64 + HD / 2)
-      bars->inv_freq[threadIdx.x - 64] = rope_inv_freq(threadIdx.x - 64, HD, p.theta);
+      bars->rope_step[threadIdx.x - 64] = rope_turn_step(rope_inv_freq(threadIdx.x - 64, HD, p.theta));
   }
   template <int BN>
-  __device__ static void tile(const TcArgs<Params>& a, const Bars* bars, uint32_t tbase, int m0, int n0, int row) {
+  __device__ static void prefetch(const TcArgs<Params>&, int, int, int, uint32_t) {}
+  template <int BN>
+  __device__ static void tile(const TcArgs<Params>& a, const Bars* bars, uint32_t tbase, int m0, int n0, int row,
+                              uint32_t stage) {
     constexpr int HALF = HD / 2, CHUNKS = HALF / 16, HEADS = BN / HD;
+    constexpr int ROWB = HD * 2, RCH = ROWB / 16;          // bytes and 16-byte chunks of a head row
+    constexpr int MASK = RCH < 8 ? RCH - 1 : 7;
+    constexpr int LPR = RCH, RPI = 32 / LPR;               // copy-out: lanes per row, rows per instruction
     static_assert(BN % HD == 0, "tiles hold whole heads");
     const Params& p = a.p;
     int* err = p.err;
+    const int lane = threadIdx.x % 32;
     const int t = m0 + row;
     const bool valid = t < a.T;
     int b = 0, s = 0, pos = 0;
@@ -88,38 +127,37 @@ struct QkvEpilogue {
     }
     const bool pos_ok = pos >= 0 && pos < p.cap;
     const int hb0 = n0 / HD;
+    const uint32_t my_row = stage + lane * ROWB;
+    const int cc = lane % LPR, rsub = lane / LPR;
 #pragma unroll 1
-    for (int c = 0; c < CHUNKS; ++c) {
-      float cs[16], sn[16];
+    for (int hh = 0; hh < HEADS; ++hh) {
+      const int hb = hb0 + hh;
+      if (hb >= a.n_heads_total) break;  // ragged N tail: uniform over the CTA
+      const bool is_q = hb < p.nh, is_k = !is_q && hb < p.nh + p.nkv;
+      __nv_bfloat16* dst = nullptr;
       if (valid) {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) rope_cos_sin(pos, bars->inv_freq[c * 16 + k], &cs[k], &sn[k]);
+        if (is_q) {
+          dst = static_cast<__nv_bfloat16*>(p.q_out) + (((size_t)b * p.nh + hb) * p.S + s) * HD;
+        } else if (pos_ok) {
+          const int j = is_k ? hb - p.nh : hb - p.nh - p.nkv;
+          dst = static_cast<__nv_bfloat16*>(is_k ? p.k_cache : p.v_cache) +
+                (((size_t)b * p.nkv + j) * p.cap + pos) * HD;
+        } else {
+          raise_error(err, GQA_DEVERR_POSITION_RANGE);
+        }
       }
 #pragma unroll 1
-      for (int hh = 0; hh < HEADS; ++hh) {
-        const int hb = hb0 + hh;
-        if (hb >= a.n_heads_total) break;  // ragged N tail: uniform over the CTA
+      for (int c = 0; c < CHUNKS; ++c) {
         uint32_t lo[16], hi[16];
         __syncwarp();  // the .sync.aligned TMEM load needs the whole warp converged
         tc::tmem_ld16(tbase + hh * HD + c * 16, lo);
         tc::tmem_ld16(tbase + hh * HD + HALF + c * 16, hi);
-        tc::tmem_ld_wait();
-        if (!valid) continue;
-        const bool is_q = hb < p.nh, is_k = !is_q && hb < p.nh + p.nkv;
-        __nv_bfloat16* dst;
-        if (is_q) {
-          dst = static_cast<__nv_bfloat16*>(p.q_out) + (((size_t)b * p.nh + hb) * p.S + s) * HD;
-        } else {
-          if (!pos_ok) {
-            if (c == 0) raise_error(err, GQA_DEVERR_POSITION_RANGE);
-            continue;
-          }
-          const int j = is_k ? hb - p.nh : hb - p.nh - p.nkv;
-          dst = static_cast<__nv_bfloat16*>(is_k ? p.k_cache : p.v_cache) +
-                (((size_t)b * p.nkv + j) * p.cap + pos) * HD;
-        }
         uint32_t olo[8], ohi[8];
         if (is_q || is_k) {
+          float cs[16], sn[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) rope_cos_sin_fx(pos, bars->rope_step[c * 16 + k], &cs[k], &sn[k]);
+          tc::tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < 16; k += 2) {
             const float x0 = __uint_as_float(lo[k]), y0 = __uint_as_float(hi[k]);
@@ -128,62 +166,125 @@ struct QkvEpilogue {
             ohi[k / 2] = pack_bf16x2(y0 * cs[k] + x0 * sn[k], y1 * cs[k + 1] + x1 * sn[k + 1]);
           }
         } else {
+          tc::tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < 16; k += 2) {
             olo[k / 2] = pack_bf16x2(__uint_as_float(lo[k]), __uint_as_float(lo[k + 1]));
             ohi[k / 2] = pack_bf16x2(__uint_as_float(hi[k]), __uint_as_float(hi[k + 1]));
           }
         }
-        tc::st_global_v4(dst + c * 16, olo[0], olo[1], olo[2], olo[3]);
-        tc::st_global_v4(dst + c * 16 + 8, olo[4], olo[5], olo[6], olo[7]);
-        tc::st_global_v4(dst + HALF + c * 16, ohi[0], ohi[1], ohi[2], ohi[3]);
-        tc::st_global_v4(dst + HALF + c * 16 + 8, ohi[4], ohi[5], ohi[6], ohi[7]);
+        // features c*16.. and HALF + c*16.. of the head row: chunks 2c, 2c+1 and RCH/2 + 2c, +1
+        tc::st_shared_v4(stage_chunk(my_row, lane, 2 * c, MASK), olo[0], olo[1], olo[2], olo[3]);
+        tc::st_shared_v4(stage_chunk(my_row, lane, 2 * c + 1, MASK), olo[4], olo[5], olo[6], olo[7]);
+        tc::st_shared_v4(stage_chunk(my_row, lane, RCH / 2 + 2 * c, MASK), ohi[0], ohi[1], ohi[2], ohi[3]);
+        tc::st_shared_v4(stage_chunk(my_row, lane, RCH / 2 + 2 * c + 1, MASK), ohi[4], ohi[5], ohi[6], ohi[7]);
       }
+      __syncwarp();
+      // copy-out: instruction i writes rows i*RPI .. i*RPI + RPI-1, LPR lanes per row
+#pragma unroll
+      for (int i = 0; i < 32 / RPI; ++i) {
+        const int rr = i * RPI + rsub;
+        const unsigned long long d = __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), rr);
+        const uint4 v = ld_shared_v4(stage_chunk(stage + rr * ROWB, rr, cc, MASK));
+        if (d) tc::st_global_v4(reinterpret_cast<uint8_t*>(d) + cc * 16, v.x, v.y, v.z, v.w);
+      }
+      __syncwarp();  // the staging rows are rewritten by the next head
     }
   }
 };
 
 // Epilogue of the output projection: out = acc + residual, rounded once.
-// Columns are stored in 8-wide vectors; a vector past N (N % 8 == 0) is
-// skipped, so a ragged N tail needs no masking inside a vector.
+// The tile's columns go in groups of 64 (one 128-byte staging row per
+// thread).  The residual of each group is fetched into the staging area with
+// coalesced cp.async copies, double-buffered: group 0 is requested before the
+// accumulator is ready, group g + 1 while group g is added and stored.  The
+// thread owning a row adds its accumulator columns to the staged residual in
+// place, then the warp copies the rows out as whole lines.  Columns go in
+// 8-wide vectors; a vector past N (N % 8 == 0) is neither read nor written,
+// so a ragged N tail needs no masking inside a vector.  out may be the
+// residual buffer: a tile's residual is read before its output is written,
+// and no other CTA touches the tile.
 struct ResidualEpilogue {
   using Params = OprojParams;
+  static constexpr int G = 64;                         // columns per group
+  static constexpr int kBufBytes = 32 * G * 2;         // one group of 32 rows
+  static constexpr int kStageBytes = 2 * kBufBytes;    // double-buffered
   __device__ static void init(const Params&, Bars*) {}
+  // cp.async of the residual's group g (rows m0 + 32w .. +31) into buffer g & 1
   template <int BN>
-  __device__ static void tile(const TcArgs<Params>& a, const Bars*, uint32_t tbase, int m0, int n0, int row) {
-    const Params& p = a.p;
-    const int t = m0 + row;
-    const bool valid = t < a.T;
+  __device__ static void fetch(const Params& p, int T, int m0w, int n0, int g, uint32_t stage) {
+    const int lane = threadIdx.x % 32, cc = lane % 8, rsub = lane / 8;
+    const uint32_t buf = stage + (g & 1) * kBufBytes;
     const __nv_bfloat16* res = static_cast<const __nv_bfloat16*>(p.residual);
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + (size_t)t * p.N;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = i * 4 + rsub, t = m0w + rr, n = n0 + g * G + cc * 8;
+      const bool in = t < T && n < p.N;
+      cp_async_16(stage_chunk(buf + rr * 128, rr, cc, 7), in ? res + (size_t)t * p.N + n : res, in ? 16 : 0);
+    }
+    cp_async_commit();
+  }
+  template <int BN>
+  __device__ static void prefetch(const TcArgs<Params>& a, int m0, int n0, int q4, uint32_t stage) {
+    if (a.p.residual) fetch<BN>(a.p, a.T, m0 + 32 * q4, n0, 0, stage);
+  }
+  template <int BN>
+  __device__ static void tile(const TcArgs<Params>& a, const Bars*, uint32_t tbase, int m0, int n0, int row,
+                              uint32_t stage) {
+    constexpr int NG = BN / G;
+    const Params& p = a.p;
+    const bool has_res = p.residual != nullptr;
+    const int lane = threadIdx.x % 32, cc = lane % 8, rsub = lane / 8;
+    const int m0w = m0 + (row - lane);
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
 #pragma unroll 1
-    for (int c = 0; c < BN / 16; ++c) {
-      const int n = n0 + c * 16;
-      if (n >= p.N) break;   // uniform over the CTA
-      uint32_t v[16];
-      __syncwarp();
-      tc::tmem_ld16(tbase + c * 16, v);
-      tc::tmem_ld_wait();
-      if (!valid) continue;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (n + 8 * h >= p.N) break;
-        float f[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(v[8 * h + k]);
-        if (res) {
-          const uint4 r = *reinterpret_cast<const uint4*>(res + (size_t)t * p.N + n + 8 * h);
-          const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&rw[k]);
-            f[2 * k] += __low2float(b2);
-            f[2 * k + 1] += __high2float(b2);
-          }
+    for (int g = 0; g < NG; ++g) {
+      if (n0 + g * G >= p.N) break;  // uniform over the CTA
+      const uint32_t buf = stage + (g & 1) * kBufBytes;
+      if (has_res) {
+        if (g + 1 < NG && n0 + (g + 1) * G < p.N) {
+          fetch<BN>(p, a.T, m0w, n0, g + 1, stage);
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
         }
-        tc::st_global_v4(out + n + 8 * h, pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                         pack_bf16x2(f[6], f[7]));
       }
+      __syncwarp();
+      const uint32_t my_row = buf + lane * 128;
+#pragma unroll
+      for (int c = 0; c < G / 16; ++c) {
+        uint32_t v[16];
+        __syncwarp();
+        tc::tmem_ld16(tbase + g * G + c * 16, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t addr = stage_chunk(my_row, lane, 2 * c + h, 7);
+          float f[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) f[k] = __uint_as_float(v[8 * h + k]);
+          if (has_res) {
+            const uint4 r = ld_shared_v4(addr);
+            const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&rw[k]);
+              f[2 * k] += __low2float(b2);
+              f[2 * k + 1] += __high2float(b2);
+            }
+          }
+          tc::st_shared_v4(addr, pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                           pack_bf16x2(f[6], f[7]));
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = i * 4 + rsub, t = m0w + rr, n = n0 + g * G + cc * 8;
+        const uint4 v = ld_shared_v4(stage_chunk(buf + rr * 128, rr, cc, 7));
+        if (t < a.T && n < p.N) tc::st_global_v4(out + (size_t)t * p.N + n, v.x, v.y, v.z, v.w);
+      }
+      __syncwarp();  // this buffer takes group g + 2
     }
   }
 };
@@ -287,19 +388,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
     // ------------------------------------------------------------ epilogue
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
+    const uint32_t stage = smem_u32(smem + STAGES * STAGE_BYTES + 1024) + q4 * Epi::kStageBytes;
     int it = 0;
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x, ++it) {
       const int buf = it & 1;
+      const int m0 = (tile / a.num_n) * BM, n0 = (tile % a.num_n) * BN;
+      Epi::template prefetch<BN>(a, m0, n0, q4, stage);
       const bool got = mbar_wait(&bars->acc_full[buf], (it >> 1) & 1, err);
       if (!__all_sync(0xffffffffu, got)) break;
       tc::fence_after_sync();
-      const int m0 = (tile / a.num_n) * BM, n0 = (tile % a.num_n) * BN;
       const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + buf * BN;
-      Epi::template tile<BN>(a, bars, tbase, m0, n0, row);
+      Epi::template tile<BN>(a, bars, tbase, m0, n0, row, stage);
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
     }
+    cp_async_wait<0>();  // no staging copy outlives the CTA
   }
 
   tc::fence_before_sync();
@@ -314,9 +418,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
 template <class Epi, class Cfg>
 cudaError_t launch_cfg(const typename Epi::Params& p, const void* x, const void* w, int T, int K, int N,
                        int n_heads_total, int num_sms, cudaStream_t st) {
+  constexpr int SMEM = Cfg::SMEM_BYTES + 4 * Epi::kStageBytes;
+  static_assert(SMEM <= 232448, "227 KB of shared memory per CTA");
   static std::atomic<bool> attr_set[64];
-  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(gemm_tc_kernel<Epi, Cfg>),
-                                     Cfg::SMEM_BYTES);
+  if (cudaError_t e = smem_attr_once(attr_set, reinterpret_cast<const void*>(gemm_tc_kernel<Epi, Cfg>), SMEM);
       e != cudaSuccess)
     return e;
   TcArgs<typename Epi::Params> a;
@@ -330,7 +435,7 @@ cudaError_t launch_cfg(const typename Epi::Params& p, const void* x, const void*
   if (!make_tmap_bf16_2d(&tx, x, K, T, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tw, w, K, N, (uint64_t)K * 2, BK, Cfg::BN)) return cudaErrorInvalidValue;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
-  gemm_tc_kernel<Epi, Cfg><<<grid, THREADS, Cfg::SMEM_BYTES, st>>>(tx, tw, a);
+  gemm_tc_kernel<Epi, Cfg><<<grid, THREADS, SMEM, st>>>(tx, tw, a);
   return cudaGetLastError();
 }
 
