@@ -297,8 +297,13 @@ size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int he
   const int split = gqa::decode_split_len(B, n_heads, n_kv_heads, cache_cap, kv_split);
   const size_t n_split = (size_t)(cache_cap + split - 1) / split;
   if (n_split > (size_t)kMaxSplits) return 0;
-  return gqa::decode_counter_bytes(B, n_kv_heads, gqa::decode_n_hgrp(n_heads, n_kv_heads)) +
-         (size_t)B * n_heads * n_split * (head_dim + gqa::kWsPad) * sizeof(float);
+  size_t partials = (size_t)B * n_heads * n_split * (head_dim + gqa::kWsPad) * sizeof(float);
+  // the keys-as-rows decode (bf16) takes its own partial slots
+  if (gqa::decode_hn_ok(B, n_heads, n_kv_heads, head_dim, cache_cap, kv_split == 0)) {
+    const size_t hn = gqa::decode_hn_partial_bytes(B, n_heads, n_kv_heads);
+    if (hn > partials) partials = hn;
+  }
+  return gqa::decode_counter_bytes(B, n_kv_heads, gqa::decode_n_hgrp(n_heads, n_kv_heads)) + partials;
 }
 
 int gqa_attn_decode(const void* q, const void* k_cache, const void* v_cache,

@@ -571,7 +571,7 @@ cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
 int launch_decode(const DecodeParams& p0, bool bf16, cudaStream_t st, cudaError_t* err) {
   if (bf16 && p0.auto_split && !p0.block_table) {
     // large batches with large head groups: tcgen05 tiles (mma.sync would be
-    // tensor-bound there)
+    // tensor-bound there), splits merged inside a cluster
     const int nc = decode_tc_splits(p0);
     if (nc > 0) {
       DecodeParams p = p0;
@@ -580,6 +580,15 @@ int launch_decode(const DecodeParams& p0, bool bf16, cudaStream_t st, cudaError_
       *err = launch_decode_tc(p, st);
       return 1;
     }
+  }
+  if (bf16 && decode_hn_ok(p0.B, p0.nh, p0.nkv, p0.hd, p0.cap, p0.auto_split != 0)) {
+    // the other large problems with head groups of 17..64 (paged caches and
+    // caches past the cluster kernel's 8 x 2048 keys): keys as the tcgen05
+    // rows, equal key ranges per SM.  On the contiguous B 64 MQA workload the
+    // cluster kernel above measured 52 us against this kernel's 54 us; with
+    // 64-key pages this kernel takes 56-59 us, the mma.sync kernel 62 us.
+    *err = launch_decode_hn(p0, st);
+    return 1;
   }
   if (bf16 && (p0.hd == 64 || p0.hd == 128)) {  // merges its splits itself
     DecodeParams p = p0;

@@ -156,6 +156,16 @@ cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st);   // head
 // problem is for the mma.sync kernel.
 cudaError_t launch_decode_tc(const DecodeParams& p, cudaStream_t st);
 int decode_tc_splits(const DecodeParams& p);
+// tcgen05 decode with the keys as the 128 MMA rows and the heads as N (bf16
+// head_dim 128, 16 < g <= 64, the library's split, at least 2^18 cached key
+// rows, at most 1024 (sequence, KV head) units): one CTA per SM over equal
+// ranges of the units' 128-key tiles.  Its partials take (kHnMaxGrid + units)
+// slots of NP x (hd + kWsPad) floats after the counters
+// (decode_hn_partial_bytes).
+constexpr int kHnMaxGrid = 160;
+bool decode_hn_ok(int B, int nh, int nkv, int hd, long long cap, bool auto_split);
+size_t decode_hn_partial_bytes(int B, int nh, int nkv);
+cudaError_t launch_decode_hn(const DecodeParams& p, cudaStream_t st);
 
 // Decode: the tensor-core kernel for bf16 head_dim 64/128 (the last split of
 // each (sequence, KV head, head group) merges the partials itself, using the

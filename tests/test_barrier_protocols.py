@@ -11,8 +11,8 @@ barriers exist for (TMEM columns and shared-memory stages are reused only
 after their readers finished) and that no schedule deadlocks.
 
 These are models of the protocols, kept next to the sources they restate
-(qkv_tc.cu, prefill_pair.cu, prefill_fa.cu, decode_tc.cu); a change to a
-kernel's waits belongs in both.  The decode's former final waits, which the
+(qkv_tc.cu, prefill_pair.cu, prefill_fa.cu, decode_tc.cu, decode_hn.cu); a
+change to a kernel's waits belongs in both.  The decode's former final waits, which the
 model flags, are kept as a planted mistake.
 """
 import random
@@ -428,6 +428,160 @@ def test_planted_decode_final_waits_are_flagged(final):
         roles, bars = decode_tc(3, final=final)
         try:
             run(roles, bars, seed)
+        except AssertionError:
+            flagged += 1
+    assert flagged > 0
+
+
+# ---------------------------------------------------------------- decode_hn.cu
+def decode_hn(pieces, KS=3, VS=3, rescale=(), zero_v=(), warps=4, p_wait=True):
+    """One CTA's range: `pieces` lists the tiles of each piece in order;
+    tiles are numbered n = 0, 1, ... across pieces.  `rescale` holds the
+    tiles whose softmax rescales O^T, `zero_v` the tiles whose V rows past
+    kv_len the softmax zeroes.  `p_wait` False drops the single P buffer's
+    wait (a planted mistake)."""
+    bars = {"p_full": Bar(warps), "p_empty": Bar(1), "drain": Bar(1)}
+    for i in range(2):
+        bars[f"q_full{i}"], bars[f"q_empty{i}"] = Bar(1), Bar(1)
+        bars[f"s_full{i}"], bars[f"s_free{i}"] = Bar(1), Bar(warps)
+        bars[f"o_final{i}"], bars[f"o_empty{i}"] = Bar(1), Bar(warps)
+        bars[f"ml_full{i}"], bars[f"ml_empty{i}"] = Bar(warps), Bar(warps)
+    for i in range(KS):
+        bars[f"k_full{i}"], bars[f"k_empty{i}"] = Bar(1), Bar(1)
+    for i in range(VS):
+        bars[f"v_full{i}"], bars[f"v_empty{i}"] = Bar(1), Bar(1)
+    tiles = []            # (n, piece, first, last)
+    for pi, cnt in enumerate(pieces):
+        for t in range(cnt):
+            tiles.append((len(tiles), pi, t == 0, t == cnt - 1))
+
+    def tma():
+        for pi in range(len(pieces)):
+            q = pi & 1
+            if pi >= 2:
+                yield ("wait", f"q_empty{q}", (pi >> 1) - 1)
+            yield ("issue", f"load_q{pi}", [f"q_full{q}"])
+            for n, tp, _, _ in tiles:
+                if tp != pi:
+                    continue
+                yield from ring_load("k", n, KS, None)
+                if n >= 1:                      # V runs one tile behind K
+                    yield from ring_load("v", n - 1, VS, None)
+        if tiles:
+            yield from ring_load("v", len(tiles) - 1, VS, None)
+
+    def mma():
+        def pv(m):
+            _, pm, first, last = tiles[m]
+            if first and pm >= 2:
+                yield ("wait", f"o_empty{pm & 1}", (pm >> 1) - 1)
+            yield ("wait", "p_full", m)
+            yield ("wait", f"v_full{m % VS}", m // VS)
+            yield ("event", f"PV{m}_start")
+            yield ("issue", f"PV{m}", [f"v_empty{m % VS}", "p_empty"] + ([f"o_final{pm & 1}"] if last else []))
+        for n, pi, first, last in tiles:
+            if first:
+                yield ("wait", f"q_full{pi & 1}", pi >> 1)
+            yield ("wait", f"k_full{n % KS}", n // KS)
+            if n >= 2:
+                yield ("wait", f"s_free{n & 1}", (n - 2) >> 1)
+            yield ("event", f"S{n}_start")
+            yield ("issue", f"S{n}", [f"k_empty{n % KS}", f"s_full{n & 1}"] + ([f"q_empty{pi & 1}"] if last else []))
+            if n >= 1:
+                yield from pv(n - 1)
+        if tiles:
+            yield from pv(len(tiles) - 1)
+        yield ("issue", "drain", ["drain"])
+        yield ("wait", "drain", 0)
+
+    def softmax(w):
+        for n, pi, first, last in tiles:
+            yield ("wait", f"s_full{n & 1}", n >> 1)
+            yield ("event", f"readS{n}_{w}")
+            yield ("arrive", f"s_free{n & 1}")
+            if n >= 1 and p_wait:
+                yield ("wait", "p_empty", n - 1)
+            if n in rescale and not first:
+                yield ("event", f"rescale{n}_{w}")
+            yield ("event", f"writeP{n}_{w}")
+            if n in zero_v:
+                yield ("wait", f"v_full{n % VS}", n // VS)
+                yield ("event", f"zeroV{n}_{w}")
+            yield ("arrive", "p_full")
+            if last:
+                if pi >= 2:
+                    yield ("wait", f"ml_empty{pi & 1}", (pi >> 1) - 1)
+                yield ("event", f"writeM{pi}_{w}")
+                yield ("arrive", f"ml_full{pi & 1}")
+
+    def epilogue(w):
+        for pi in range(len(pieces)):
+            yield ("wait", f"o_final{pi & 1}", pi >> 1)
+            yield ("wait", f"ml_full{pi & 1}", pi >> 1)
+            yield ("event", f"readO{pi}_{w}")
+            yield ("arrive", f"o_empty{pi & 1}")
+            yield ("arrive", f"ml_empty{pi & 1}")
+
+    roles = {"tma": tma(), "mma": mma()}
+    roles.update({f"sm{w}": softmax(w) for w in range(warps)})
+    roles.update({f"ep{w}": epilogue(w) for w in range(warps)})
+    return roles, bars, tiles
+
+
+def check_hn(tiles, pos, zero_v, KS, VS):
+    W = range(4)
+    piece_tiles = {}
+    for n, pi, _, _ in tiles:
+        piece_tiles.setdefault(pi, []).append(n)
+    for n, pi, first, last in tiles:
+        for w in W:
+            assert pos[("done", f"S{n}")] < pos[("event", f"readS{n}_{w}")]
+            assert pos[("event", f"writeP{n}_{w}")] < pos[("event", f"PV{n}_start")]
+            if n >= 1:      # one P buffer: P(n) is written after P.V(n-1) read P(n-1)
+                assert pos[("done", f"PV{n - 1}")] < pos[("event", f"writeP{n}_{w}")]
+            if n >= 2:      # S(n) reuses the TMEM columns S(n-2) was read from
+                assert pos[("event", f"readS{n - 2}_{w}")] < pos[("event", f"S{n}_start")]
+            if ("event", f"rescale{n}_{w}") in pos:
+                assert pos[("done", f"PV{n - 1}")] < pos[("event", f"rescale{n}_{w}")] < pos[("event", f"PV{n}_start")]
+            if n in zero_v:
+                assert pos[("done", f"load_v{n}")] < pos[("event", f"zeroV{n}_{w}")] < pos[("event", f"PV{n}_start")]
+        if n >= KS:         # a K stage is reloaded only after the S that read it completed
+            assert pos[("done", f"S{n - KS}")] < pos[("issue", f"load_k{n}")]
+        if n >= VS:
+            assert pos[("done", f"PV{n - VS}")] < pos[("issue", f"load_v{n}")]
+    for pi, ns in piece_tiles.items():
+        for w in W:         # O^T of a piece is read after its last P.V and before piece pi + 2 reuses it
+            assert pos[("done", f"PV{ns[-1]}")] < pos[("event", f"readO{pi}_{w}")]
+            assert pos[("event", f"writeM{pi}_{w}")] < pos[("event", f"readO{pi}_{w}")]
+            if pi + 2 in piece_tiles:
+                assert pos[("event", f"readO{pi}_{w}")] < pos[("event", f"PV{piece_tiles[pi + 2][0]}_start")]
+                assert pos[("event", f"readO{pi}_{w}")] < pos[("event", f"writeM{pi + 2}_{w}")]
+        if pi + 2 in piece_tiles:   # a Q buffer is reloaded after the piece's last S completed
+            assert pos[("done", f"S{ns[-1]}")] < pos[("issue", f"load_q{pi + 2}")]
+
+
+HN_CASES = [([1], (), (0,)), ([3], (0, 2), (2,)), ([2, 1], (0, 1), (1, 2)), ([1, 1, 1], (0, 1, 2), (0, 1, 2)),
+            ([4, 2, 3], (0, 3, 5, 8), (3, 5)), ([5, 1, 1, 2], (0, 2, 5, 6, 7), (4, 6, 8))]
+
+
+@pytest.mark.parametrize("pieces,rescale,zero_v", HN_CASES, ids=lambda c: str(c))
+@pytest.mark.parametrize("KS,VS", [(3, 3), (2, 3), (3, 2)])
+def test_decode_keys_as_rows_protocol(pieces, rescale, zero_v, KS, VS):
+    for seed in range(40):
+        roles, bars, tiles = decode_hn(pieces, KS, VS, rescale, zero_v)
+        pos = first(run(roles, bars, seed))
+        check_hn(tiles, pos, zero_v, KS, VS)
+
+
+def test_planted_decode_keys_as_rows_missing_p_wait_is_flagged():
+    """Without the wait for the previous P.V, the softmax can overwrite the
+    single P buffer while the tensor cores still read it."""
+    flagged = 0
+    for seed in range(60):
+        roles, bars, tiles = decode_hn([3, 2], 3, 3, (), (), p_wait=False)
+        try:
+            pos = first(run(roles, bars, seed))
+            check_hn(tiles, pos, (), 3, 3)
         except AssertionError:
             flagged += 1
     assert flagged > 0

@@ -388,6 +388,56 @@ def test_decode_tcgen05_large_batch(hd, nh, nkv, B):
     gate(got[1:], want[1:], dtype, "tcgen05 decode")
 
 
+def _hn_lens(B, cap, seed, edge):
+    rng = np.random.default_rng(seed)
+    return np.array(edge + list(rng.integers(1, cap + 1, size=B - len(edge))), dtype=np.int32)[:B]
+
+
+@pytest.mark.parametrize("g,nkv", [(32, 1), (24, 2), (48, 1), (64, 1)], ids=["g32", "g24-nkv2", "g48", "g64"])
+def test_decode_keys_as_rows(g, nkv):
+    """Large batches with 16 < g <= 64 at head_dim 128 whose cache is longer
+    than the cluster kernel takes (here 20000 keys) use the decode with the
+    keys as the 128 MMA rows and the heads as N (padded to a multiple of 16):
+    equal tile ranges per SM, pieces merged through the workspace by the last
+    piece of each (sequence, KV head).  Ragged lengths with 0, 1 and 128-key
+    tile edges; two calls on one workspace leave its counters at zero."""
+    dtype, hd, cap, B = "bf16", 128, 20000, 16
+    nh = g * nkv
+    lens = _hn_lens(B, cap, 31 + g, [0, 1, 127, 128, 129, 1000, 8191, 16384, 19999, 20000])
+    q = W.normal_tensor((B, nh, hd), 16 + g, 0, dtype)
+    kc = nan_padded(B, nkv, cap, hd, lens, 16 + g, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, lens, 16 + g, 2, dtype)
+    want = ref.decode_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens)
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap, 0) // 4 + 1,
+                     dtype=torch.float32, device="cuda")
+    n_counters = B * nkv * ((g + 15) // 16)
+    gqa.gqa_device_error()
+    for call in range(2):
+        out = torch.empty((B, nh, hd), dtype=torch.bfloat16, device="cuda")
+        gqa.gqa_attn_decode(dev(q), dev(kc), dev(vc), dev_i32(lens), out, ws)
+        got = host(out)
+        assert np.all(got[0] == 0)
+        gate(got[1:], want[1:], dtype, f"keys-as-rows decode, call {call}")
+        assert int(ws[:n_counters].view(torch.int32).abs().sum()) == 0
+    assert gqa.gqa_device_error() == 0
+
+
+@pytest.mark.parametrize("long_len", (20000, 8192), ids=["172-tiles", "79-tiles"])
+def test_decode_keys_as_rows_many_pieces(long_len):
+    """One long sequence among 15 one-key sequences.  20000 keys: 172 tiles
+    over the SMs, so the long sequence is cut into pieces of one or two tiles
+    on over 100 CTAs, more than the shared-memory merge takes at once (its
+    merge runs in rounds over the workspace).  8192 keys: 79 tiles, fewer than
+    the SMs, so the tiles are cut over 79 CTAs of one tile and the rest idle."""
+    dtype, hd, nh, nkv, cap, B = "bf16", 128, 32, 1, 20000, 16
+    lens = np.array([1] * 6 + [long_len] + [1] * 9, dtype=np.int32)
+    q = W.normal_tensor((B, nh, hd), 23, 0, dtype)
+    kc = nan_padded(B, nkv, cap, hd, lens, 23, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, lens, 23, 2, dtype)
+    want = ref.decode_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), lens)
+    gate(host(run_decode(q, kc, vc, lens, nh, dtype)), want, dtype, "keys-as-rows decode, many pieces")
+
+
 def test_decode_long_cache_uses_workspace_splits():
     """A cache longer than 8 x 2048 keys takes the workspace splits even when
     the split is left to the library."""
@@ -456,6 +506,31 @@ def test_paged_decode_parity(hd, g, nkv, ps):
         gate(got[keep], want[keep], "bf16", f"paged decode split={split}")
         flat = run_decode(q, kc, vc, lens, nh, "bf16", kv_split=split)
         np.testing.assert_array_equal(bits(got_t), bits(flat))
+    assert gqa.gqa_device_error() == 0
+
+
+@pytest.mark.parametrize("ps", (64, 192))
+def test_paged_decode_keys_as_rows(ps):
+    """The keys-as-rows decode (B 32, 32 heads on one KV head, up to 8192
+    keys) over shuffled pages: every 64-key half of a 128-key tile is mapped
+    to its page (a 192-key page holds one and a half tiles); against the
+    oracle's paged decode, and bit for bit against the same keys in a
+    contiguous cache of 20000 slots (long enough that the contiguous call
+    takes the same kernel: only the address of each tile differs)."""
+    hd, g, nkv, B = 128, 32, 1, 32
+    nh = g * nkv
+    lens = _hn_lens(B, 8192, 77 + ps, [8192, 0, 1, 64, 127, 128, 129, 191, 192, 193, 5000])
+    q, kc, vc, kp, vp, table, cap = paged_inputs(B, nh, nkv, hd, ps, lens, 90 + ps)
+    want = ref.paged_decode_attention(q.f64, kp.f64, vp.f64, table, lens, ps)
+    gqa.gqa_device_error()
+    got_t = run_decode_paged(q, kp, vp, table, lens, nh)
+    got = host(got_t)
+    assert np.all(got[1] == 0)
+    keep = lens > 0
+    gate(got[keep], want[keep], "bf16", f"paged keys-as-rows decode ps={ps}")
+    wide = lambda c: W.Tensor(np.pad(c.store, ((0, 0), (0, 0), (0, 20000 - c.store.shape[2]), (0, 0))), "bf16")
+    flat = run_decode(q, wide(kc), wide(vc), lens, nh, "bf16")
+    np.testing.assert_array_equal(bits(got_t), bits(flat))
     assert gqa.gqa_device_error() == 0
 
 
