@@ -395,7 +395,7 @@ def measure_workloads(dev, peaks, iters=10, only=None, checks=True):
     transform on the Llama-2-7B projection (32 -> 8 KV heads): GB/s.  Each
     kernel is timed alone with CUDA events, L2 flushed before every timed call
     (a 512 MB write), median of `iters`.  ``only``: a set of section names
-    (decode, prefill8k, generate, small, varlen, meanpool) to measure; None =
+    (decode, decode_mqa, prefill8k, generate, small, varlen, meanpool) to measure; None =
     all.  ``checks``: also compare sampled outputs of each config with the
     float64 oracle and time the oracle on the host cores (scaled linearly
     from the sample to the whole config)."""
@@ -431,7 +431,7 @@ def measure_workloads(dev, peaks, iters=10, only=None, checks=True):
     want = (lambda name: only is None or name in only)
 
     # ---- batched decode
-    if want("decode"):
+    if want("decode") or want("decode_mqa"):
         wl = W.LLAMA2_DECODE
         e = wl.extra
         B, nh, hd, cap = e["batch"], wl.shape.n_heads, wl.shape.head_dim, e["cap"]
@@ -439,7 +439,8 @@ def measure_workloads(dev, peaks, iters=10, only=None, checks=True):
         lens = torch.from_numpy(lens_np).to(dev)
         q = torch.randn(B, nh, hd, generator=gen, device=dev).to(bf)
         dec = {}
-        for nkv in e["n_kv_heads_cases"]:
+        # "decode_mqa" alone: only the one-KV-head case (a small problem for a profiler)
+        for nkv in (e["n_kv_heads_cases"] if want("decode") else (1,)):
             kc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
             vc = torch.randn(B, nkv, cap, hd, generator=gen, device=dev, dtype=torch.float32).to(bf)
             o = torch.empty(B, nh, hd, dtype=bf, device=dev)
@@ -1014,7 +1015,7 @@ def main():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the per-kernel measurements of the decode, 8K-prefill and generation workloads")
     ap.add_argument("--workloads", default=None,
-                    help="comma-separated workload sections to measure (decode, prefill8k, generate, small, "
+                    help="comma-separated workload sections to measure (decode, decode_mqa, prefill8k, generate, small, "
                          "varlen, meanpool, tiny); default all")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()

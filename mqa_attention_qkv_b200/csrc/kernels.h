@@ -174,9 +174,13 @@ cudaError_t launch_decode_hn(const DecodeParams& p, cudaStream_t st);
 int launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st, cudaError_t* err);
 
 // Raise a kernel's dynamic shared-memory limit on the current device, once per
-// device (`done` is the caller's per-kernel flag array).  The attribute is
-// idempotent, so two threads racing on a first call both set it; devices past
-// the array are set on every call.
+// device (`done` is the caller's per-kernel flag array), and ask for the
+// largest shared-memory carveout: every pipelined kernel of the library then
+// runs with the same L1/shared split, so consecutive launches do not make the
+// SMs reconfigure it (on B200 a step whose kernels alternated between a small
+// and a 215 KB shared-memory configuration lost ~25 us at the switch).  The
+// attributes are idempotent, so two threads racing on a first call both set
+// them; devices past the array are set on every call.
 inline cudaError_t smem_attr_once(std::atomic<bool> (&done)[64], const void* func, int bytes) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -185,7 +189,9 @@ inline cudaError_t smem_attr_once(std::atomic<bool> (&done)[64], const void* fun
   }
   const bool cached = dev >= 0 && dev < 64;
   if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess && cached) done[dev].store(true, std::memory_order_release);
   return e;
 }
