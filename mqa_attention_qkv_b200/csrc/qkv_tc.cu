@@ -55,7 +55,26 @@ template <class P>
 struct TcArgs {
   P p;
   int T, n_heads_total, num_n, num_tiles, num_kb;
+  // Work items: items below n_full are whole BN-wide tiles; the tiles of a
+  // last, partial wave are each cut into two BN/2-wide halves (items n_full
+  // and up), so that the last wave keeps twice as many SMs busy for half as
+  // long.  Without a partial wave, n_full = num_items = num_tiles.
+  int n_full, num_items;
 };
+
+// Tile of work item i: rows m0.., columns n0.. (width BN or BN/2).
+template <int BN, class A>
+__device__ __forceinline__ void item_tile(const A& a, int i, int& m0, int& n0, int& width) {
+  int t = i, half = 0;
+  width = BN;
+  if (i >= a.n_full) {
+    t = a.n_full + ((i - a.n_full) >> 1);
+    half = (i - a.n_full) & 1;
+    width = BN / 2;
+  }
+  m0 = (t / a.num_n) * BM;
+  n0 = (t % a.num_n) * BN + half * (BN / 2);
+}
 
 struct Bars {
   uint64_t full[MAX_STAGES], empty[MAX_STAGES], acc_full[2], acc_empty[2], drain;
@@ -292,10 +311,11 @@ struct ResidualEpilogue {
 template <class Epi, class Cfg>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmw,
-               TcArgs<typename Epi::Params> a) {
+               const __grid_constant__ CUtensorMap tmw_half, TcArgs<typename Epi::Params> a) {
   constexpr int BN = Cfg::BN, STAGES = Cfg::STAGES, A_BYTES = Cfg::A_BYTES, STAGE_BYTES = Cfg::STAGE_BYTES;
   constexpr int TMEM_COLS = Cfg::TMEM_COLS;
   constexpr uint32_t IDESC = Cfg::IDESC;
+  constexpr uint32_t IDESC_HALF = tc::idesc_bf16(BM, BN / 2, false, false);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
@@ -319,6 +339,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
   if (warp == 0 && lane == 0) {
     tc::prefetch_tmap(&tmx);
     tc::prefetch_tmap(&tmw);
+    if (a.num_items > a.n_full) tc::prefetch_tmap(&tmw_half);
   }
   if (warp == 1) tc::tmem_alloc(&bars->tmem_base, TMEM_COLS);
   tc::fence_before_sync();
@@ -332,14 +353,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x) {
-        const int m0 = (tile / a.num_n) * BM, n0 = (tile % a.num_n) * BN;
+      for (int item = blockIdx.x; ok && item < a.num_items; item += gridDim.x) {
+        int m0, n0, width;
+        item_tile<BN>(a, item, m0, n0, width);
+        const CUtensorMap* wmap = width == BN ? &tmw : &tmw_half;
         for (int kb = 0; kb < a.num_kb; ++kb) {
           if (!mbar_wait(&bars->empty[stage], phase ^ 1, err)) { ok = false; break; }
           uint8_t* sa = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&bars->full[stage], STAGE_BYTES);
+          mbar_arrive_expect_tx(&bars->full[stage], A_BYTES + width * BK * 2);
           tc::tma_load_2d(sa, &tmx, kb * BK, m0, &bars->full[stage]);
-          tc::tma_load_2d(sa + A_BYTES, &tmw, kb * BK, n0, &bars->full[stage]);
+          tc::tma_load_2d(sa + A_BYTES, wmap, kb * BK, n0, &bars->full[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -358,8 +381,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int tile = blockIdx.x; ok && tile < a.num_tiles; tile += gridDim.x, ++it) {
+      for (int item = blockIdx.x; ok && item < a.num_items; item += gridDim.x, ++it) {
         const int buf = it & 1;
+        const uint32_t idesc = item < a.n_full ? IDESC : IDESC_HALF;
         if (!mbar_wait(&bars->acc_empty[buf], ((it >> 1) & 1) ^ 1, err)) { ok = false; break; }
         tc::fence_after_sync();
         const uint32_t d = tmem + buf * BN;
@@ -371,7 +395,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             tc::mma_bf16_ss(d, tc::sdesc_sw128(sa + k * 32, 16, 1024), tc::sdesc_sw128(sb + k * 32, 16, 1024),
-                            IDESC, (kb | k) != 0);
+                            idesc, (kb | k) != 0);
           }
           tc::mma_commit(&bars->empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -390,15 +414,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
     const int row = q4 * 32 + lane;
     const uint32_t stage = smem_u32(smem + STAGES * STAGE_BYTES + 1024) + q4 * Epi::kStageBytes;
     int it = 0;
-    for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x, ++it) {
+    for (int item = blockIdx.x; item < a.num_items; item += gridDim.x, ++it) {
       const int buf = it & 1;
-      const int m0 = (tile / a.num_n) * BM, n0 = (tile % a.num_n) * BN;
+      int m0, n0, width;
+      item_tile<BN>(a, item, m0, n0, width);
       Epi::template prefetch<BN>(a, m0, n0, q4, stage);
       const bool got = mbar_wait(&bars->acc_full[buf], (it >> 1) & 1, err);
       if (!__all_sync(0xffffffffu, got)) break;
       tc::fence_after_sync();
       const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + buf * BN;
-      Epi::template tile<BN>(a, bars, tbase, m0, n0, row, stage);
+      if constexpr (BN == 256) {
+        if (width == BN) Epi::template tile<BN>(a, bars, tbase, m0, n0, row, stage);
+        else Epi::template tile<BN / 2>(a, bars, tbase, m0, n0, row, stage);
+      } else {
+        Epi::template tile<BN>(a, bars, tbase, m0, n0, row, stage);
+      }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[buf]);
@@ -431,11 +461,21 @@ cudaError_t launch_cfg(const typename Epi::Params& p, const void* x, const void*
   a.num_n = (N + Cfg::BN - 1) / Cfg::BN;
   a.num_tiles = ((T + BM - 1) / BM) * a.num_n;
   a.num_kb = (K + BK - 1) / BK;
-  CUtensorMap tx, tw;
+  // a partial last wave of wide tiles goes as twice as many half-width tiles
+  // when they still fit in one wave
+  const int rem = num_sms > 0 ? a.num_tiles % num_sms : 0;
+  if (Cfg::BN == 256 && a.num_tiles > num_sms && rem > 0 && 2 * rem <= num_sms) {
+    a.n_full = a.num_tiles - rem;
+    a.num_items = a.num_tiles + rem;
+  } else {
+    a.n_full = a.num_items = a.num_tiles;
+  }
+  CUtensorMap tx, tw, tw_half;
   if (!make_tmap_bf16_2d(&tx, x, K, T, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tw, w, K, N, (uint64_t)K * 2, BK, Cfg::BN)) return cudaErrorInvalidValue;
-  const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
-  gemm_tc_kernel<Epi, Cfg><<<grid, THREADS, SMEM, st>>>(tx, tw, a);
+  if (!make_tmap_bf16_2d(&tw_half, w, K, N, (uint64_t)K * 2, BK, Cfg::BN / 2)) return cudaErrorInvalidValue;
+  const int grid = a.num_items < num_sms ? a.num_items : num_sms;
+  gemm_tc_kernel<Epi, Cfg><<<grid, THREADS, SMEM, st>>>(tx, tw, tw_half, a);
   return cudaGetLastError();
 }
 

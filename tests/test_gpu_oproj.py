@@ -31,6 +31,7 @@ CASES = [
     (40, 8, 64, 2056), (20, 6, 32, 1040),
     (8, 48, 128, 6144),                               # MQA generation step shape
     (65, 32, 64, 2048), (200, 5, 32, 264), (300, 8, 128, 1032), (1000, 16, 64, 1024),
+    (4000, 16, 64, 1536),                             # 192 tiles: the last wave's 44 as 88 half-width tiles
 ]
 
 
