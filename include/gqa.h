@@ -178,7 +178,13 @@ int gqa_attn_prefill_varlen(const void* q, const void* k, const void* v, const i
  * needs for these sizes: a block of split counters (one 32-bit word per
  * sequence, KV head and group of up to 16 query heads, rounded up to 256
  * bytes) followed by float32 partial results (a running max, a sum and an
- * unnormalised output row per sequence, query head and key split).
+ * unnormalised output row per sequence, query head and key split).  When the
+ * split is left to the library and the problem may take the decode that cuts
+ * the sequences' keys into equal ranges per SM (head_dim 128, 17..64 query
+ * heads per KV head, at least 2^18 cached key rows, at most 512 sequence x
+ * KV head pairs), the partials take at most (160 + B * n_kv_heads) slots of
+ * n_heads / n_kv_heads (rounded up to 16) rows of head_dim + 4 floats, and
+ * the size covers the larger of the two layouts.
  * kv_split: keys per split, 0 = the library's choice, else a multiple of 64.
  * Returns 0 for invalid arguments.
  */
@@ -196,8 +202,12 @@ size_t gqa_attn_decode_workspace_size(int B, int n_heads, int n_kv_heads, int he
  * (max m, sum l, unnormalised o) per head and the partials are merged with a
  * log-sum-exp combine, which is exact.  On the tensor-core path (bf16,
  * head_dim 64/128) the last chunk of a (sequence, KV head) to finish does the
- * merge, found through a counter in the workspace; a sequence with a single
- * chunk is written directly.
+ * merge, found through a counter in the workspace (or, for the library's own
+ * split of small caches, inside a thread-block cluster); a sequence with a
+ * single chunk is written directly.  Large problems with 17..64 query heads
+ * per KV head at head_dim 128 whose cache is paged or longer than 8 x 2048
+ * keys cut the concatenated 128-key tiles of all sequences into one equal
+ * range per SM instead; its pieces merge the same way.
  *
  *   q          [B, n_heads, head_dim] dtype (the new token, already rotated)
  *   k_cache,
