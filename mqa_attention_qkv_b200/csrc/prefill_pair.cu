@@ -352,6 +352,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     const size_t tok = VARLEN ? (size_t)sq.q0 + s0 + row : (size_t)b * p.S + (s0 + row);
     __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + (tok * p.nh + h) * HD;
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    // this warp's 32 output rows (128 bytes each) staged in the idle K ring,
+    // 16-byte chunk ch of row r at chunk ch ^ (r & 7), then copied out with 8
+    // lanes per row so that each store writes whole lines of 4 rows
+    const uint32_t stage = smem_u32(sK) + (uint32_t)((warp & 3) * 32 * 128);
 #pragma unroll 1
     for (int c = 0; c < HD / 16; ++c) {
       uint32_t r[16];
@@ -363,13 +367,25 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
 #pragma unroll
         for (int i = 0; i < 16; ++i) r[i] = 0u;
       }
-      if (my_valid) {
-        uint32_t o[8];
+      uint32_t o[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          o[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-        tc::st_global_v4(dst + c * 16, o[0], o[1], o[2], o[3]);
-        tc::st_global_v4(dst + c * 16 + 8, o[4], o[5], o[6], o[7]);
+      for (int i = 0; i < 8; ++i)
+        o[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+      tc::st_shared_v4(stage + lane * 128 + (((2 * c) ^ (lane & 7)) << 4), o[0], o[1], o[2], o[3]);
+      tc::st_shared_v4(stage + lane * 128 + (((2 * c + 1) ^ (lane & 7)) << 4), o[4], o[5], o[6], o[7]);
+    }
+    __syncwarp();
+    {
+      const unsigned long long my_dst = my_valid ? reinterpret_cast<unsigned long long>(dst) : 0ull;
+      const int cc = lane & 7, rsub = lane >> 3;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = i * 4 + rsub;
+        const unsigned long long d = __shfl_sync(0xffffffffu, my_dst, rr);
+        uint32_t v0, v1, v2, v3;
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                     : "r"(stage + rr * 128 + ((cc ^ (rr & 7)) << 4)) : "memory");
+        if (d) tc::st_global_v4(reinterpret_cast<uint8_t*>(d) + cc * 16, v0, v1, v2, v3);
       }
     }
   }
