@@ -440,6 +440,29 @@ def test_decode_keys_as_rows_many_pieces(long_len):
     gate(host(run_decode(q, kc, vc, lens, nh, dtype)), want, dtype, "keys-as-rows decode, many pieces")
 
 
+def test_decode_keys_as_rows_degenerate_lengths():
+    """The keys-as-rows decode with every length 0 (no tiles anywhere: every
+    output row is written as zeros by its CTA) and with lengths past the
+    cache (clamped to it and flagged)."""
+    dtype, hd, nh, nkv, cap, B = "bf16", 128, 32, 1, 20000, 16
+    q = W.normal_tensor((B, nh, hd), 29, 0, dtype)
+    zero = np.zeros(B, dtype=np.int32)
+    kc = nan_padded(B, nkv, cap, hd, zero, 29, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, zero, 29, 2, dtype)
+    gqa.gqa_device_error()
+    out = run_decode(q, kc, vc, zero, nh, dtype)
+    assert np.all(host(out) == 0)
+    assert gqa.gqa_device_error() == 0
+    lens = np.array([cap + 5] + [700] * (B - 1), dtype=np.int32)
+    full = np.minimum(lens, cap).astype(np.int32)
+    kc = nan_padded(B, nkv, cap, hd, full, 30, 1, dtype)
+    vc = nan_padded(B, nkv, cap, hd, full, 30, 2, dtype)
+    got = host(run_decode(q, kc, vc, lens, nh, dtype))
+    assert gqa.gqa_device_error() & 2
+    want = ref.decode_attention(q.f64, np.nan_to_num(kc.f64), np.nan_to_num(vc.f64), full)
+    gate(got, want, dtype, "keys-as-rows decode, clamped lengths")
+
+
 def test_decode_long_cache_uses_workspace_splits():
     """A cache longer than 8 x 2048 keys takes the workspace splits even when
     the split is left to the library."""
