@@ -167,10 +167,12 @@ bool decode_hn_ok(int B, int nh, int nkv, int hd, long long cap, bool auto_split
 size_t decode_hn_partial_bytes(int B, int nh, int nkv);
 cudaError_t launch_decode_hn(const DecodeParams& p, cudaStream_t st);
 
-// Decode: the tensor-core kernel for bf16 head_dim 64/128 (the last split of
-// each (sequence, KV head, head group) merges the partials itself, using the
-// counters), else SIMT partials + the log-sum-exp combine kernel.  Partial m
-// is in log2 units.  Returns the number of kernels launched; *err the status.
+// Decode: for bf16, the tcgen05 cluster decode (contiguous caches it takes,
+// g > 16), else the keys-as-rows tcgen05 decode (decode_hn_ok), else the
+// mma.sync decode for head_dim 64/128 (the last split of each (sequence, KV
+// head, head group) merges the partials itself, using the counters); other
+// cases: SIMT partials + the log-sum-exp combine kernel.  Partial m is in log2
+// units.  Returns the number of kernels launched; *err the status.
 int launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st, cudaError_t* err);
 
 // Raise a kernel's dynamic shared-memory limit on the current device, once per
