@@ -3,10 +3,12 @@ memory where they run it (a serving loop whose device memory another
 allocator has fully reserved, a plugin that gets only the op's tensors, a
 path on which a possibly synchronising allocation is not allowed).
 
-Its split-KV scratch is a fixed static array inside the library.  Every case
-here passes an explicit kv_split, so the decode merges its splits through
-that array (split counters plus partials) rather than inside a thread-block
-cluster.  Two calls in a row with different inputs must each give what the
+Its split-KV scratch is a fixed static array inside the library.  The
+parametrised cases pass an explicit kv_split, so the decode merges its
+splits through that array (split counters plus partials) rather than inside
+a thread-block cluster; one more case leaves the split to the library on a
+problem that takes the keys-as-rows decode, whose pieces merge through the
+same array.  Two calls in a row with different inputs must each give what the
 workspace-taking gqa_attn_decode gives and what the float64 oracle gives,
 within the bf16 gate of the parity tests: the second call starts from the
 counters and partials the first one left in the shared array.  A fresh
@@ -66,6 +68,30 @@ def test_noalloc_decode_matches_workspace_decode_on_two_calls(case):
         torch.cuda.synchronize()
         gate(host(got), host(base), dt, f"no-alloc vs workspace decode, call {call}")
         gate(host(got), want, dt, f"no-alloc decode vs oracle, call {call}")
+
+
+def test_noalloc_keys_as_rows_decode_on_two_calls():
+    """The library's own split on a problem that takes the keys-as-rows
+    decode (B 16, 32 heads on one KV head, hd 128, a 20000-key cache): its
+    split counters and per-piece partials live in the static array; two calls
+    in a row with different lengths each match gqa_attn_decode and the
+    oracle."""
+    B, nh, nkv, hd, cap = 16, 32, 1, 128, 20000
+    rng = np.random.default_rng(41)
+    ws = torch.zeros(gqa.gqa_attn_decode_workspace_size(B, nh, nkv, hd, cap, 0), dtype=torch.uint8, device="cuda")
+    for call in range(2):
+        lens = np.array([cap, 1, 0, 8191] + list(rng.integers(1, cap + 1, size=B - 4)), dtype=np.int32)
+        (q, kc, vc, lnd), want = _problem(50 + call, B, nh, nkv, hd, cap, lens, "bf16")
+        base = torch.empty((B, nh, hd), dtype=torch.bfloat16, device="cuda")
+        got = torch.full((B, nh, hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+        gqa.gqa_attn_decode(q, kc, vc, lnd, base, ws)
+        gqa.gqa_attn_decode_noalloc(q, kc, vc, lnd, got)
+        torch.cuda.synchronize()
+        g = host(got)
+        assert np.all(g[2] == 0)
+        keep = lens > 0
+        gate(g[keep], host(base)[keep], "bf16", f"no-alloc vs workspace keys-as-rows decode, call {call}")
+        gate(g[keep], want[keep], "bf16", f"no-alloc keys-as-rows decode vs oracle, call {call}")
 
 
 _FRESH = r"""
