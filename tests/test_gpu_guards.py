@@ -77,8 +77,9 @@ def test_packed_prefill_writes_only_its_output():
 
 
 @pytest.mark.parametrize("B,nh,nkv,hd,cap,split", [(8, 48, 1, 128, 1040, 0), (8, 48, 1, 128, 1040, 64),
-                                                    (32, 48, 1, 64, 8192, 0), (5, 8, 8, 32, 300, 0)],
-                         ids=["cluster", "workspace", "tcgen05", "simt-hd32"])
+                                                    (32, 48, 1, 64, 8192, 0), (5, 8, 8, 32, 300, 0),
+                                                    (16, 48, 1, 128, 20000, 0), (16, 128, 2, 128, 20000, 0)],
+                         ids=["cluster", "workspace", "tcgen05", "simt-hd32", "keys-as-rows-g48", "keys-as-rows-g64"])
 def test_decode_writes_only_its_output(B, nh, nkv, hd, cap, split):
     lens = np.clip(W.ragged_lengths(B, 1, cap, 4), 1, cap).astype(np.int32)
     q = dev(W.normal_tensor((B, nh, hd), 4, 0, "bf16"))
