@@ -32,6 +32,7 @@ CASES = [
     (8, 48, 128, 6144),                               # MQA generation step shape
     (65, 32, 64, 2048), (200, 5, 32, 264), (300, 8, 128, 1032), (1000, 16, 64, 1024),
     (4000, 16, 64, 1536),                             # 192 tiles: the last wave's 44 as 88 half-width tiles
+    (6000, 8, 64, 904),                               # split last wave with a ragged N: a half tile of 8 columns
 ]
 
 

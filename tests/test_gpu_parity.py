@@ -54,6 +54,7 @@ QKV_CASES = [
     ("bf16", 2, 1024, 512, 16, 4, 64, 1024, True),  # 96 tiles: several per persistent CTA
     ("bf16", 2, 2000, 512, 16, 4, 64, 2048, True),  # 192 tiles, T tail: the last wave's 44 tiles as 88 halves
     ("bf16", 1, 4000, 256, 8, 2, 128, 4096, False),  # the same split at hd 128 (a half tile is one head)
+    ("bf16", 3, 2000, 256, 10, 2, 64, 2048, True),  # N = 896: the last column tile's second half lies past N
     ("bf16", 2, 70, 100, 4, 2, 64, 80, True),       # hidden % 8 != 0: the SIMT path
     # few tokens, hidden % 64 == 0 and the hidden states fit in shared memory:
     # the TMA-ring kernel, every token-count variant
