@@ -60,6 +60,12 @@ struct TcArgs {
   // and up), so that the last wave keeps twice as many SMs busy for half as
   // long.  Without a partial wave, n_full = num_items = num_tiles.
   int n_full, num_items;
+  // K split (ksplit > 1, few-token problems whose tiles would leave most SMs
+  // idle): the ksplit CTAs of a cluster each take one tile's k-blocks
+  // [rank num_kb / ksplit, (rank + 1) num_kb / ksplit); the ranks above 0
+  // leave their partial sums in their shared memory and the leader adds them
+  // into its accumulator before the epilogue.  One tile per CTA.
+  int ksplit;
 };
 
 // Tile of work item i: rows m0.., columns n0.. (width BN or BN/2).
@@ -109,6 +115,58 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int s
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// K-split partial sums in shared memory: row r of the tile (BN fp32, i.e.
+// BN / 4 chunks of 16 bytes) at r * BN * 4, chunk c at (c & ~7) | ((c ^ r) & 7),
+// so that the 32 rows of a warp spread over the banks.
+__device__ __forceinline__ uint32_t part_chunk(uint32_t row_base, int r, int c) {
+  return row_base + (uint32_t)(((c & ~7) | ((c ^ r) & 7)) * 16);
+}
+// a rank above 0: its accumulator row (TMEM lane of this thread) -> shared memory
+template <int BN>
+__device__ __forceinline__ void store_partial(uint32_t tbase, int row, uint32_t part) {
+  const uint32_t rb = part + (uint32_t)(row * BN * 4);
+#pragma unroll 1
+  for (int c = 0; c < BN / 16; ++c) {
+    uint32_t v[16];
+    __syncwarp();
+    tc::tmem_ld16(tbase + c * 16, v);
+    tc::tmem_ld_wait();
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+      tc::st_shared_v4(part_chunk(rb, row, 4 * c + h), v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]);
+  }
+}
+// the leader: add ranks 1 .. ks-1's rows (read from their shared memory
+// across the cluster, a whole row of one rank in flight at a time) into its
+// accumulator row
+template <int BN>
+__device__ __forceinline__ void add_partials(uint32_t tbase, int row, uint32_t part, int ks) {
+  constexpr int NCH = BN / 4;   // 16-byte chunks of a row
+  const uint32_t rb = part + (uint32_t)(row * BN * 4);
+#pragma unroll 1
+  for (int q = 1; q < ks; ++q) {
+    float4 f[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) f[c] = tc::ld_dsmem_f32x4(tc::mapa_shared(part_chunk(rb, row, c), q));
+#pragma unroll
+    for (int c = 0; c < BN / 16; ++c) {
+      uint32_t v[16];
+      __syncwarp();
+      tc::tmem_ld16(tbase + c * 16, v);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        v[4 * h] = __float_as_uint(__uint_as_float(v[4 * h]) + f[4 * c + h].x);
+        v[4 * h + 1] = __float_as_uint(__uint_as_float(v[4 * h + 1]) + f[4 * c + h].y);
+        v[4 * h + 2] = __float_as_uint(__uint_as_float(v[4 * h + 2]) + f[4 * c + h].z);
+        v[4 * h + 3] = __float_as_uint(__uint_as_float(v[4 * h + 3]) + f[4 * c + h].w);
+      }
+      tc::tmem_st16(tbase + c * 16, v);
+    }
+    tc::tmem_st_wait();
+  }
+}
 
 // Epilogue of the QKV projection: RoPE on q/k, head-major scatter.  One
 // thread owns token row `row` of the 128 x BN tile at (m0, n0); `tbase` is
@@ -335,7 +393,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
     bars->abort = 0;
     fence_mbar_init();
   }
-  Epi::init(a.p, bars);
   if (warp == 0 && lane == 0) {
     tc::prefetch_tmap(&tmx);
     tc::prefetch_tmap(&tmw);
@@ -346,6 +403,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
+  // K split: rank within the cluster, its k-blocks, and one tile per CTA
+  const int ks = a.ksplit, rank = ks > 1 ? (int)(blockIdx.x % ks) : 0;
+  const int item0 = ks > 1 ? (int)(blockIdx.x / ks) : (int)blockIdx.x;
+  const int item_step = ks > 1 ? a.num_items : (int)gridDim.x;
+  const int kb0 = rank * a.num_kb / ks, kb1 = (rank + 1) * a.num_kb / ks;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -353,11 +415,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int item = blockIdx.x; ok && item < a.num_items; item += gridDim.x) {
+      for (int item = item0; ok && item < a.num_items; item += item_step) {
         int m0, n0, width;
         item_tile<BN>(a, item, m0, n0, width);
         const CUtensorMap* wmap = width == BN ? &tmw : &tmw_half;
-        for (int kb = 0; kb < a.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&bars->empty[stage], phase ^ 1, err)) { ok = false; break; }
           uint8_t* sa = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&bars->full[stage], A_BYTES + width * BK * 2);
@@ -381,13 +443,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
       uint32_t phase = 0;
       bool ok = true;
       int it = 0;
-      for (int item = blockIdx.x; ok && item < a.num_items; item += gridDim.x, ++it) {
+      for (int item = item0; ok && item < a.num_items; item += item_step, ++it) {
         const int buf = it & 1;
         const uint32_t idesc = item < a.n_full ? IDESC : IDESC_HALF;
         if (!mbar_wait(&bars->acc_empty[buf], ((it >> 1) & 1) ^ 1, err)) { ok = false; break; }
         tc::fence_after_sync();
         const uint32_t d = tmem + buf * BN;
-        for (int kb = 0; kb < a.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&bars->full[stage], phase, err)) { ok = false; break; }
           tc::fence_after_sync();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
@@ -395,7 +457,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             tc::mma_bf16_ss(d, tc::sdesc_sw128(sa + k * 32, 16, 1024), tc::sdesc_sw128(sb + k * 32, 16, 1024),
-                            idesc, (kb | k) != 0);
+                            idesc, kb > kb0 || k != 0);
           }
           tc::mma_commit(&bars->empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -413,16 +475,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t stage = smem_u32(smem + STAGES * STAGE_BYTES + 1024) + q4 * Epi::kStageBytes;
+    // the epilogue's table (RoPE angle steps), made while the first loads fly
+    Epi::init(a.p, bars);
+    tc::named_sync(1, 128);
     int it = 0;
-    for (int item = blockIdx.x; item < a.num_items; item += gridDim.x, ++it) {
+    for (int item = item0; item < a.num_items; item += item_step, ++it) {
       const int buf = it & 1;
       int m0, n0, width;
       item_tile<BN>(a, item, m0, n0, width);
-      Epi::template prefetch<BN>(a, m0, n0, q4, stage);
+      if (rank == 0) Epi::template prefetch<BN>(a, m0, n0, q4, stage);
       const bool got = mbar_wait(&bars->acc_full[buf], (it >> 1) & 1, err);
       if (!__all_sync(0xffffffffu, got)) break;
       tc::fence_after_sync();
       const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16) + buf * BN;
+      if (ks > 1) {
+        // K split: the leader's epilogue runs once every rank's sums are in
+        if constexpr (BN <= 128) {
+          if (rank > 0) store_partial<BN>(tbase, row, smem_u32(smem));
+        }
+        break;
+      }
       if constexpr (BN == 256) {
         if (width == BN) Epi::template tile<BN>(a, bars, tbase, m0, n0, row, stage);
         else Epi::template tile<BN / 2>(a, bars, tbase, m0, n0, row, stage);
@@ -438,6 +510,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
 
   tc::fence_before_sync();
   __syncthreads();
+  if constexpr (BN <= 128) {
+    if (ks > 1) {
+      // every rank's partial sums are in its shared memory
+      tc::cluster_sync();
+      if (rank == 0 && warp >= 2 && !*reinterpret_cast<volatile int*>(&bars->abort)) {
+        tc::fence_after_sync();
+        const int q4 = warp & 3, row = q4 * 32 + lane;
+        const uint32_t stage = smem_u32(smem + STAGES * STAGE_BYTES + 1024) + q4 * Epi::kStageBytes;
+        const uint32_t tbase = tmem + ((uint32_t)(q4 * 32) << 16);
+        int m0, n0, width;
+        item_tile<BN>(a, item0, m0, n0, width);
+        add_partials<BN>(tbase, row, smem_u32(smem), ks);
+        Epi::template tile<BN>(a, bars, tbase, m0, n0, row, stage);
+        cp_async_wait<0>();
+      }
+      // no rank leaves while the leader may still read its shared memory
+      tc::cluster_sync();
+      tc::fence_before_sync();
+      __syncthreads();
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     tc::fence_after_sync();
@@ -447,7 +540,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
 
 template <class Epi, class Cfg>
 cudaError_t launch_cfg(const typename Epi::Params& p, const void* x, const void* w, int T, int K, int N,
-                       int n_heads_total, int num_sms, cudaStream_t st) {
+                       int n_heads_total, int num_sms, cudaStream_t st, int ksplit = 1) {
   constexpr int SMEM = Cfg::SMEM_BYTES + 4 * Epi::kStageBytes;
   static_assert(SMEM <= 232448, "227 KB of shared memory per CTA");
   static std::atomic<bool> attr_set[64];
@@ -463,8 +556,9 @@ cudaError_t launch_cfg(const typename Epi::Params& p, const void* x, const void*
   a.num_kb = (K + BK - 1) / BK;
   // a partial last wave of wide tiles goes as twice as many half-width tiles
   // when they still fit in one wave
+  a.ksplit = ksplit;
   const int rem = num_sms > 0 ? a.num_tiles % num_sms : 0;
-  if (Cfg::BN == 256 && a.num_tiles > num_sms && rem > 0 && 2 * rem <= num_sms) {
+  if (Cfg::BN == 256 && ksplit == 1 && a.num_tiles > num_sms && rem > 0 && 2 * rem <= num_sms) {
     a.n_full = a.num_tiles - rem;
     a.num_items = a.num_tiles + rem;
   } else {
@@ -474,9 +568,34 @@ cudaError_t launch_cfg(const typename Epi::Params& p, const void* x, const void*
   if (!make_tmap_bf16_2d(&tx, x, K, T, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tw, w, K, N, (uint64_t)K * 2, BK, Cfg::BN)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tw_half, w, K, N, (uint64_t)K * 2, BK, Cfg::BN / 2)) return cudaErrorInvalidValue;
+  if (ksplit > 1) {   // one tile per CTA, the ksplit CTAs of a tile in one cluster
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.num_tiles * ksplit));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ksplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<Epi, Cfg>, tx, tw, tw_half, a);
+  }
   const int grid = a.num_items < num_sms ? a.num_items : num_sms;
   gemm_tc_kernel<Epi, Cfg><<<grid, THREADS, SMEM, st>>>(tx, tw, tw_half, a);
   return cudaGetLastError();
+}
+
+// K split for problems whose narrow tiles fill less than half of the SMs:
+// two CTAs per tile, each with at least 4 k-blocks.  Measured on B200 (128
+// tokens, hidden 2048): 3 or 4 ranks were no faster than 2 for the QKV
+// projection and slower for the output projection (the leader reads more
+// partials), and 48 clusters of 3 CTAs of ~210 KB did not all fit at once.
+inline int ksplit_for(long long tiles, int num_kb, int num_sms) {
+  if (tiles <= 0 || 2 * tiles > num_sms || num_kb < 8) return 1;
+  return 2;
 }
 
 // Wide tiles unless they would leave more than half of the SMs idle; then
@@ -486,10 +605,13 @@ cudaError_t launch_gemm(const typename Epi::Params& p, const void* x, const void
                         int n_heads_total, int num_sms, cudaStream_t st) {
   const long long wide_tiles = (long long)((T + BM - 1) / BM) * ((N + 255) / 256);
   if (2 * wide_tiles >= num_sms) return launch_cfg<Epi, GemmCfg<256, 4>>(p, x, w, T, K, N, n_heads_total, num_sms, st);
+  constexpr int NBN = MIN_BN <= 64 ? 64 : 128;
+  const long long tiles = (long long)((T + BM - 1) / BM) * ((N + NBN - 1) / NBN);
+  const int ks = ksplit_for(tiles, (K + BK - 1) / BK, num_sms);
   if constexpr (MIN_BN <= 64)
-    return launch_cfg<Epi, GemmCfg<64, 8>>(p, x, w, T, K, N, n_heads_total, num_sms, st);
+    return launch_cfg<Epi, GemmCfg<64, 8>>(p, x, w, T, K, N, n_heads_total, num_sms, st, ks);
   else
-    return launch_cfg<Epi, GemmCfg<128, 6>>(p, x, w, T, K, N, n_heads_total, num_sms, st);
+    return launch_cfg<Epi, GemmCfg<128, 6>>(p, x, w, T, K, N, n_heads_total, num_sms, st, ks);
 }
 
 }  // namespace

@@ -56,6 +56,12 @@ QKV_CASES = [
     ("bf16", 1, 4000, 256, 8, 2, 128, 4096, False),  # the same split at hd 128 (a half tile is one head)
     ("bf16", 3, 2000, 256, 10, 2, 64, 2048, True),  # N = 896: the last column tile's second half lies past N
     ("bf16", 2, 70, 100, 4, 2, 64, 80, True),       # hidden % 8 != 0: the SIMT path
+    # 128 tokens or fewer over tiles that fill less than half of the SMs: the K
+    # split across a cluster (ranks' partial sums added by the leader)
+    ("bf16", 1, 128, 2048, 32, 4, 64, 128, False),  # TinyLlama 1 x 128: 40 tiles x 2 ranks
+    ("bf16", 1, 100, 2048, 32, 4, 64, 160, True),   # ragged T: rows past T masked in every rank
+    ("bf16", 1, 96, 4096, 32, 8, 128, 96, True),    # hd 128: 48 tiles of 128 columns x 2 ranks
+    ("bf16", 2, 50, 1024, 16, 4, 32, 64, True),     # hd 32: 12 tiles x 2 ranks
     # few tokens, hidden % 64 == 0 and the hidden states fit in shared memory:
     # the TMA-ring kernel, every token-count variant
     ("bf16", 3, 1, 2048, 32, 4, 64, 16, True),
