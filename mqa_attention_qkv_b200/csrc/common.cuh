@@ -97,6 +97,16 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may start while the kernel before it in the
+// stream is still running: it must wait (pdl_wait) before its first access to
+// global memory that the earlier kernel may write or read, after which all of
+// that kernel's writes are visible.  Without such a predecessor both are
+// no-ops.  pdl_launch_dependents lets the next kernel in the stream launch as
+// soon as every CTA of this one has issued it (that kernel waits in its turn).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

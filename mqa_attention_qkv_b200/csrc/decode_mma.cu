@@ -108,6 +108,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant
   const int hg = CL ? blockIdx.x / p.n_split : blockIdx.x % n_hgrp;
   const int g = p.nh / p.nkv;
   int* err = p.err;
+  pdl_launch_dependents();
+  pdl_wait();   // q, the lengths and the new cache rows may come from the kernel before this one
 
   int kv_len = p.kv_lens[b];
   if (kv_len > p.cap || kv_len < 0) {
@@ -524,23 +526,9 @@ cudaError_t launch_hd(const DecodeParams& p, cudaStream_t st) {
   if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, rows, HD * 2, 64, KT)) return cudaErrorInvalidValue;
   const dim3 grid((unsigned)(p.n_split * p.n_hgrp), p.nkv, p.B);
-  if (!CL) {
-    decode_mma_kernel<HD, MT, false><<<grid, THREADS, C::SMEM, st>>>(tk, tv, p, p.n_hgrp);
-    return cudaGetLastError();
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.n_split;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_mma_kernel<HD, MT, true>, tk, tv, p, p.n_hgrp);
+  if (!CL) return launch_ex(decode_mma_kernel<HD, MT, false>, grid, dim3(THREADS), C::SMEM, st, 1u, tk, tv, p, p.n_hgrp);
+  return launch_ex(decode_mma_kernel<HD, MT, true>, grid, dim3(THREADS), C::SMEM, st, (unsigned)p.n_split, tk, tv, p,
+                   p.n_hgrp);
 }
 
 // Splits per (sequence, KV head, head group) for the cluster-merged decode,

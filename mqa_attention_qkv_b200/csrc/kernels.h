@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 namespace gqa {
 
@@ -183,6 +184,34 @@ int launch_decode(const DecodeParams& p, bool bf16, cudaStream_t st, cudaError_t
 // and a 215 KB shared-memory configuration lost ~25 us at the switch).  The
 // attributes are idempotent, so two threads racing on a first call both set
 // them; devices past the array are set on every call.
+// Launch with programmatic stream serialization (the kernel calls pdl_wait
+// before touching global memory) and, for cluster_x > 1, clusters of
+// cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 inline cudaError_t smem_attr_once(std::atomic<bool> (&done)[64], const void* func, int bytes) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {

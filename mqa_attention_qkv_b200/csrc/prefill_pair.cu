@@ -68,6 +68,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   Bars* bars = reinterpret_cast<Bars*>(smem + BAR_OFF);
   int* err = p.err;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  pdl_launch_dependents();
+  pdl_wait();   // lengths, offsets and inputs may come from the kernel before this one
 
   const int bh_count = p.B * p.nh;
   const int u = blockIdx.x;
@@ -429,8 +431,8 @@ cudaError_t launch_pair(const PrefillParams& p, cudaStream_t st) {
   }
   const int n_qt = (p.S + BQ - 1) / BQ;
   const long long grid = (long long)n_qt * p.B * p.nh;
-  prefill_pair_kernel<VARLEN><<<(unsigned)grid, THREADS, SMEM, st>>>(tq, tk, tv, p, n_qt);
-  return cudaGetLastError();
+  return launch_ex(prefill_pair_kernel<VARLEN>, dim3((unsigned)grid), dim3(THREADS), SMEM, st, 1u, tq, tk, tv, p,
+                   n_qt);
 }
 
 }  // namespace

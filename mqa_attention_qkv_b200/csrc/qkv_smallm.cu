@@ -270,6 +270,7 @@ w_stream_kernel(const __grid_constant__ CUtensorMap tmw, typename Epi::Params p,
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int T = Epi::T(p);
   int* err = Epi::err(p);
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstages; ++s) {
@@ -279,6 +280,7 @@ w_stream_kernel(const __grid_constant__ CUtensorMap tmw, typename Epi::Params p,
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();   // the inputs may come from the kernel before this one
 
   if (warp == SW_WARPS) {
     // ------------------------------------------------------------ TMA producer
@@ -481,8 +483,8 @@ cudaError_t launch_stream_epi(const typename Epi::Params& p, const void* w, int 
   const uint32_t wbox[3] = {64, 8, SW_KB};
   if (!make_tmap_bf16_3d(&tw, w, wd, ws, wbox)) return cudaErrorInvalidValue;
   const int grid = n_units < per_sm * num_sms ? n_units : per_sm * num_sms;
-  w_stream_kernel<NT, Epi><<<grid, (SW_WARPS + 1) * 32, smem, st>>>(tw, p, n_units, stages);
-  return cudaGetLastError();
+  return launch_ex(w_stream_kernel<NT, Epi>, dim3((unsigned)grid), dim3((SW_WARPS + 1) * 32), smem, st, 1u, tw, p,
+                   n_units, stages);
 }
 
 template <int NT, int HD>

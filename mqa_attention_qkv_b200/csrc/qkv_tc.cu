@@ -379,6 +379,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
   Bars* bars = reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   int* err = a.p.err;
+  pdl_launch_dependents();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -403,6 +404,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ 
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
+  pdl_wait();   // the inputs may come from the kernel before this one
   // K split: rank within the cluster, its k-blocks, and one tile per CTA
   const int ks = a.ksplit, rank = ks > 1 ? (int)(blockIdx.x % ks) : 0;
   const int item0 = ks > 1 ? (int)(blockIdx.x / ks) : (int)blockIdx.x;
@@ -568,24 +570,10 @@ cudaError_t launch_cfg(const typename Epi::Params& p, const void* x, const void*
   if (!make_tmap_bf16_2d(&tx, x, K, T, (uint64_t)K * 2, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tw, w, K, N, (uint64_t)K * 2, BK, Cfg::BN)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tw_half, w, K, N, (uint64_t)K * 2, BK, Cfg::BN / 2)) return cudaErrorInvalidValue;
-  if (ksplit > 1) {   // one tile per CTA, the ksplit CTAs of a tile in one cluster
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(a.num_tiles * ksplit));
-    cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)ksplit;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<Epi, Cfg>, tx, tw, tw_half, a);
-  }
-  const int grid = a.num_items < num_sms ? a.num_items : num_sms;
-  gemm_tc_kernel<Epi, Cfg><<<grid, THREADS, SMEM, st>>>(tx, tw, tw_half, a);
-  return cudaGetLastError();
+  // K split: one tile per CTA, the ksplit CTAs of a tile in one cluster
+  const int grid = ksplit > 1 ? a.num_tiles * ksplit : (a.num_items < num_sms ? a.num_items : num_sms);
+  return launch_ex(gemm_tc_kernel<Epi, Cfg>, dim3((unsigned)grid), dim3(THREADS), SMEM, st, (unsigned)ksplit,
+                   tx, tw, tw_half, a);
 }
 
 // K split for problems whose narrow tiles fill less than half of the SMs:
