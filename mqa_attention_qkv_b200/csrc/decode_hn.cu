@@ -185,13 +185,15 @@ struct PieceWalk {
   }
 };
 
-// Merge of a unit's np partials, written to slots slot0 .. slot0 + np - 1
-// (o rows, then (m, l) per head), into its bf16 output rows, by the 128
+// Merge of a unit's np partials, written to workspace slots slot0 .. slot0 +
+// np - 1 (o rows, then (m, l) per head), into its bf16 output rows, by the 128
 // epilogue threads (te).  Per group of 32 heads, thread te takes float4
-// columns d4 of heads hg + h0, hg + h0 + 4, ...; the pieces go two at a time
-// with all their (m, l) and o loads in flight at once, folded into a running
-// maximum, sum and accumulator per head.  Kept out of line so that its
-// registers do not add to those of the pipeline loops.
+// columns d4 of heads hg + h0, hg + h0 + 4, ...  The arithmetic is that of
+// merge_smem, step for step (the maximum over the pieces in piece order,
+// then fmaf sums weighted by 2^(m_k - M) in piece order), so that a unit's
+// output has the same bits whichever of its pieces finishes last and merges;
+// the second pass keeps two pieces' loads in flight.  Kept out of line so
+// that its registers do not add to those of the pipeline loops.
 template <int NP>
 __device__ __noinline__ void merge_unit(const DecodeParams& p, int g, int b, int j, int slot0, int np, int te,
                                         __nv_bfloat16* out) {
@@ -208,6 +210,15 @@ __device__ __noinline__ void merge_unit(const DecodeParams& p, int g, int b, int
       M[i] = -INFINITY;
       Lr[i] = 0.f;
       acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll 1
+    for (int k = 0; k < np; ++k) {
+      const float* slot_k = p.ws + (size_t)(slot0 + k) * NP * WS_ROW;
+#pragma unroll
+      for (int i = 0; i < NH; ++i) {
+        const int h = hg + h0 + 4 * i;
+        if (h < g) M[i] = fmaxf(M[i], __ldcg(slot_k + h * WS_ROW + HD));
+      }
     }
 #pragma unroll 1
     for (int k0 = 0; k0 < np; k0 += KC) {
@@ -230,17 +241,15 @@ __device__ __noinline__ void merge_unit(const DecodeParams& p, int g, int b, int
       }
 #pragma unroll
       for (int k = 0; k < KC; ++k) {
+        if (k0 + k >= np) break;
 #pragma unroll
         for (int i = 0; i < NH; ++i) {
-          if (ml[k][i].x == -INFINITY) continue;
-          const float Mn = fmaxf(M[i], ml[k][i].x);
-          const float a = tc::ex2(M[i] - Mn), wk = tc::ex2(ml[k][i].x - Mn);
-          Lr[i] = Lr[i] * a + ml[k][i].y * wk;
-          acc[i].x = acc[i].x * a + ov[k][i].x * wk;
-          acc[i].y = acc[i].y * a + ov[k][i].y * wk;
-          acc[i].z = acc[i].z * a + ov[k][i].z * wk;
-          acc[i].w = acc[i].w * a + ov[k][i].w * wk;
-          M[i] = Mn;
+          const float wk = tc::ex2(ml[k][i].x - M[i]);
+          Lr[i] = fmaf(ml[k][i].y, wk, Lr[i]);
+          acc[i].x = fmaf(ov[k][i].x, wk, acc[i].x);
+          acc[i].y = fmaf(ov[k][i].y, wk, acc[i].y);
+          acc[i].z = fmaf(ov[k][i].z, wk, acc[i].z);
+          acc[i].w = fmaf(ov[k][i].w, wk, acc[i].w);
         }
       }
     }
@@ -292,6 +301,8 @@ template <int NP>
 __global__ void __launch_bounds__(THREADS, 1)
 decode_hn_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, DecodeParams p, int rows_total) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   using C = HnCfg<NP>;
   constexpr int KS = C::KS, VS = C::VS;
   extern __shared__ uint8_t smem_raw[];
@@ -787,8 +798,7 @@ cudaError_t launch_np(const DecodeParams& p, cudaStream_t st) {
   if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, rows, HD * 2, 64, 64)) return cudaErrorInvalidValue;
   int grid = sm_count_cached();
   if (grid > kMaxGrid) grid = kMaxGrid;
-  decode_hn_kernel<NP><<<grid, THREADS, SMEM, st>>>(tq, tk, tv, p, (int)rows);
-  return cudaGetLastError();
+  return launch_ex(decode_hn_kernel<NP>, dim3((unsigned)grid), dim3(THREADS), SMEM, st, 1u, tq, tk, tv, p, (int)rows);
 }
 
 int hn_np(int nh, int nkv) { return (nh / nkv + 15) / 16 * 16; }

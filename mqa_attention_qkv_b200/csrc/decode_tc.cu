@@ -80,6 +80,8 @@ template <int HD>
 __global__ void __launch_bounds__(THREADS, 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                  const __grid_constant__ CUtensorMap tmv, DecodeParams p, int n_hg) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   using C = DtCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -432,19 +434,8 @@ cudaError_t launch_hd(const DecodeParams& p, int n_hg, cudaStream_t st) {
   if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, kv_rows, HD * 2, 64, BKV)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, kv_rows, HD * 2, 64, BKV)) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.n_split * n_hg), (unsigned)p.nkv, (unsigned)p.B);
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.n_split;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tc_kernel<HD>, tq, tk, tv, p, n_hg);
+  return launch_ex(decode_tc_kernel<HD>, dim3((unsigned)(p.n_split * n_hg), (unsigned)p.nkv, (unsigned)p.B),
+                   dim3(THREADS), C::SMEM, st, (unsigned)p.n_split, tq, tk, tv, p, n_hg);
 }
 
 }  // namespace

@@ -125,6 +125,8 @@ __device__ __forceinline__ RowRef row_ref(const Fp8QuantParams& p, long long r) 
 
 template <int HD>
 __global__ void __launch_bounds__(256) fp8_amax_kernel(Fp8QuantParams p, long long n_rows) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   constexpr int E = HD / 32;
   const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const long long nwarps = (long long)gridDim.x * blockDim.x / 32;
@@ -157,6 +159,8 @@ __device__ __forceinline__ float inv_scale(const float* amax, int t) {
 // q and k rows -> e4m3 rows (rotated)
 template <int HD>
 __global__ void __launch_bounds__(256) fp8_quant_qk_kernel(Fp8QuantParams p, long long n_rows) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   constexpr int E = HD / 32;
   const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const long long nwarps = (long long)gridDim.x * blockDim.x / 32;
@@ -181,6 +185,8 @@ __global__ void __launch_bounds__(256) fp8_quant_qk_kernel(Fp8QuantParams p, lon
 // v rows -> e4m3, transposed per (b, j) to [hd, cap]; CTA = 64 slots of one (b, j)
 template <int HD>
 __global__ void __launch_bounds__(256) fp8_quant_v_kernel(Fp8QuantParams p, int slot_tiles) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   constexpr int E = HD / 32, SLOTS = 64;
   __shared__ uint8_t tile[HD][SLOTS + 4];
   const int bj = blockIdx.x / slot_tiles, s0 = (blockIdx.x % slot_tiles) * SLOTS;
@@ -225,15 +231,17 @@ cudaError_t launch_hd(const Fp8QuantParams& p, int num_sms, cudaStream_t st) {
   const long long rows = nq + 2 * nc;
   long long blocks = (rows + 7) / 8;
   if (blocks > (long long)num_sms * 16) blocks = (long long)num_sms * 16;
-  fp8_amax_kernel<HD><<<(unsigned)blocks, 256, 0, st>>>(p, rows);
-  if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
+  if (cudaError_t e = launch_ex(fp8_amax_kernel<HD>, dim3((unsigned)blocks), dim3(256), 0, st, 1u, p, rows);
+      e != cudaSuccess)
+    return e;
   long long qk_blocks = (nq + nc + 7) / 8;
   if (qk_blocks > (long long)num_sms * 16) qk_blocks = (long long)num_sms * 16;
-  fp8_quant_qk_kernel<HD><<<(unsigned)qk_blocks, 256, 0, st>>>(p, nq + nc);
-  if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
+  if (cudaError_t e = launch_ex(fp8_quant_qk_kernel<HD>, dim3((unsigned)qk_blocks), dim3(256), 0, st, 1u, p, nq + nc);
+      e != cudaSuccess)
+    return e;
   const int slot_tiles = (p.cap + 63) / 64;
-  fp8_quant_v_kernel<HD><<<(unsigned)((long long)p.B * p.nkv * slot_tiles), 256, 0, st>>>(p, slot_tiles);
-  return cudaGetLastError();
+  return launch_ex(fp8_quant_v_kernel<HD>, dim3((unsigned)((long long)p.B * p.nkv * slot_tiles)), dim3(256), 0, st, 1u,
+                   p, slot_tiles);
 }
 
 }  // namespace

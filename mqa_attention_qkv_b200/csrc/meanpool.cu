@@ -64,6 +64,8 @@ __device__ __forceinline__ void store_vec(void* p, const float (&v)[Vec<BF16>::N
 template <bool BF16>
 __global__ void __launch_bounds__(256) meanpool_kernel(const void* __restrict__ w_in, void* __restrict__ w_out, int nh,
                                                        int nkv, int hd, int D, long long n_vec) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   using V = Vec<BF16>;
   using T = typename V::T;
   const T* in = static_cast<const T*>(w_in);
@@ -126,13 +128,16 @@ extern "C" int gqa_meanpool_kv_heads(const void* w_qkv_mha, int hidden, int n_he
   long long grid = (n_vec + 255) / 256;
   if (grid > 148 * 8) grid = 148 * 8;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dtype == GQA_BF16)
-    gqa::meanpool_kernel<true><<<(unsigned)grid, 256, 0, s>>>(w_qkv_mha, w_qkv_gqa, n_heads, n_kv_heads, head_dim,
-                                                               hidden, n_vec);
-  else
-    gqa::meanpool_kernel<false><<<(unsigned)grid, 256, 0, s>>>(w_qkv_mha, w_qkv_gqa, n_heads, n_kv_heads,
-                                                                head_dim, hidden, n_vec);
+  const cudaError_t e =
+      dtype == GQA_BF16
+          ? gqa::launch_ex(gqa::meanpool_kernel<true>, dim3((unsigned)grid), dim3(256), 0, s, 1u, w_qkv_mha, w_qkv_gqa,
+                           n_heads, n_kv_heads, head_dim, hidden, n_vec)
+          : gqa::launch_ex(gqa::meanpool_kernel<false>, dim3((unsigned)grid), dim3(256), 0, s, 1u, w_qkv_mha, w_qkv_gqa,
+                           n_heads, n_kv_heads, head_dim, hidden, n_vec);
   gqa::count_launches(1);
-  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH_FAILED;
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_LAUNCH_FAILED;
+  }
   return GQA_OK;
 }

@@ -64,6 +64,8 @@ template <int NT>
 __global__ void __launch_bounds__(THREADS, 1)
 oproj_smallt_kernel(const __grid_constant__ CUtensorMap tmw, const __grid_constant__ CUtensorMap tmx, OprojParams p,
                     int split, int n_kb) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   using C = SmallCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -254,19 +256,8 @@ cudaError_t launch_nt(const OprojParams& p, int num_sms, cudaStream_t st) {
   CUtensorMap tw, tx;
   if (!make_tmap_bf16_2d(&tw, p.w, p.K, p.N, (uint64_t)p.K * 2, BK, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tx, p.x, p.K, p.T, (uint64_t)p.K * 2, BK, NT)) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(n_mblk * split), 1, 1);
-  cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)split;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, oproj_smallt_kernel<NT>, tw, tx, p, split, n_kb);
+  return launch_ex(oproj_smallt_kernel<NT>, dim3((unsigned)(n_mblk * split)), dim3(THREADS), C::SMEM, st,
+                   (unsigned)split, tw, tx, p, split, n_kb);
 }
 
 }  // namespace

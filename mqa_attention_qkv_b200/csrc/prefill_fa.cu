@@ -75,6 +75,8 @@ template <int HD, int POLY, bool VARLEN>
 __global__ void __launch_bounds__(THREADS, 1)
 prefill_fa_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, PrefillParams p, int n_qt) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   using C = FaCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -440,8 +442,8 @@ cudaError_t launch_hd(const PrefillParams& p, cudaStream_t st) {
   }
   const int n_qt = (p.S + BQ - 1) / BQ;
   const long long grid = (long long)((n_qt + 1) / 2) * p.B * p.nh;
-  prefill_fa_kernel<HD, POLY, VARLEN><<<(unsigned)grid, THREADS, C::SMEM, st>>>(tq, tk, tv, p, n_qt);
-  return cudaGetLastError();
+  return launch_ex(prefill_fa_kernel<HD, POLY, VARLEN>, dim3((unsigned)grid), dim3(THREADS), C::SMEM, st, 1u, tq, tk,
+                   tv, p, n_qt);
 }
 
 }  // namespace

@@ -82,6 +82,8 @@ struct Bars {
 __global__ void __launch_bounds__(THREADS, 1)
 prefill_fp8_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                    const __grid_constant__ CUtensorMap tmv, Fp8AttnParams p, int n_qt) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + BAR_OFF);
@@ -390,8 +392,7 @@ cudaError_t launch_prefill_fp8(const Fp8AttnParams& p, cudaStream_t st) {
   if (!make_tmap_u8_2d(&tv, p.v8t, (uint64_t)p.cap, v_rows, (uint64_t)p.cap, 128, 128)) return cudaErrorInvalidValue;
   const int n_qt = (p.S + BQ - 1) / BQ;
   const long long grid = (long long)((n_qt + 1) / 2) * p.B * p.nh;
-  prefill_fp8_kernel<<<(unsigned)grid, THREADS, SMEM, st>>>(tq, tk, tv, p, n_qt);
-  return cudaGetLastError();
+  return launch_ex(prefill_fp8_kernel, dim3((unsigned)grid), dim3(THREADS), SMEM, st, 1u, tq, tk, tv, p, n_qt);
 }
 
 }  // namespace gqa

@@ -89,6 +89,8 @@ __device__ __forceinline__ void rope_store_pair(const QkvParams& p, int hb, int 
 
 template <int NT, int HD>
 __global__ void __launch_bounds__(WARPS * 32, 2) qkv_smallm_kernel(QkvParams p) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   constexpr int U = NT == 1 ? 8 : (NT == 2 ? 4 : 2);   // K blocks in flight per thread
   constexpr int TP = NT * 8;                            // padded token count
   __shared__ float red[WARPS][16][TP + 1];
@@ -507,12 +509,11 @@ cudaError_t launch_nt(const QkvParams& p, cudaStream_t st) {
   const int N = (p.nh + 2 * p.nkv) * p.hd;
   const unsigned grid = (unsigned)(N / 16);
   switch (p.hd) {
-    case 32: qkv_smallm_kernel<NT, 32><<<grid, WARPS * 32, 0, st>>>(p); break;
-    case 64: qkv_smallm_kernel<NT, 64><<<grid, WARPS * 32, 0, st>>>(p); break;
-    case 128: qkv_smallm_kernel<NT, 128><<<grid, WARPS * 32, 0, st>>>(p); break;
+    case 32: return launch_ex(qkv_smallm_kernel<NT, 32>, dim3(grid), dim3(WARPS * 32), 0, st, 1u, p);
+    case 64: return launch_ex(qkv_smallm_kernel<NT, 64>, dim3(grid), dim3(WARPS * 32), 0, st, 1u, p);
+    case 128: return launch_ex(qkv_smallm_kernel<NT, 128>, dim3(grid), dim3(WARPS * 32), 0, st, 1u, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace

@@ -25,6 +25,8 @@ namespace {
 // ---------------------------------------------------------------------------
 template <typename T, int HD>
 __global__ void __launch_bounds__(256) qkv_simt_kernel(QkvParams p) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   constexpr int BM = 32, BK = 32, HALF = HD / 2, NRG = 256 / HALF, RPT = BM / NRG;
   __shared__ float xs[BM][BK + 1];
   __shared__ float ws[HD][BK + 1];
@@ -117,6 +119,8 @@ __device__ __forceinline__ float round_p<__nv_bfloat16>(float v) {
 
 template <typename T, int HD, bool DECODE>
 __global__ void __launch_bounds__(128) attn_simt_kernel(PrefillParams pp, DecodeParams dp) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   constexpr int PER = HD / 32;
   __shared__ float qs[kRows][HD];
   __shared__ float ks[kKT][HD + 1];
@@ -282,6 +286,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(PrefillParams pp, Decode
 // ---------------------------------------------------------------------------
 template <typename T, int HD>
 __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   constexpr int PER = HD / 32;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const size_t row = (size_t)blockIdx.x * 4 + warp;
@@ -319,6 +325,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(DecodeParams p) {
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(128) oproj_simt_kernel(OprojParams p) {
+  pdl_launch_dependents();
+  pdl_wait();   // inputs may come from the kernel before this one
   constexpr int CH = 256;
   __shared__ float xs[CH];
   const int n = blockIdx.x * 128 + threadIdx.x;
@@ -347,36 +355,33 @@ cudaError_t qkv_dispatch(const QkvParams& p, cudaStream_t st) {
   const int T_tot = p.B * p.S;
   dim3 grid((T_tot + 31) / 32, p.nh + 2 * p.nkv);
   switch (p.hd) {
-    case 32: qkv_simt_kernel<T, 32><<<grid, 256, 0, st>>>(p); break;
-    case 64: qkv_simt_kernel<T, 64><<<grid, 256, 0, st>>>(p); break;
-    case 128: qkv_simt_kernel<T, 128><<<grid, 256, 0, st>>>(p); break;
+    case 32: return launch_ex(qkv_simt_kernel<T, 32>, dim3(grid), dim3(256), 0, st, 1u, p);
+    case 64: return launch_ex(qkv_simt_kernel<T, 64>, dim3(grid), dim3(256), 0, st, 1u, p);
+    case 128: return launch_ex(qkv_simt_kernel<T, 128>, dim3(grid), dim3(256), 0, st, 1u, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 template <typename T, bool DECODE>
 cudaError_t attn_dispatch(const PrefillParams& pp, const DecodeParams& dp, dim3 grid, int hd,
                           cudaStream_t st) {
   switch (hd) {
-    case 32: attn_simt_kernel<T, 32, DECODE><<<grid, 128, 0, st>>>(pp, dp); break;
-    case 64: attn_simt_kernel<T, 64, DECODE><<<grid, 128, 0, st>>>(pp, dp); break;
-    case 128: attn_simt_kernel<T, 128, DECODE><<<grid, 128, 0, st>>>(pp, dp); break;
+    case 32: return launch_ex(attn_simt_kernel<T, 32, DECODE>, dim3(grid), dim3(128), 0, st, 1u, pp, dp);
+    case 64: return launch_ex(attn_simt_kernel<T, 64, DECODE>, dim3(grid), dim3(128), 0, st, 1u, pp, dp);
+    case 128: return launch_ex(attn_simt_kernel<T, 128, DECODE>, dim3(grid), dim3(128), 0, st, 1u, pp, dp);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 template <typename T>
 cudaError_t combine_dispatch(const DecodeParams& p, cudaStream_t st) {
   dim3 grid((unsigned)(((size_t)p.B * p.nh + 3) / 4));
   switch (p.hd) {
-    case 32: decode_combine_kernel<T, 32><<<grid, 128, 0, st>>>(p); break;
-    case 64: decode_combine_kernel<T, 64><<<grid, 128, 0, st>>>(p); break;
-    case 128: decode_combine_kernel<T, 128><<<grid, 128, 0, st>>>(p); break;
+    case 32: return launch_ex(decode_combine_kernel<T, 32>, dim3(grid), dim3(128), 0, st, 1u, p);
+    case 64: return launch_ex(decode_combine_kernel<T, 64>, dim3(grid), dim3(128), 0, st, 1u, p);
+    case 128: return launch_ex(decode_combine_kernel<T, 128>, dim3(grid), dim3(128), 0, st, 1u, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace
@@ -403,11 +408,8 @@ cudaError_t launch_decode_simt(const DecodeParams& p, bool bf16, cudaStream_t st
 
 cudaError_t launch_oproj_simt(const OprojParams& p, bool bf16, cudaStream_t st) {
   dim3 grid((unsigned)((p.N + 127) / 128), (unsigned)(p.T < 65535 ? p.T : 65535));
-  if (bf16)
-    oproj_simt_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(p);
-  else
-    oproj_simt_kernel<float><<<grid, 128, 0, st>>>(p);
-  return cudaGetLastError();
+  if (bf16) return launch_ex(oproj_simt_kernel<__nv_bfloat16>, dim3(grid), dim3(128), 0, st, 1u, p);
+  return launch_ex(oproj_simt_kernel<float>, dim3(grid), dim3(128), 0, st, 1u, p);
 }
 
 namespace {
