@@ -86,6 +86,20 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const int row = (warp & 3) * 32 + lane;
   int my_lim = 0;
   bool my_valid = false;
+  // Without explicit positions a row's key limit grows with the row, so the
+  // tile's key tiles follow from its last row, and thread 0 (the TMA thread)
+  // can issue Q and the first two K tiles as soon as the barriers exist.
+  const bool closed = p.q_pos == nullptr;
+  const int rows_here = min(BQ, sq.S - s0);
+  const int hi_closed = !p.causal ? kv_len : max(0, min(kv_len, kv_len - sq.S + s0 + rows_here));
+  const int n_kv_closed = (hi_closed + BKV - 1) / BKV;
+  const int kv_row0 = VARLEN ? 0 : (b * p.nkv + j) * p.cap;
+  // failure-path testing only: the first CTA leaves one K tile unloaded
+  const int skip = blockIdx.x == 0 ? p.dbg_skip_tile1 - 1 : -1;
+  const int early_k = closed ? min(n_kv_closed, 2) : 0;   // K tiles issued before the role split
+  uint8_t* sQ = smem + Q_OFF;
+  uint8_t* sK = smem + K_OFF;
+  uint8_t* sV = smem + V_OFF;
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->v_clean, 1);
@@ -102,13 +116,26 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
     }
-    bars->lim_max = -1;
+    bars->lim_max = closed ? hi_closed : -1;
     fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
     tc::prefetch_tmap(&tmq);
     tc::prefetch_tmap(&tmk);
     tc::prefetch_tmap(&tmv);
+    if (closed && n_kv_closed > 0) {
+      mbar_arrive_expect_tx(&bars->q_full, TILE);
+      if (VARLEN)
+        tc::tma_load_3d(sQ, &tmq, 0, h, sq.q0 + s0, &bars->q_full);
+      else
+        tc::tma_load_2d(sQ, &tmq, 0, (b * p.nh + h) * p.S + s0, &bars->q_full);
+      for (int t = 0; t < early_k; ++t) {
+        if (t == skip) continue;
+        mbar_arrive_expect_tx(&bars->k_full[t], TILE);
+        if (VARLEN)
+          tc::tma_load_3d(sK + t * TILE, &tmk, 0, j, sq.k0 + t * BKV, &bars->k_full[t]);
+        else
+          tc::tma_load_2d(sK + t * TILE, &tmk, 0, kv_row0 + t * BKV, &bars->k_full[t]);
+      }
+    }
   }
   if (warp == 1) tc::tmem_alloc(&bars->tmem_base, kTmemCols);
   __syncthreads();
@@ -118,7 +145,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
     if (my_valid) {
       const int pos = p.q_pos ? p.q_pos[(size_t)b * p.S + s] : kv_len - sq.S + s;
       my_lim = p.causal ? max(0, min(kv_len, pos + 1)) : kv_len;
-      atomicMax(&bars->lim_max, my_lim);
+      if (!closed) atomicMax(&bars->lim_max, my_lim);
     }
   }
   tc::fence_before_sync();
@@ -128,10 +155,6 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
   const int kv_hi = bars->lim_max < 0 ? 0 : bars->lim_max;
   const int n_kv = (kv_hi + BKV - 1) / BKV;
   const bool sanitize = n_kv > 0 && kv_len < n_kv * BKV;
-  const int kv_row0 = VARLEN ? 0 : (b * p.nkv + j) * p.cap;
-  uint8_t* sQ = smem + Q_OFF;
-  uint8_t* sK = smem + K_OFF;
-  uint8_t* sV = smem + V_OFF;
 
   if (warp == 0) {
     // ================================================================ TMA
@@ -143,10 +166,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
       auto wait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait(bar, parity, err));
       };
-      // failure-path testing only: the first CTA leaves one K tile unloaded
-      const int skip = blockIdx.x == 0 ? p.dbg_skip_tile1 - 1 : -1;
-      int nk = 0, nv = 0;   // tiles issued
-      if (lane == 0) {
+      int nk = early_k, nv = 0;   // tiles issued
+      if (lane == 0 && !closed) {
         mbar_arrive_expect_tx(&bars->q_full, TILE);
         if (VARLEN)
           tc::tma_load_3d(sQ, &tmq, 0, h, sq.q0 + s0, &bars->q_full);
@@ -177,8 +198,10 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_consta
           tc::tma_load_2d(sV + st * TILE, &tmv, 0, kv_row0 + t * BKV, &bars->v_full[st]);
         return true;
       };
-      ok = load_k(0);
-      if (ok && n_kv > 1) ok = load_k(1);
+      if (early_k == 0) {
+        ok = load_k(0);
+        if (ok && n_kv > 1) ok = load_k(1);
+      }
       for (int t = 0; ok && t < n_kv; ++t) {
         if (t + 2 < n_kv) ok = load_k(t + 2);
         if (ok) ok = load_v(t);
