@@ -185,14 +185,35 @@ struct PieceWalk {
   }
 };
 
+// One step of the log-sum-exp merge: fold a piece's (m, l, o) into the
+// running (M, L, acc).  Both merges below take exactly these steps, in piece
+// order, with every product rounded on its own (no contraction into an FMA
+// the compiler might choose differently in the two places), so that a unit's
+// output has the same bits whichever of its pieces finishes last and merges.
+__device__ __forceinline__ void merge_step(float& M, float& L, float4& acc, float m_k, float l_k, const float4& v) {
+  if (m_k == -INFINITY) return;
+  const float Mn = fmaxf(M, m_k);
+  const float a = tc::ex2(M - Mn), wk = tc::ex2(m_k - Mn);
+  L = fmaf(l_k, wk, __fmul_rn(L, a));
+  acc.x = fmaf(v.x, wk, __fmul_rn(acc.x, a));
+  acc.y = fmaf(v.y, wk, __fmul_rn(acc.y, a));
+  acc.z = fmaf(v.z, wk, __fmul_rn(acc.z, a));
+  acc.w = fmaf(v.w, wk, __fmul_rn(acc.w, a));
+  M = Mn;
+}
+
+__device__ __forceinline__ void merge_store(__nv_bfloat16* dst_row, int d4, float L, const float4& acc) {
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(dst_row + d4);
+  dst[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  dst[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+}
+
 // Merge of a unit's np partials, written to workspace slots slot0 .. slot0 +
 // np - 1 (o rows, then (m, l) per head), into its bf16 output rows, by the 128
 // epilogue threads (te).  Per group of 32 heads, thread te takes float4
-// columns d4 of heads hg + h0, hg + h0 + 4, ...  The arithmetic is that of
-// merge_smem, step for step (the maximum over the pieces in piece order,
-// then fmaf sums weighted by 2^(m_k - M) in piece order), so that a unit's
-// output has the same bits whichever of its pieces finishes last and merges;
-// the second pass keeps two pieces' loads in flight.  Kept out of line so
+// columns d4 of heads hg + h0, hg + h0 + 4, ...; the pieces go two at a time
+// with all their (m, l) and o loads in flight at once.  Kept out of line so
 // that its registers do not add to those of the pipeline loops.
 template <int NP>
 __device__ __noinline__ void merge_unit(const DecodeParams& p, int g, int b, int j, int slot0, int np, int te,
@@ -210,15 +231,6 @@ __device__ __noinline__ void merge_unit(const DecodeParams& p, int g, int b, int
       M[i] = -INFINITY;
       Lr[i] = 0.f;
       acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll 1
-    for (int k = 0; k < np; ++k) {
-      const float* slot_k = p.ws + (size_t)(slot0 + k) * NP * WS_ROW;
-#pragma unroll
-      for (int i = 0; i < NH; ++i) {
-        const int h = hg + h0 + 4 * i;
-        if (h < g) M[i] = fmaxf(M[i], __ldcg(slot_k + h * WS_ROW + HD));
-      }
     }
 #pragma unroll 1
     for (int k0 = 0; k0 < np; k0 += KC) {
@@ -240,28 +252,14 @@ __device__ __noinline__ void merge_unit(const DecodeParams& p, int g, int b, int
         }
       }
 #pragma unroll
-      for (int k = 0; k < KC; ++k) {
-        if (k0 + k >= np) break;
+      for (int k = 0; k < KC; ++k)
 #pragma unroll
-        for (int i = 0; i < NH; ++i) {
-          const float wk = tc::ex2(ml[k][i].x - M[i]);
-          Lr[i] = fmaf(ml[k][i].y, wk, Lr[i]);
-          acc[i].x = fmaf(ov[k][i].x, wk, acc[i].x);
-          acc[i].y = fmaf(ov[k][i].y, wk, acc[i].y);
-          acc[i].z = fmaf(ov[k][i].z, wk, acc[i].z);
-          acc[i].w = fmaf(ov[k][i].w, wk, acc[i].w);
-        }
-      }
+        for (int i = 0; i < NH; ++i) merge_step(M[i], Lr[i], acc[i], ml[k][i].x, ml[k][i].y, ov[k][i]);
     }
 #pragma unroll
     for (int i = 0; i < NH; ++i) {
       const int h = hg + h0 + 4 * i;
-      if (h < g) {
-        const float inv = Lr[i] > 0.f ? 1.f / Lr[i] : 0.f;
-        __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * p.nh + j * g + h) * HD + d4);
-        dst[0] = __floats2bfloat162_rn(acc[i].x * inv, acc[i].y * inv);
-        dst[1] = __floats2bfloat162_rn(acc[i].z * inv, acc[i].w * inv);
-      }
+      if (h < g) merge_store(out + ((size_t)b * p.nh + j * g + h) * HD, d4, Lr[i], acc[i]);
     }
   }
 }
@@ -276,24 +274,13 @@ __device__ __noinline__ void merge_smem(const float* part, const DecodeParams& p
   const int d4 = (te & 31) * 4, h0 = te >> 5;
 #pragma unroll 2
   for (int h = h0; h < g; h += 4) {
-    float M = -INFINITY;
-    for (int k = 0; k < np; ++k) M = fmaxf(M, part[((size_t)k * NP + h) * WS_ROW + HD]);
-    float L = 0.f;
+    float M = -INFINITY, L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int k = 0; k < np; ++k) {
       const float* row = part + ((size_t)k * NP + h) * WS_ROW;
-      const float wk = tc::ex2(row[HD] - M);
-      const float4 v = *reinterpret_cast<const float4*>(row + d4);
-      L = fmaf(row[HD + 1], wk, L);
-      acc.x = fmaf(v.x, wk, acc.x);
-      acc.y = fmaf(v.y, wk, acc.y);
-      acc.z = fmaf(v.z, wk, acc.z);
-      acc.w = fmaf(v.w, wk, acc.w);
+      merge_step(M, L, acc, row[HD], row[HD + 1], *reinterpret_cast<const float4*>(row + d4));
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * p.nh + j * g + h) * HD + d4);
-    dst[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    dst[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    merge_store(out + ((size_t)b * p.nh + j * g + h) * HD, d4, L, acc);
   }
 }
 
