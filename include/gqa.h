@@ -22,6 +22,15 @@
  *   never allocates, frees, synchronises or prints.  Every call is
  *   asynchronous on `stream` (a cudaStream_t passed as void*; NULL = the
  *   legacy default stream) and may be captured in a CUDA graph.
+ * - Kernels are launched with programmatic stream serialization: a kernel of
+ *   the library may start while the kernel before it on `stream` is still
+ *   running, and waits for it (griddepcontrol.wait) before its first access
+ *   to global memory, so stream order holds for every buffer.  Each library
+ *   kernel also lets the next kernel on the stream launch early; a kernel of
+ *   the caller's that follows a library call and is itself launched with the
+ *   programmatic-serialization attribute must call
+ *   cudaGridDependencySynchronize() before it reads the call's outputs
+ *   (kernels launched without that attribute wait for completion as usual).
  * - Tensors are dense, row-major ("C order") with the shapes given below, and
  *   every tensor pointer must be 16-byte aligned (int32 arrays: 4-byte).
  * - dtype: GQA_F32 (float32 everywhere, FFMA arithmetic, no TF32) or
