@@ -557,9 +557,10 @@ cudaError_t launch_decode_mma(const DecodeParams& p, cudaStream_t st) {
 }
 
 int launch_decode(const DecodeParams& p0, bool bf16, cudaStream_t st, cudaError_t* err) {
-  if (bf16 && p0.auto_split && !p0.block_table) {
+  if (bf16 && p0.auto_split) {
     // large batches with large head groups: tcgen05 tiles (mma.sync would be
-    // tensor-bound there), splits merged inside a cluster
+    // tensor-bound there), splits merged inside a cluster; contiguous or
+    // paged (each 64-key tile mapped to its page)
     const int nc = decode_tc_splits(p0);
     if (nc > 0) {
       DecodeParams p = p0;
@@ -570,11 +571,11 @@ int launch_decode(const DecodeParams& p0, bool bf16, cudaStream_t st, cudaError_
     }
   }
   if (bf16 && decode_hn_ok(p0.B, p0.nh, p0.nkv, p0.hd, p0.cap, p0.auto_split != 0)) {
-    // the other large problems with head groups of 17..64 (paged caches and
-    // caches past the cluster kernel's 8 x 2048 keys): keys as the tcgen05
-    // rows, equal key ranges per SM.  On the contiguous B 64 MQA workload the
-    // cluster kernel above measured 52 us against this kernel's 54 us; with
-    // 64-key pages this kernel takes 56-59 us, the mma.sync kernel 62 us.
+    // the other large problems with head groups of 17..64 (caches past the
+    // cluster kernel's 8 x 2048 keys): keys as the tcgen05 rows, equal key
+    // ranges per SM.  On the B 64 MQA workload the cluster kernel above
+    // measured 42 us back to back against this kernel's 51 us, contiguous or
+    // with 64-key pages.
     *err = launch_decode_hn(p0, st);
     return 1;
   }

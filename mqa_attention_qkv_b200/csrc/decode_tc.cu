@@ -16,6 +16,9 @@
 // 32 heads, 1 KV head, hd 128, ragged 512..8192 keys: this kernel 51 us, the
 // mma.sync kernel 60 us, and this kernel with fixed 1024- or 2048-key splits
 // merged through a workspace instead of a cluster 63 / 55 us.
+// The cache is contiguous or paged: with a block table every 64-key tile is
+// mapped to its page (pages hold a multiple of 64 keys, so a tile never
+// crosses one), an entry outside the page pool is flagged and read as zeros.
 // CTA = (sequence b, KV head j, group of <= 128 heads, key split c); the
 // n_split CTAs of a (b, j, head group) form one thread-block cluster and the
 // sequence's 64-key tiles are dealt out evenly over them.  Per CTA:
@@ -106,7 +109,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
   const int n_t = t_hi - t_lo;
   const int k_lo = t_lo * BKV, k_hi = min(kv_len, t_hi * BKV);
   const bool sanitize = n_t > 0 && k_hi == kv_len && (kv_len % BKV) != 0;
-  const int kv_row0 = (b * p.nkv + j) * p.cap + k_lo;
+  // cache row of the 64-key tile that starts at `key`: contiguous
+  // [B, nkv, cap, hd], or through the block table (pages are multiples of 64
+  // keys, so a tile never crosses a page); an entry outside the page pool is
+  // flagged and its tile read past the pool's end, i.e. as zeros
+  auto tile_row = [&](int key) {
+    if (!p.block_table) return (b * p.nkv + j) * p.cap + key;
+    const int lp = key / p.page_size;
+    const int pg = __ldg(p.block_table + (size_t)b * p.max_pages + lp);
+    if (pg < 0 || pg >= p.num_pages) {
+      raise_error(err, GQA_DEVERR_PAGE_RANGE);
+      return p.num_pages * p.nkv * p.page_size;
+    }
+    return (pg * p.nkv + j) * p.page_size + (key - lp * p.page_size);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -152,17 +168,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant_
       auto load_k = [&](int t) {
         const int st = t % C::KS;
         if (!mbar_wait(&bars->k_empty[st], ((t / C::KS) & 1) ^ 1, err)) return false;
+        const int row = tile_row(k_lo + t * BKV);
         mbar_arrive_expect_tx(&bars->k_full[st], C::KV_TILE);
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tc::tma_load_2d(sK + st * C::KV_TILE + bx * C::KV_BOX, &tmk, bx * 64, kv_row0 + t * BKV, &bars->k_full[st]);
+          tc::tma_load_2d(sK + st * C::KV_TILE + bx * C::KV_BOX, &tmk, bx * 64, row, &bars->k_full[st]);
         return true;
       };
       auto load_v = [&](int t) {
         const int st = t % C::VS;
         if (!mbar_wait(&bars->v_empty[st], ((t / C::VS) & 1) ^ 1, err)) return false;
+        const int row = tile_row(k_lo + t * BKV);
         mbar_arrive_expect_tx(&bars->v_full[st], C::KV_TILE);
         for (int bx = 0; bx < C::NBOX; ++bx)
-          tc::tma_load_2d(sV + st * C::KV_TILE + bx * C::KV_BOX, &tmv, bx * 64, kv_row0 + t * BKV, &bars->v_full[st]);
+          tc::tma_load_2d(sV + st * C::KV_TILE + bx * C::KV_BOX, &tmv, bx * 64, row, &bars->v_full[st]);
         return true;
       };
       // K runs one tile ahead of V
@@ -430,7 +448,8 @@ cudaError_t launch_hd(const DecodeParams& p, int n_hg, cudaStream_t st) {
       e != cudaSuccess)
     return e;
   CUtensorMap tq, tk, tv;
-  const uint64_t q_rows = (uint64_t)p.B * p.nh, kv_rows = (uint64_t)p.B * p.nkv * p.cap;
+  const uint64_t q_rows = (uint64_t)p.B * p.nh;
+  const uint64_t kv_rows = p.block_table ? (uint64_t)p.num_pages * p.nkv * p.page_size : (uint64_t)p.B * p.nkv * p.cap;
   if (!make_tmap_bf16_2d(&tq, p.q, HD, q_rows, HD * 2, 64, BM)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tk, p.k_cache, HD, kv_rows, HD * 2, 64, BKV)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16_2d(&tv, p.v_cache, HD, kv_rows, HD * 2, 64, BKV)) return cudaErrorInvalidValue;

@@ -483,11 +483,12 @@ def test_decode_long_cache_uses_workspace_splits():
     gate(host(run_decode(q, kc, vc, lens, nh, dtype)), want, dtype, "long-cache decode")
 
 
-def paged_inputs(B, nh, nkv, hd, ps, lens, seed, extra_pages=5):
+def paged_inputs(B, nh, nkv, hd, ps, lens, seed, extra_pages=5, min_cap=0):
     """The seeded contiguous decode cache cut into pages of ``ps`` keys, the
     pages shuffled into a pool with ``extra_pages`` NaN-filled pages that no
-    table names; table entries past a sequence's last page are -1."""
-    cap = -(-max(int(lens.max()), 1) // ps) * ps
+    table names; table entries past a sequence's last page are -1.  The
+    table's width (the logical capacity) covers at least ``min_cap`` keys."""
+    cap = -(-max(int(lens.max()), 1, min_cap) // ps) * ps
     max_pages = cap // ps
     q = W.normal_tensor((B, nh, hd), seed, 0, "bf16")
     kc = nan_padded(B, nkv, cap, hd, lens, seed, 1, "bf16")
@@ -544,15 +545,16 @@ def test_paged_decode_parity(hd, g, nkv, ps):
 @pytest.mark.parametrize("ps", (64, 192))
 def test_paged_decode_keys_as_rows(ps):
     """The keys-as-rows decode (B 32, 32 heads on one KV head, up to 8192
-    keys) over shuffled pages: every 64-key half of a 128-key tile is mapped
-    to its page (a 192-key page holds one and a half tiles); against the
-    oracle's paged decode, and bit for bit against the same keys in a
-    contiguous cache of 20000 slots (long enough that the contiguous call
-    takes the same kernel: only the address of each tile differs)."""
+    keys) over shuffled pages, its table wide enough (20000 keys) that the
+    cluster kernel does not take it: every 64-key half of a 128-key tile is
+    mapped to its page (a 192-key page holds one and a half tiles); against
+    the oracle's paged decode, and bit for bit against the same keys in a
+    contiguous cache of 20000 slots (the same kernel: only the address of
+    each tile differs)."""
     hd, g, nkv, B = 128, 32, 1, 32
     nh = g * nkv
     lens = _hn_lens(B, 8192, 77 + ps, [8192, 0, 1, 64, 127, 128, 129, 191, 192, 193, 5000])
-    q, kc, vc, kp, vp, table, cap = paged_inputs(B, nh, nkv, hd, ps, lens, 90 + ps)
+    q, kc, vc, kp, vp, table, cap = paged_inputs(B, nh, nkv, hd, ps, lens, 90 + ps, min_cap=20000)
     want = ref.paged_decode_attention(q.f64, kp.f64, vp.f64, table, lens, ps)
     gqa.gqa_device_error()
     got_t = run_decode_paged(q, kp, vp, table, lens, nh)
@@ -560,10 +562,47 @@ def test_paged_decode_keys_as_rows(ps):
     assert np.all(got[1] == 0)
     keep = lens > 0
     gate(got[keep], want[keep], "bf16", f"paged keys-as-rows decode ps={ps}")
-    wide = lambda c: W.Tensor(np.pad(c.store, ((0, 0), (0, 0), (0, 20000 - c.store.shape[2]), (0, 0))), "bf16")
-    flat = run_decode(q, wide(kc), wide(vc), lens, nh, "bf16")
+    assert kc.shape[2] >= 20000           # the contiguous copy is as wide as the table
+    flat = run_decode(q, kc, vc, lens, nh, "bf16")
     np.testing.assert_array_equal(bits(got_t), bits(flat))
     assert gqa.gqa_device_error() == 0
+
+
+@pytest.mark.parametrize("hd,ps", [(128, 64), (128, 192), (64, 128)])
+def test_paged_decode_cluster_kernel(hd, ps):
+    """Large paged batches with g > 16 and at most 8 x 2048 keys per
+    sequence take the cluster tcgen05 decode (heads as the MMA rows), with
+    each 64-key tile mapped to its page: against the oracle's paged decode,
+    bit for bit against the same keys in a contiguous cache of the same
+    capacity (the same kernel), and with bad table entries flagged and read
+    as zeros."""
+    g, nkv, B = 32, 1, 32
+    nh = g * nkv
+    lens = _hn_lens(B, 8192, 55 + ps + hd, [8192, 0, 1, 63, 64, 65, 191, 192, 193, 2048, 5000])
+    q, kc, vc, kp, vp, table, cap = paged_inputs(B, nh, nkv, hd, ps, lens, 95 + ps + hd)
+    assert cap <= 8 * 2048
+    want = ref.paged_decode_attention(q.f64, kp.f64, vp.f64, table, lens, ps)
+    gqa.gqa_device_error()
+    got_t = run_decode_paged(q, kp, vp, table, lens, nh)
+    got = host(got_t)
+    assert np.all(got[1] == 0)
+    keep = lens > 0
+    gate(got[keep], want[keep], "bf16", f"paged cluster decode hd={hd} ps={ps}")
+    flat = run_decode(q, kc, vc, lens, nh, "bf16")
+    np.testing.assert_array_equal(bits(got_t), bits(flat))
+    assert gqa.gqa_device_error() == 0
+    # two bad entries: past the pool, and negative, inside the sequences' key ranges
+    n_pool = kp.shape[0]
+    bad = table.copy()
+    bad[0, 3] = n_pool + 11
+    bad[5, 0] = -3
+    got = host(run_decode_paged(q, kp, vp, bad, lens, nh))
+    assert gqa.gqa_device_error() & 8
+    zk = np.concatenate([kp.f64, np.zeros((1,) + kp.shape[1:])])
+    zv = np.concatenate([vp.f64, np.zeros((1,) + vp.shape[1:])])
+    zt = np.where((bad < 0) | (bad >= n_pool), n_pool, bad)
+    want = ref.paged_decode_attention(q.f64, zk, zv, zt, lens, ps)
+    gate(got[keep], want[keep], "bf16", "paged cluster decode, zero-read pages")
 
 
 def test_paged_decode_shared_pages():
