@@ -11,9 +11,11 @@ barriers exist for (TMEM columns and shared-memory stages are reused only
 after their readers finished) and that no schedule deadlocks.
 
 These are models of the protocols, kept next to the sources they restate
-(qkv_tc.cu, prefill_pair.cu, prefill_fa.cu, decode_tc.cu, decode_hn.cu); a
-change to a kernel's waits belongs in both.  The decode's former final waits, which the
-model flags, are kept as a planted mistake.
+(qkv_tc.cu, its K split across a cluster included, prefill_pair.cu,
+prefill_fa.cu, decode_tc.cu, decode_hn.cu); a change to a kernel's waits
+belongs in both.  The decode's former final waits, and a K-split leader that
+reads its partner's partial sums before the cluster barrier, are kept as
+planted mistakes that the model flags.
 """
 import random
 
@@ -156,6 +158,100 @@ def test_qkv_gemm_protocol(n_tiles, n_kb):
                     assert pos[("event", f"acc_read{it}_{w}")] < pos[("event", f"acc_write{it + 2}")]
         for j in range(4, n_tiles * n_kb):
             assert pos[("done", f"mma{j - 4}")] < pos[("issue", f"load_ab{j}")]
+
+
+def qkv_tc_ksplit(n_kb, STAGES=4, warps=4, ks=2, leader_waits=True):
+    """The K split of qkv_tc.cu: the ks CTAs of a cluster each take one
+    tile's k-blocks [r n_kb / ks, (r + 1) n_kb / ks); ranks above 0 write
+    their accumulator rows to their own shared memory, every thread of every
+    rank meets at a cluster barrier, the leader's epilogue warps read those
+    rows, and a second cluster barrier keeps the other ranks alive until then.
+    ``leader_waits=False`` plants the mistake of reading before the first
+    cluster barrier."""
+    n_roles = ks * (2 + warps)
+    bars = {"cluster1": Bar(n_roles), "cluster2": Bar(n_roles)}
+    roles = {}
+    for r in range(ks):
+        kb0, kb1 = r * n_kb // ks, (r + 1) * n_kb // ks
+        bars[f"drain_{r}"] = Bar(1)
+        bars[f"acc_full_{r}"] = Bar(1)
+        for s in range(STAGES):
+            bars[f"ab{r}_full{s}"] = Bar(1)
+            bars[f"ab{r}_empty{s}"] = Bar(1)
+
+        def producer(r=r, kb0=kb0, kb1=kb1):
+            for j in range(kb1 - kb0):
+                yield from ring_load(f"ab{r}", j, STAGES, None)
+            yield ("arrive", "cluster1")
+            yield ("wait", "cluster1", 0)
+            yield ("arrive", "cluster2")
+            yield ("wait", "cluster2", 0)
+
+        def mma(r=r, kb0=kb0, kb1=kb1):
+            for j in range(kb1 - kb0):
+                yield ("wait", f"ab{r}_full{j % STAGES}", j // STAGES)
+                yield ("issue", f"mma{r}_{j}", [f"ab{r}_empty{j % STAGES}"])
+            yield ("issue", f"acc{r}", [f"acc_full_{r}"])
+            yield ("issue", f"drain{r}", [f"drain_{r}"])
+            yield ("wait", f"drain_{r}", 0)
+            yield ("arrive", "cluster1")
+            yield ("wait", "cluster1", 0)
+            yield ("arrive", "cluster2")
+            yield ("wait", "cluster2", 0)
+
+        def epilogue(w, r=r):
+            yield ("wait", f"acc_full_{r}", 0)
+            if r > 0:
+                yield ("event", f"partial_write{r}_{w}")
+            if r == 0 and not leader_waits:
+                for q in range(1, ks):
+                    yield ("event", f"partial_read{q}_{w}")
+            yield ("arrive", "cluster1")
+            yield ("wait", "cluster1", 0)
+            if r == 0:
+                if leader_waits:
+                    for q in range(1, ks):
+                        yield ("event", f"partial_read{q}_{w}")
+                yield ("event", f"tile_epilogue_{w}")
+            yield ("arrive", "cluster2")
+            yield ("wait", "cluster2", 0)
+            yield ("event", f"exit{r}_{w}")
+
+        roles[f"tma{r}"] = producer()
+        roles[f"mma{r}"] = mma()
+        roles.update({f"epi{r}_{w}": epilogue(w) for w in range(warps)})
+    return roles, bars
+
+
+def check_ksplit(pos, ks, warps=4):
+    for q in range(1, ks):
+        for w in range(warps):
+            assert pos[("done", f"acc{q}")] < pos[("event", f"partial_write{q}_{w}")]
+            for w2 in range(warps):
+                # every row of rank q is written before the leader reads any, and read before rank q leaves
+                assert pos[("event", f"partial_write{q}_{w}")] < pos[("event", f"partial_read{q}_{w2}")]
+                assert pos[("event", f"partial_read{q}_{w2}")] < pos[("event", f"exit{q}_{w}")]
+    for w in range(warps):
+        assert pos[("done", "acc0")] < pos[("event", f"tile_epilogue_{w}")]
+
+
+@pytest.mark.parametrize("n_kb,ks", [(8, 2), (9, 2), (12, 3), (16, 4)])
+def test_qkv_gemm_ksplit_protocol(n_kb, ks):
+    for seed in range(60):
+        roles, bars = qkv_tc_ksplit(n_kb, ks=ks)
+        check_ksplit(first(run(roles, bars, seed)), ks)
+
+
+def test_planted_ksplit_read_before_the_cluster_barrier_is_flagged():
+    flagged = False
+    for seed in range(60):
+        roles, bars = qkv_tc_ksplit(8, leader_waits=False)
+        try:
+            check_ksplit(first(run(roles, bars, seed)), 2)
+        except AssertionError:
+            flagged = True
+            break
+    assert flagged
 
 
 # ---------------------------------------------------------------- prefill_pair.cu
