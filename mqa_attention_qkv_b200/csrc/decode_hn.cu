@@ -45,10 +45,9 @@
 // Measured on B200 for the B 64 MQA decode (32 heads, ragged 512..8192 keys,
 // 167 MB of K/V): ~1.5-1.9 us per tile and SM while streaming, ~7 us of
 // launch, prefix sums and first-tile latency, ~4-6 us of partial epilogues
-// and final merges.  That is slower than the cluster kernel on contiguous
-// caches of up to 8 x 2048 keys (54 vs 52 us), so the dispatcher uses this
-// kernel for paged caches and longer caches only (56-59 us with 64-key
-// pages, against 62 us for the mma.sync kernel).
+// and final merges.  That is slower than the cluster kernel on caches of up
+// to 8 x 2048 keys, contiguous or paged (51 against 42 us when the calls run
+// back to back), so the dispatcher uses this kernel for longer caches only.
 #include <atomic>
 #include <cstddef>
 

@@ -13,9 +13,10 @@
 //
 // It serves large batches (the HBM-bound case); small decode steps, which are
 // latency-bound, stay on the mma.sync kernel.  Measured on B200 for B 64,
-// 32 heads, 1 KV head, hd 128, ragged 512..8192 keys: this kernel 51 us, the
-// mma.sync kernel 60 us, and this kernel with fixed 1024- or 2048-key splits
-// merged through a workspace instead of a cluster 63 / 55 us.
+// 32 heads, 1 KV head, hd 128, ragged 512..8192 keys, one call between two
+// events: this kernel 51 us (42 us per call back to back), the mma.sync
+// kernel 60 us, and this kernel with fixed 1024- or 2048-key splits merged
+// through a workspace instead of a cluster 63 / 55 us.
 // The cache is contiguous or paged: with a block table every 64-key tile is
 // mapped to its page (pages hold a multiple of 64 keys, so a tile never
 // crosses one), an entry outside the page pool is flagged and read as zeros.
